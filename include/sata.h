@@ -1,0 +1,196 @@
+/*
+ * sata.h - C ABI of libsata: causal symmetry-aware Taylor (SATA) attention on
+ * NVIDIA B200 (sm_100a).
+ *
+ * The method (sources cited by page title and section):
+ *   [CC-TAYLOR] "Self-attention at constant cost per token via symmetry-aware
+ *               Taylor approximation" (blog.hotdry.top, 2026-02-05)
+ *   [CC-HW]     "Constant-cost attention: hardware optimization" (same blog)
+ *
+ *   exp(q.k / c) ~= sum_{p=0}^{P-1} alpha_p <phi_p(q), phi_p(k)>_{C_p},
+ *   alpha_p = 1 / (p! c^p),  c = sqrt(d_K)          ([CC-TAYLOR] "The Taylor
+ *                                                     approximation", "Feature
+ *                                                     maps and linear attention")
+ *   phi_p(x)[r] = prod_m x[M_p[r][m]] over the nondecreasing index tuples M_p,
+ *   C_p[r] = number of times tuple r's monomial occurs in (q.k)^p.
+ *   Z_p = sum_t phi_p(k_t),  S_p = sum_t phi_p(k_t) v_t^T            (states)
+ *   y_T = sum_p alpha_p phi_p(q_T)^T C_p S_p / sum_p alpha_p <phi_p(q_T), Z_p>_C
+ *                                            ([CC-TAYLOR] "Feature maps and
+ *                                             linear attention")
+ *
+ * Conventions shared by every entry point:
+ *   - P is the number of Taylor terms (degrees 0..P-1).  F = binom(d_K+P-1, P-1)
+ *     features per head, concatenated p = 0..P-1, lexicographic within a degree.
+ *   - The causal range is inclusive: token t's output sees tokens 0..t; a decode
+ *     step adds (k, v) to the state before reading it.
+ *   - Attention inputs q, k, v are bf16, row-major [B][H][N][d] (prefill) or
+ *     [B][H][d] (decode); outputs are fp32 [B][H][N][d_V] / [B][H][d_V].
+ *   - The state is fp32, unweighted (alpha_p and C_p are applied on the query
+ *     side): S [B][H][F][d_V], Z [B][H][F], features in the order above.
+ *   - All device pointers must be 16-byte aligned.  Buffers are owned by the
+ *     caller; the library owns only its cached basis tables and internal
+ *     workspaces (freed by sata_shutdown).
+ *   - Every call returns SATA_OK (0) or a negative status; none throws.  Work is
+ *     enqueued asynchronously on a CUDA stream; argument checks happen before any
+ *     launch.  Launch failures return SATA_ECUDA (sata_last_cuda_error() gives
+ *     the cudaError_t).  Device-side conditions (a bounded wait that gave up, an
+ *     input outside the prefill's operand range) set a per-device flag that
+ *     sata_sync_status() reports.
+ *   - Supported: 1 <= d_K <= 128, d_V in {4, 8, 16, 32, 64, 128}, 1 <= P <= 4.
+ *     Other values return SATA_EUNSUPPORTED.  There is no CPU fallback.
+ *   - The library-owned workspaces are shared by all calls on a device: calls
+ *     that may overlap on different streams must pass their own workspace
+ *     (sata_prefill_ex) or be ordered by the caller.
+ *   - The first call for a given (device, d_K, P) uploads the basis tables with
+ *     synchronous copies; make it before capturing a CUDA graph.
+ */
+#ifndef SATA_H
+#define SATA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define SATA_API __attribute__((visibility("default")))
+#else
+#define SATA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+enum sata_status {
+    SATA_OK = 0,
+    SATA_EINVAL = -1,        /* invalid argument (null, negative size, state mismatch) */
+    SATA_EUNSUPPORTED = -2,  /* valid, but d_K / d_V / P outside the supported set */
+    SATA_ECUDA = -3,         /* CUDA runtime or launch error; see sata_last_cuda_error() */
+    SATA_ETIMEOUT = -4,      /* a bounded device-side wait expired (reported at sync) */
+    SATA_ENOMEM = -5,        /* internal workspace allocation failed, or too small */
+    SATA_ERANGE = -6,        /* inputs exceed the prefill's fp16 operand range (at sync) */
+    SATA_EALIGN = -7         /* a device pointer is not 16-byte aligned */
+};
+
+/* Per-sequence recurrent state: caller-allocated struct and device buffers. */
+typedef struct sata_state {
+    int32_t B, H, d_K, d_V, P;
+    int64_t F;        /* features per head */
+    float *S;         /* device [B][H][F][d_V] fp32 */
+    float *Z;         /* device [B][H][F] fp32 */
+    void *stream;     /* cudaStream_t used by sata_decode_step (NULL: legacy stream) */
+    int64_t tokens;   /* tokens absorbed so far (prefill + decode) */
+} sata_state;
+
+/* Human-readable name of a status code (static string). */
+SATA_API const char *sata_status_string(int status);
+/* cudaError_t of the last failed CUDA call made by this library on this thread. */
+SATA_API int sata_last_cuda_error(void);
+/* Library version: major * 10000 + minor * 100 + patch. */
+SATA_API int sata_version(void);
+
+/* F = binom(d_K+P-1, P-1): number of features of the truncated basis
+ * ([CC-TAYLOR] "Hidden-state size and FLOPs").  Host only. */
+SATA_API int sata_num_features(int d_K, int P, int64_t *F_out);
+
+/*
+ * Minimal symmetric basis ([CC-TAYLOR] "The Taylor approximation": keep one
+ * representative of each monomial, the upper-triangular / nondecreasing index
+ * tuples, binom(d_K+p-1, p) of them; "Feature maps and linear attention": C_p
+ * counts each monomial's occurrences; [CC-HW] "Compute density":
+ * phi = x[..., M].prod(-1)).  Host only, deterministic, bit-exact.
+ *   M       [F][max(P-1,1)] uint8: row r holds the p indices of feature r
+ *           (nondecreasing) followed by 0xFF padding; NULL to skip.
+ *   C       [F] uint32 multiplicities p!/prod(mult!); NULL to skip.
+ *   offsets [P+1]: first feature of degree p, offsets[P] = F; NULL to skip.
+ *   F_out   receives F; NULL to skip.  All NULL: size query.
+ * Requires d_K <= 255 (indices fit a byte).
+ */
+SATA_API int sata_build_basis(int d_K, int P, uint8_t *M, uint32_t *C, int64_t *offsets, int64_t *F_out);
+
+/* Stream used by sata_prefill (the plain form); default: the legacy stream.
+ * Process-wide; set it before launching from another stream. */
+SATA_API int sata_set_stream(void *stream);
+
+/* Synchronise `stream` and report device-side conditions raised since the last
+ * call on this device: SATA_ETIMEOUT, SATA_ERANGE, or SATA_OK.  Clears them. */
+SATA_API int sata_sync_status(void *stream);
+
+/* Free the library's cached device tables and workspaces on every device. */
+SATA_API void sata_shutdown(void);
+
+/* Bytes of S and Z for a state of this shape ([CC-TAYLOR] "Hidden-state size
+ * and FLOPs": (d_V + 1) binom(d_K+P-1, P-1) values per head). */
+SATA_API int sata_state_bytes(int B, int H, int d_K, int d_V, int P, size_t *S_bytes, size_t *Z_bytes);
+
+/* Fill *st for caller-owned device buffers S, Z (sizes from sata_state_bytes)
+ * and zero them on `stream` (an empty context).  tokens = 0. */
+SATA_API int sata_state_init(sata_state *st, int B, int H, int d_K, int d_V, int P,
+                    float *S, float *Z, void *stream);
+
+/* Workspace bytes sata_prefill_ex needs for this shape. */
+SATA_API int sata_workspace_bytes(int B, int H, int64_t N, int d_K, int d_V, int P, size_t *bytes);
+
+/*
+ * Causal SATA prefill over N tokens of B*H independent heads, fresh (zero)
+ * state, on the stream set by sata_set_stream, library-owned workspace.
+ *   q, k: bf16 [B][H][N][d_K];  v: bf16 [B][H][N][d_V];  out: fp32 [B][H][N][d_V].
+ * Output y_t for every token: the chunked form of the state recurrence
+ * ([CC-TAYLOR] "Feature maps and linear attention": the recurrence may be
+ * evaluated sequentially or as a parallel prefix scan).  N = 0 is a no-op.
+ */
+SATA_API int sata_prefill(const void *q, const void *k, const void *v, float *out,
+                 int B, int H, int64_t N, int d_K, int d_V, int P);
+
+/*
+ * As sata_prefill, with explicit state, workspace and stream.
+ *   st:        NULL (fresh state, final state discarded) or a state of the same
+ *              (B, H, d_K, d_V, P): the prefill continues from it and leaves the
+ *              final state there; st->tokens += N.
+ *   workspace: NULL (library-owned) or a device buffer of ws_bytes >=
+ *              sata_workspace_bytes(...), used only while the enqueued work runs.
+ *   stream:    cudaStream_t (NULL: legacy stream).
+ */
+SATA_API int sata_prefill_ex(const void *q, const void *k, const void *v, float *out,
+                    int B, int H, int64_t N, int d_K, int d_V, int P,
+                    sata_state *st, void *workspace, size_t ws_bytes, void *stream);
+
+/*
+ * One decode step for every head of `st`, on st->stream: the state absorbs
+ * (k, v) and the output is read with q ([CC-TAYLOR] "Feature maps and linear
+ * attention": Z_T = Z_{T-1} + phi(k_T), S_T = S_{T-1} + phi(k_T) v_T^T, then
+ * y_T; [CC-HW] "Fixed-size hidden state": constant cost per token).
+ *   q, k: bf16 [B][H][d_K];  v: bf16 [B][H][d_V];  out: fp32 [B][H][d_V].
+ * The state streams through HBM once (read and write).  st->tokens += 1.
+ */
+SATA_API int sata_decode_step(sata_state *st, const void *q, const void *k, const void *v, float *out);
+
+/* Tuning and test options (process-wide).  Keys: */
+enum sata_option {
+    SATA_OPT_PREFILL_PATH = 1,   /* 0 auto, 1 CUDA-core path, 2 tensor-core path */
+    SATA_OPT_WAIT_LIMIT = 2,     /* bounded-wait iteration limit (0 = default) */
+    SATA_OPT_TEST_STALL = 3,     /* 1: the next tensor-core prefill launch withholds
+                                    one producer signal, so its bounded wait expires
+                                    (tests the SATA_ETIMEOUT path); auto-resets */
+    SATA_OPT_TIME_KERNELS = 4    /* 1: bracket every kernel launch with CUDA events on
+                                    its own stream (read with sata_kernel_stats) */
+};
+SATA_API int sata_set_option(int key, int64_t value);
+SATA_API int sata_get_option(int key, int64_t *value);
+
+/* Per-kernel launch statistics since the last reset: launches are always
+ * counted; device time (ms, from the events) only while SATA_OPT_TIME_KERNELS
+ * is on.  Reading synchronises the recorded events.  Entries: one per kernel
+ * that launched at least once; *n_out receives the count (<= max_entries). */
+typedef struct sata_kernel_stat {
+    char name[40];
+    int64_t launches;
+    double ms;
+} sata_kernel_stat;
+SATA_API int sata_kernel_stats(sata_kernel_stat *out, int max_entries, int *n_out);
+SATA_API int sata_reset_kernel_stats(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SATA_H */

@@ -1,0 +1,91 @@
+// Internal declarations shared by the libsata translation units.
+#pragma once
+
+#include <cstdint>
+#include <vector>
+
+#include <cuda_runtime.h>
+
+#include "sata.h"
+
+namespace sata {
+
+constexpr int kMaxDK = 128;
+constexpr int kMaxDV = 128;
+constexpr int kMaxP = 4;      // degrees 0..3: packed tables hold three indices
+
+// Host copy of the basis (sata_build_basis serves from it).
+struct HostBasis {
+    int d_K = 0, P = 0;
+    std::vector<std::vector<uint8_t>> tuples;  // [F] nondecreasing indices
+    std::vector<uint8_t> degree;               // [F]
+    std::vector<uint32_t> mult;                // [F] C_p
+    std::vector<int64_t> offsets;              // [P+1]
+};
+
+int64_t binom64(int n, int k);
+int64_t num_features(int d_K, int P);
+bool build_basis_host(int d_K, int P, HostBasis &hb);
+
+// Device copy of the basis for the kernels, cached per (device, d_K, P).
+//   packed[f] = a | b << 8 | l << 16 | p << 24: feature f is x[a] * x[b] * x[l]
+//   where index d_K stands for the constant 1 (degree-p tuples are left-padded
+//   with it, so every feature is a "prefix pair (a, b) times a last index l").
+//   coef[f]  = alpha_p * C_p[f] = C_p[f] / (p! c^p), c = sqrt(d_K)  (fp32)
+//   mcoef[f] = C_p[f] / p! = 1 / prod(mult!)                     (fp32)
+struct DeviceBasis {
+    int d_K = 0, P = 0;
+    int64_t F = 0;
+    int64_t offsets[kMaxP + 1] = {0, 0, 0, 0, 0};
+    uint32_t *packed = nullptr;
+    float *coef = nullptr;
+    float *mcoef = nullptr;
+};
+
+// Device-side status words, one set per device: [0] timeout, [1] range.
+enum { kFlagTimeout = 0, kFlagRange = 1, kNumFlags = 4 };
+
+// Library-owned per-device resources (basis cache, status flags, workspaces).
+const DeviceBasis *device_basis(int d_K, int P, cudaError_t *err);
+int *device_flags(cudaError_t *err);
+void *device_workspace(int slot, size_t bytes, cudaError_t *err);
+
+// Kernel identities for launch statistics.
+enum KernelId {
+    kDecodeStream = 0, kDecodeFinish, kSimtScan, kSimtFinish, kTcPrep, kTcScan, kTcFinish,
+    kNumKernels
+};
+const char *kernel_name(int id);
+// Call around every kernel launch: begin() records a start event when timing is
+// on, end() records the stop event and counts the launch.
+void launch_begin(int id, cudaStream_t s);
+void launch_end(int id, cudaStream_t s);
+
+// Runtime options.
+extern int64_t g_opt_prefill_path;
+extern int64_t g_opt_wait_limit;
+extern int64_t g_opt_test_stall;
+extern int64_t g_opt_time_kernels;
+
+// ---- decode (decode.cu) ----
+size_t decode_workspace_bytes(int BH, int64_t F, int d_V);
+cudaError_t launch_decode(const DeviceBasis &basis, int BH, int d_V, float *S, float *Z,
+                          const void *q, const void *k, const void *v, float *out,
+                          float *partials, cudaStream_t stream);
+
+// ---- prefill, CUDA-core path (prefill_simt.cu) ----
+size_t prefill_simt_workspace_bytes(int BH, int64_t N, int64_t F, int d_V, bool need_state);
+cudaError_t launch_prefill_simt(const DeviceBasis &basis, int BH, int64_t N, int d_V,
+                                const void *q, const void *k, const void *v, float *out,
+                                float *S, float *Z, bool state_in, void *ws, size_t ws_bytes,
+                                cudaStream_t stream);
+
+// ---- prefill, tensor-core path (prefill_tc.cu) ----
+bool prefill_tc_supported(int d_K, int d_V, int P);
+size_t prefill_tc_workspace_bytes(int BH, int64_t N, int64_t F, int d_K, int d_V, bool need_state);
+cudaError_t launch_prefill_tc(const DeviceBasis &basis, int BH, int64_t N, int d_V,
+                              const void *q, const void *k, const void *v, float *out,
+                              float *S, float *Z, bool state_in, void *ws, size_t ws_bytes,
+                              int *flags, cudaStream_t stream);
+
+}  // namespace sata

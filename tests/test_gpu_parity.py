@@ -1,0 +1,201 @@
+"""GPU parity: libsata (through the C ABI) against the float64 oracle.
+
+Every case feeds both sides the same seeded bf16 inputs (the oracle widens
+them to float64) and gates the per-token normwise error at parity.TOL.
+Small cases cover every token and span several feature tiles, several chunks
+and a ragged tail; the full-size workloads are checked on the heads and
+token ranges the oracle can finish in seconds.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from symmetric_taylor_self_b200 import workloads as wl
+from tests.parity import TOL, token_rel_err
+
+pytestmark = pytest.mark.gpu
+
+PATHS = {"cuda_core": 1, "auto": 0}
+
+
+@pytest.fixture(scope="module")
+def sata():
+    from symmetric_taylor_self_b200 import build as b
+    b.build()
+    import symmetric_taylor_self_b200 as s
+    s.load()
+    assert torch.cuda.is_available()
+    yield s
+    s.sata_set_option(s.SATA_OPT_PREFILL_PATH, 0)
+
+
+def _set_path(sata, path):
+    sata.sata_set_option(sata.SATA_OPT_PREFILL_PATH, PATHS[path])
+
+
+def _oracle_heads(oracle_mod, q, k, v, P, heads, T=None):
+    return oracle_mod.prefill(q, k, v, P, heads=heads, T=T)
+
+
+def _check_heads(y_gpu, ref, T=None, what=""):
+    for (b, h), (y, den, S, Z) in ref.items():
+        yy = y_gpu[b, h, : (T or y.shape[0])].double().cpu().numpy()
+        err, excl, tens = token_rel_err(yy, y)
+        assert err <= TOL, f"{what} head {(b, h)}: max per-token rel err {err:.3e} > {TOL}"
+        assert excl == 0
+
+
+@pytest.mark.parametrize("path", list(PATHS))
+@pytest.mark.parametrize("d,N", [(8, 1), (8, 33), (8, 300), (16, 127), (16, 129), (32, 1),
+                                 (32, 257), (64, 31), (64, 129)])
+def test_prefill_small_ragged(sata, oracle_mod, path, d, N):
+    _set_path(sata, path)
+    q, k, v = wl.random_inputs(1, 2, N, d, d, seed=1000 + d * 7 + N)
+    y = sata.prefill(q.cuda(), k.cuda(), v.cuda(), P=4)
+    torch.cuda.synchronize()
+    assert sata.sata_sync_status() == 0
+    ref = _oracle_heads(oracle_mod, q, k, v, 4, [(0, 0), (0, 1)])
+    _check_heads(y, ref, what=f"d={d} N={N}")
+
+
+@pytest.mark.parametrize("P", [1, 2, 3])
+def test_prefill_lower_P(sata, oracle_mod, P):
+    _set_path(sata, "auto")
+    q, k, v = wl.random_inputs(1, 1, 100, 16, 16, seed=50 + P)
+    y = sata.prefill(q.cuda(), k.cuda(), v.cuda(), P=P)
+    ref = _oracle_heads(oracle_mod, q, k, v, P, [(0, 0)])
+    _check_heads(y, ref, what=f"P={P}")
+
+
+@pytest.mark.parametrize("name", ["tiny_d8", "prefill_d16"])
+def test_prefill_workload_all_heads(sata, oracle_mod, name):
+    _set_path(sata, "auto")
+    w = wl.WORKLOADS[name]
+    (q, k, v), _ = wl.make_inputs(w)
+    y = sata.prefill(q.cuda(), k.cuda(), v.cuda(), P=w.P)
+    ref = _oracle_heads(oracle_mod, q, k, v, w.P, list(w.oracle_heads))
+    _check_heads(y, ref, what=name)
+
+
+def test_prefill_workload_d32(sata, oracle_mod):
+    _set_path(sata, "auto")
+    w = wl.WORKLOADS["prefill_d32"]
+    (q, k, v), _ = wl.make_inputs(w)
+    y = sata.prefill(q.cuda(), k.cuda(), v.cuda(), P=w.P)
+    ref = _oracle_heads(oracle_mod, q, k, v, w.P, list(w.oracle_heads))
+    _check_heads(y, ref, what="prefill_d32 full heads")
+    allh = [(b, h) for b in range(w.B) for h in range(w.H)]
+    ref = _oracle_heads(oracle_mod, q, k, v, w.P, allh, T=1024)
+    _check_heads(y, ref, T=1024, what="prefill_d32 all heads t<1024")
+
+
+def test_prefill_workload_d64(sata, oracle_mod):
+    _set_path(sata, "auto")
+    w = wl.WORKLOADS["prefill_d64"]
+    (q, k, v), _ = wl.make_inputs(w)
+    y = sata.prefill(q.cuda(), k.cuda(), v.cuda(), P=w.P)
+    ref = _oracle_heads(oracle_mod, q, k, v, w.P, list(w.oracle_heads), T=w.oracle_tokens)
+    _check_heads(y, ref, T=w.oracle_tokens, what="prefill_d64 head 0, first 2048 tokens")
+    # every head: outputs are finite and the last tokens are convex-ish averages of v
+    assert torch.isfinite(y).all()
+
+
+def test_decode_workload(sata, oracle_mod):
+    """8192-token prefill into a state, then 1024 decode steps; four heads are
+    followed by the oracle through all 9216 tokens."""
+    _set_path(sata, "auto")
+    w = wl.WORKLOADS["decode_d32"]
+    (q, k, v), (qs, ks, vs) = wl.make_inputs(w)
+    st = sata.State(w.B, w.H, w.d_K, w.d_V, w.P)
+    y = sata.prefill(q.cuda(), k.cuda(), v.cuda(), P=w.P, state=st)
+    qs, ks, vs = qs.cuda(), ks.cuda(), vs.cuda()
+    outs = torch.empty((w.steps, w.B, w.H, w.d_V), dtype=torch.float32, device="cuda")
+    for i in range(w.steps):
+        sata.decode_step(st, qs[i], ks[i], vs[i], out=outs[i])
+    torch.cuda.synchronize()
+    assert st.tokens == w.N + w.steps
+    heads = list(w.oracle_heads)
+    qf = torch.cat([q, qs.cpu().permute(1, 2, 0, 3)], dim=2)
+    kf = torch.cat([k, ks.cpu().permute(1, 2, 0, 3)], dim=2)
+    vf = torch.cat([v, vs.cpu().permute(1, 2, 0, 3)], dim=2)
+    ref = oracle_mod.prefill(qf, kf, vf, w.P, heads=heads)
+    for (b, h), (yr, den, S, Z) in ref.items():
+        err, _, _ = token_rel_err(y[b, h].cpu().numpy(), yr[: w.N])
+        assert err <= TOL, f"prefill part of head {(b, h)}: {err:.3e}"
+        err, _, _ = token_rel_err(outs[:, b, h].cpu().numpy(), yr[w.N:])
+        assert err <= TOL, f"decode part of head {(b, h)}: {err:.3e}"
+        Sg = st.S[b, h].double().cpu().numpy()
+        Zg = st.Z[b, h].double().cpu().numpy()
+        assert np.abs(Sg - S).max() / np.abs(S).max() <= TOL
+        assert np.abs(Zg - Z).max() / np.abs(Z).max() <= TOL
+
+
+@pytest.mark.parametrize("path", list(PATHS))
+def test_state_output_and_continuation(sata, oracle_mod, path):
+    """prefill(N) == prefill(N - m) then prefill(m) from the state == prefill(N - m)
+    then m decode steps; the final state matches the oracle's."""
+    _set_path(sata, path)
+    B, H, N, d, m = 2, 3, 200, 16, 37
+    q, k, v = wl.random_inputs(B, H, N, d, d, seed=77)
+    qc, kc, vc = q.cuda(), k.cuda(), v.cuda()
+    y_full = sata.prefill(qc, kc, vc, P=4)
+    st = sata.State(B, H, d, d, 4)
+    y_a = sata.prefill(qc[:, :, : N - m].contiguous(), kc[:, :, : N - m].contiguous(),
+                       vc[:, :, : N - m].contiguous(), P=4, state=st)
+    st2 = sata.State(B, H, d, d, 4)
+    st2.S.copy_(st.S)
+    st2.Z.copy_(st.Z)
+    st2.st.tokens = st.tokens
+    y_b = sata.prefill(qc[:, :, N - m:].contiguous(), kc[:, :, N - m:].contiguous(),
+                       vc[:, :, N - m:].contiguous(), P=4, state=st)
+    dec = [sata.decode_step(st2, qc[:, :, t].contiguous(), kc[:, :, t].contiguous(),
+                            vc[:, :, t].contiguous()) for t in range(N - m, N)]
+    torch.cuda.synchronize()
+    y_seg = torch.cat([y_a, y_b], dim=2)
+    y_dec = torch.cat([y_a, torch.stack(dec, dim=2)], dim=2)
+    ref = oracle_mod.prefill(q, k, v, 4)
+    for (b, h), (yr, den, S, Z) in ref.items():
+        for name, yy in (("one call", y_full), ("two calls", y_seg), ("decode", y_dec)):
+            err, _, _ = token_rel_err(yy[b, h].cpu().numpy(), yr)
+            assert err <= TOL, f"{name} head {(b, h)}: {err:.3e}"
+        for stt in (st, st2):
+            Sg, Zg = stt.S[b, h].double().cpu().numpy(), stt.Z[b, h].double().cpu().numpy()
+            assert np.abs(Sg - S).max() / np.abs(S).max() <= TOL
+            assert np.abs(Zg - Z).max() / np.abs(Z).max() <= TOL
+    assert st.tokens == N and st2.tokens == N
+
+
+@pytest.mark.parametrize("path", list(PATHS))
+def test_deterministic(sata, path):
+    _set_path(sata, path)
+    q, k, v = wl.random_inputs(1, 4, 333, 32, 32, seed=5)
+    qc, kc, vc = q.cuda(), k.cuda(), v.cuda()
+    a = sata.prefill(qc, kc, vc, P=4)
+    b = sata.prefill(qc, kc, vc, P=4)
+    assert torch.equal(a, b)
+
+
+def test_empty_inputs_are_noops(sata):
+    x = torch.empty((1, 2, 0, 16), dtype=torch.bfloat16, device="cuda")
+    y = sata.prefill(x, x, x, P=4)
+    assert y.shape == (1, 2, 0, 16)
+    x = torch.empty((0, 2, 5, 16), dtype=torch.bfloat16, device="cuda")
+    assert sata.prefill(x, x, x, P=4).shape == (0, 2, 5, 16)
+    assert sata.sata_sync_status() == 0
+
+
+def test_decode_small_against_oracle(sata, oracle_mod):
+    """Decode from an empty state for every supported d_V, all heads."""
+    for d in (4, 8, 16, 64, 128):
+        B, H, T = 1, 2, 5
+        q, k, v = wl.random_inputs(B, H, T, d, d, seed=900 + d)
+        st = sata.State(B, H, d, d, 4)
+        outs = [sata.decode_step(st, q[:, :, t].contiguous().cuda(), k[:, :, t].contiguous().cuda(),
+                                 v[:, :, t].contiguous().cuda()) for t in range(T)]
+        torch.cuda.synchronize()
+        yg = torch.stack(outs, dim=2).cpu().numpy()
+        for (b, h), (yr, _, _, _) in oracle_mod.prefill(q, k, v, 4).items():
+            err, _, _ = token_rel_err(yg[b, h], yr)
+            assert err <= TOL, f"d={d}: {err:.3e}"
