@@ -17,7 +17,7 @@ from tests.parity import TOL, token_rel_err
 
 pytestmark = pytest.mark.gpu
 
-PATHS = {"cuda_core": 1, "auto": 0}
+PATHS = {"cuda_core": 1, "auto": 0}     # auto: tensor cores for d_K = d_V in {16, 32, 64}
 
 
 @pytest.fixture(scope="module")
@@ -199,3 +199,61 @@ def test_decode_small_against_oracle(sata, oracle_mod):
         for (b, h), (yr, _, _, _) in oracle_mod.prefill(q, k, v, 4).items():
             err, _, _ = token_rel_err(yg[b, h], yr)
             assert err <= TOL, f"d={d}: {err:.3e}"
+
+
+@pytest.mark.parametrize("d", [16, 32, 64])
+def test_tensor_core_path_selected_and_multi_segment_state(sata, oracle_mod, d):
+    """The tensor-core path serves d in {16, 32, 64}; a state carried in from a
+    previous call is honoured."""
+    sata.sata_set_option(sata.SATA_OPT_PREFILL_PATH, 2)
+    B, H, N = 1, 2, 300
+    q, k, v = wl.random_inputs(B, H, N, d, d, seed=31 + d)
+    qc, kc, vc = q.cuda(), k.cuda(), v.cuda()
+    sata.sata_reset_kernel_stats()
+    st = sata.State(B, H, d, d, 4)
+    y1 = sata.prefill(qc[:, :, :170].contiguous(), kc[:, :, :170].contiguous(), vc[:, :, :170].contiguous(),
+                      P=4, state=st)
+    y2 = sata.prefill(qc[:, :, 170:].contiguous(), kc[:, :, 170:].contiguous(), vc[:, :, 170:].contiguous(),
+                      P=4, state=st)
+    torch.cuda.synchronize()
+    assert sata.sata_sync_status() == 0
+    stats = sata.sata_kernel_stats()
+    assert stats.get("tc_scan", (0, 0))[0] >= 2
+    y = torch.cat([y1, y2], dim=2)
+    for (b, h), (yr, _, S, Z) in oracle_mod.prefill(q, k, v, 4).items():
+        err, _, _ = token_rel_err(y[b, h].cpu().numpy(), yr)
+        assert err <= TOL, f"d={d} head {h}: {err:.3e}"
+        assert np.abs(st.S[b, h].double().cpu().numpy() - S).max() / np.abs(S).max() <= TOL
+    sata.sata_set_option(sata.SATA_OPT_PREFILL_PATH, 0)
+
+
+def test_bounded_wait_reports_timeout(sata):
+    """A producer signal withheld on purpose: every wait gives up after the
+    limit, the kernel exits cleanly, and the status comes back as SATA_ETIMEOUT;
+    the next call runs normally."""
+    sata.sata_set_option(sata.SATA_OPT_PREFILL_PATH, 2)
+    sata.sata_set_option(sata.SATA_OPT_WAIT_LIMIT, 50_000_000)      # 50 ms
+    q, k, v = wl.random_inputs(1, 1, 512, 16, 16, seed=8)
+    qc, kc, vc = q.cuda(), k.cuda(), v.cuda()
+    assert sata.sata_sync_status() == 0
+    sata.sata_set_option(sata.SATA_OPT_TEST_STALL, 1)
+    sata.prefill(qc, kc, vc, P=4)
+    assert sata.sata_sync_status() == sata.SATA_ETIMEOUT
+    assert sata.sata_get_option(sata.SATA_OPT_TEST_STALL) == 0
+    sata.sata_set_option(sata.SATA_OPT_WAIT_LIMIT, 0)
+    a = sata.prefill(qc, kc, vc, P=4)
+    assert sata.sata_sync_status() == 0
+    b = sata.prefill(qc, kc, vc, P=4)
+    assert torch.equal(a, b)
+    sata.sata_set_option(sata.SATA_OPT_PREFILL_PATH, 0)
+
+
+def test_out_of_range_inputs_are_reported(sata):
+    sata.sata_set_option(sata.SATA_OPT_PREFILL_PATH, 2)
+    q, k, v = wl.random_inputs(1, 1, 64, 32, 32, seed=9, scale=100.0)
+    sata.prefill(q.cuda(), k.cuda(), v.cuda(), P=4)
+    assert sata.sata_sync_status() == sata.SATA_ERANGE
+    q, k, v = wl.random_inputs(1, 1, 64, 32, 32, seed=9)
+    sata.prefill(q.cuda(), k.cuda(), v.cuda(), P=4)
+    assert sata.sata_sync_status() == 0
+    sata.sata_set_option(sata.SATA_OPT_PREFILL_PATH, 0)
