@@ -117,6 +117,18 @@ __device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
         : "memory");
     return ok != 0;
 }
+// try_wait with a suspend-time hint: the thread sleeps in hardware until the
+// phase completes or the hint (ns) elapses, instead of spinning.
+__device__ __forceinline__ bool mbar_try_sleep(uint32_t bar, uint32_t parity, uint32_t hint_ns) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}\n"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity), "r"(hint_ns)
+        : "memory");
+    return ok != 0;
+}
 __device__ __forceinline__ int64_t gtimer() {
     uint64_t t;
     asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
@@ -200,7 +212,7 @@ struct Waiter {
         if (mbar_try(bar, parity)) return true;
         const int64_t t0 = gtimer();
         while (true) {
-            if (mbar_try(bar, parity)) return true;
+            if (mbar_try_sleep(bar, parity, 100000u)) return true;
             if (*abort_flag) return false;
             if (gtimer() - t0 > limit) {
                 *abort_flag = 1;
@@ -212,7 +224,7 @@ struct Waiter {
     // Bounded wait that ignores the abort flag (draining in-flight async work).
     __device__ __forceinline__ bool drain(uint32_t bar, uint32_t parity) const {
         const int64_t t0 = gtimer();
-        while (!mbar_try(bar, parity)) {
+        while (!mbar_try_sleep(bar, parity, 100000u)) {
             if (gtimer() - t0 > limit) {
                 atomicExch(gflag, 1);
                 return false;
@@ -596,13 +608,17 @@ __global__ void __launch_bounds__(kScanThreads, 1) tc_scan_kernel(const ScanPara
                     if (!(ok = W.wait(BAR(C::B_AE + s), ((seq / kNS) & 1) ^ 1))) break;
                     uint8_t *stage = smem + C::OFF_RING + s * kStageBytes + hoff;
                     const uint8_t *x = side ? xk : xq;
-                    const uint32_t *tj = tab + j * 128 + fgrp * 8;
-                    const __half *mj = mc + j * 128 + fgrp * 8;
+                    const uint4 *tj4 = reinterpret_cast<const uint4 *>(tab + j * 128 + fgrp * 8);
+                    const uint4 t_lo = tj4[0], t_hi = tj4[1];
+                    const uint32_t tw[8] = {t_lo.x, t_lo.y, t_lo.z, t_lo.w, t_hi.x, t_hi.y, t_hi.z, t_hi.w};
+                    __align__(16) __half mj[8];
+                    if (side == 0)
+                        *reinterpret_cast<uint4 *>(mj) = *reinterpret_cast<const uint4 *>(mc + j * 128 + fgrp * 8);
                     uint32_t prev = 0xFFFFFFFFu;
                     uint4 pre = make_uint4(0, 0, 0, 0);
 #pragma unroll
                     for (int i = 0; i < 8; ++i) {
-                        const uint32_t w = tj[i];
+                        const uint32_t w = tw[i];
                         if ((w & 0xFFFFu) != prev) {   // new prefix pair (a, b)
                             prev = w & 0xFFFFu;
                             const uint4 xa = *reinterpret_cast<const uint4 *>(x + (w & 255u) * C::ROW + xoff);
@@ -637,24 +653,52 @@ __global__ void __launch_bounds__(kScanThreads, 1) tc_scan_kernel(const ScanPara
 
 // Per (head, chunk): sum the feature tiles' inter-chunk partials, add the
 // intra-chunk block sum_{s<=t} w_ts [v_s | 1] (fp32 from the bf16 inputs) and
-// divide.
+// divide.  Partial sums stream with float4 loads, several in flight per thread.
 template <int DK, int DV>
 __global__ void __launch_bounds__(256)
 tc_finish_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k,
                  const __nv_bfloat16 *__restrict__ v, const float *__restrict__ part,
                  float *__restrict__ out, int BH, int G, int c0, int nc, int64_t N, int P, float inv_c) {
-    constexpr int KP = DK + 1, WP = kL + 1, VP = DV + 1, HALF = (DV + 2) / 2;
+    constexpr int VP = DV + 1, WP = kL + 1, HW = DV / 2;
+    constexpr int ITEMS = VP * (kL / 4);            // float4 items of one chunk's partial
+    constexpr int PER = (ITEMS + 255) / 256;
     extern __shared__ float fsm[];
-    float *fq = fsm;               // [128][KP]   (later: fv [128][VP], then staging)
-    float *fk = fq + kL * KP;      // [128][KP]
-    float *Wt = fk + kL * KP;      // [128][WP]
-    __shared__ float den[kL];
+    float *Ps = fsm;                 // [VP][128]  summed partials (col-major by token)
+    float *fqT = Ps + VP * kL;       // [DK][128]  q^T  (later: staging [128][DV])
+    float *fkT = fqT + DK * kL;      // [DK][128]  k^T  (later: v [128][DV])
+    float *Wt = fkT + DK * kL;       // [128][WP]
     const int tid = threadIdx.x;
+    const float4 *p4 = reinterpret_cast<const float4 *>(part);
     for (int64_t idx = blockIdx.x; idx < (int64_t)BH * nc; idx += gridDim.x) {
         const int64_t bh = idx / nc;
         const int cl = (int)(idx % nc);
         const int64_t t0 = (int64_t)(c0 + cl) * kL;
         const int nt = (int)(N - t0 < kL ? N - t0 : kL);
+        // (1) sum over the G feature-tile groups
+        {
+            const int64_t gstride = (int64_t)nc * ITEMS;
+            const int64_t base = ((int64_t)bh * G * nc + cl) * ITEMS;
+            float4 acc[PER];
+#pragma unroll
+            for (int u = 0; u < PER; ++u) acc[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+            for (int gg = 0; gg < G; ++gg) {
+                const float4 *src = p4 + base + gg * gstride;
+#pragma unroll
+                for (int u = 0; u < PER; ++u) {
+                    const int item = tid + u * 256;
+                    if (item < ITEMS) {
+                        const float4 x = src[item];
+                        acc[u].x += x.x; acc[u].y += x.y; acc[u].z += x.z; acc[u].w += x.w;
+                    }
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < PER; ++u) {
+                const int item = tid + u * 256;
+                if (item < ITEMS) reinterpret_cast<float4 *>(Ps)[item] = acc[u];
+            }
+        }
+        // (2) q^T, k^T in fp32
         for (int e = tid; e < kL * DK; e += 256) {
             const int t = e / DK, i = e % DK;
             float a = 0.f, b = 0.f;
@@ -662,13 +706,13 @@ tc_finish_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__res
                 a = __bfloat162float(q[(bh * N + t0 + t) * DK + i]);
                 b = __bfloat162float(k[(bh * N + t0 + t) * DK + i]);
             }
-            fq[t * KP + i] = a;
-            fk[t * KP + i] = b;
+            fqT[i * kL + t] = a;
+            fkT[i * kL + t] = b;
         }
         __syncthreads();
-        // W[t][s] for 8x8 blocks on or below the diagonal
-        for (int blk = tid; blk < 16 * 16; blk += 256) {
-            const int tb = blk / 16, sbk = blk % 16;
+        // (3) W[t][s] = sum_{p<P} (q_t.k_s / c)^p / p! for s <= t, by 8x8 blocks
+        {
+            const int tb = tid / 16, sbk = tid % 16;
             float acc[8][8];
 #pragma unroll
             for (int a = 0; a < 8; ++a)
@@ -676,11 +720,12 @@ tc_finish_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__res
                 for (int b = 0; b < 8; ++b) acc[a][b] = 0.f;
             if (sbk <= tb) {
                 for (int i = 0; i < DK; ++i) {
-                    float xa[8], xb[8];
-#pragma unroll
-                    for (int a = 0; a < 8; ++a) xa[a] = fq[(tb * 8 + a) * KP + i];
-#pragma unroll
-                    for (int b = 0; b < 8; ++b) xb[b] = fk[(sbk * 8 + b) * KP + i];
+                    const float4 qa0 = *reinterpret_cast<const float4 *>(fqT + i * kL + tb * 8);
+                    const float4 qa1 = *reinterpret_cast<const float4 *>(fqT + i * kL + tb * 8 + 4);
+                    const float4 kb0 = *reinterpret_cast<const float4 *>(fkT + i * kL + sbk * 8);
+                    const float4 kb1 = *reinterpret_cast<const float4 *>(fkT + i * kL + sbk * 8 + 4);
+                    const float xa[8] = {qa0.x, qa0.y, qa0.z, qa0.w, qa1.x, qa1.y, qa1.z, qa1.w};
+                    const float xb[8] = {kb0.x, kb0.y, kb0.z, kb0.w, kb1.x, kb1.y, kb1.z, kb1.w};
 #pragma unroll
                     for (int a = 0; a < 8; ++a)
 #pragma unroll
@@ -691,51 +736,55 @@ tc_finish_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__res
             for (int a = 0; a < 8; ++a)
 #pragma unroll
                 for (int b = 0; b < 8; ++b) {
-                    const int t = tb * 8 + a, s = sbk * 8 + b;
+                    const int t = tb * 8 + a, s2 = sbk * 8 + b;
                     float w = 0.f;
-                    if (s <= t && t < nt) {
+                    if (s2 <= t && t < nt) {
                         const float x = acc[a][b] * inv_c;
-                        float h = 1.f;   // sum_{p<P} x^p / p!, Horner
+                        float h = 1.f;   // Horner form of sum_{p<P} x^p / p!
                         for (int pp = P - 1; pp >= 1; --pp) h = fmaf(h, x / (float)pp, 1.f);
                         w = h;
                     }
-                    Wt[t * WP + s] = w;
+                    Wt[t * WP + s2] = w;
                 }
         }
         __syncthreads();
-        float *fv = fq;   // [128][VP], [v | 1]
-        for (int e = tid; e < kL * VP; e += 256) {
-            const int t = e / VP, j = e % VP;
-            float a = 0.f;
-            if (t < nt) a = j < DV ? __bfloat162float(v[(bh * N + t0 + t) * DV + j]) : 1.f;
-            fv[e] = a;
+        // (4) v rows (fp32) over k^T's space
+        float *fv = fkT;   // [128][DV]
+        for (int e = tid; e < kL * DV; e += 256) {
+            const int t = e / DV;
+            fv[e] = t < nt ? __bfloat162float(v[(bh * N + t0) * DV + e]) : 0.f;
         }
         __syncthreads();
-        const int t = tid % kL, hseg = tid / kL;     // token, column half
-        const int j0 = hseg * HALF, j1 = (j0 + HALF < VP) ? j0 + HALF : VP;
-        float acc[HALF];
+        // (5) out[t][j] = (partial num + sum_s W[t][s] v[s][j]) / (partial den + sum_s W[t][s])
+        {
+            const int t = tid % kL, h = tid / kL;
+            float num[HW];
 #pragma unroll
-        for (int jj = 0; jj < HALF; ++jj) acc[jj] = 0.f;
-        for (int gg = 0; gg < G; ++gg) {
-            const float *src = part + (((bh * G + gg) * nc + cl) * (int64_t)VP) * kL + t;
+            for (int jj = 0; jj < HW; ++jj) num[jj] = Ps[(h * HW + jj) * kL + t];
+            float den = Ps[DV * kL + t];
+            for (int s2 = 0; s2 < kL; ++s2) {
+                const float w = Wt[t * WP + s2];
+                den += w;
+                const float *vr = fv + s2 * DV + h * HW;
 #pragma unroll
-            for (int jj = 0; jj < HALF; ++jj)
-                if (j0 + jj < j1) acc[jj] += src[(j0 + jj) * kL];
+                for (int jj = 0; jj < HW; jj += 4) {
+                    const float4 x = *reinterpret_cast<const float4 *>(vr + jj);
+                    num[jj] = fmaf(w, x.x, num[jj]);
+                    num[jj + 1] = fmaf(w, x.y, num[jj + 1]);
+                    num[jj + 2] = fmaf(w, x.z, num[jj + 2]);
+                    num[jj + 3] = fmaf(w, x.w, num[jj + 3]);
+                }
+            }
+            float *stage = fqT;   // [128][DV]
+#pragma unroll
+            for (int jj = 0; jj < HW; ++jj) stage[t * DV + h * HW + jj] = num[jj] / den;
         }
-        for (int s = 0; s < kL; ++s) {
-            const float w = Wt[t * WP + s];
-#pragma unroll
-            for (int jj = 0; jj < HALF; ++jj)
-                if (j0 + jj < j1) acc[jj] = fmaf(w, fv[s * VP + j0 + jj], acc[jj]);
+        __syncthreads();
+        {
+            const float4 *st4 = reinterpret_cast<const float4 *>(fqT);
+            float4 *o4 = reinterpret_cast<float4 *>(out + (bh * N + t0) * DV);
+            for (int e = tid; e < nt * DV / 4; e += 256) o4[e] = st4[e];
         }
-        if (j0 <= DV && DV < j1) den[t] = acc[DV - j0];
-        __syncthreads();
-        float *stage = fk;   // [128][DV] staging for coalesced stores
-#pragma unroll
-        for (int jj = 0; jj < HALF; ++jj)
-            if (j0 + jj < DV) stage[t * DV + j0 + jj] = acc[jj] / den[t];
-        __syncthreads();
-        for (int e = tid; e < nt * DV; e += 256) out[(bh * N + t0) * DV + e] = stage[e];
         __syncthreads();
     }
 }
@@ -811,7 +860,7 @@ cudaError_t run(const DeviceBasis &basis, int BH, int64_t N, const void *q, cons
     }
     e = cudaFuncSetAttribute(tc_scan_kernel<DK, DV>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
     if (e != cudaSuccess) return e;
-    const size_t fin_smem = sizeof(float) * ((size_t)2 * kL * (DK + 1) + (size_t)kL * (kL + 1));
+    const size_t fin_smem = sizeof(float) * ((size_t)(DV + 1) * kL + (size_t)2 * DK * kL + (size_t)kL * (kL + 1));
     e = cudaFuncSetAttribute(tc_finish_kernel<DK, DV>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)fin_smem);
     if (e != cudaSuccess) return e;
     int stall = -1;
