@@ -192,12 +192,19 @@ def barrier(torch, world):
 
 
 def max_over_ranks(torch, world, x: float) -> float:
+    """Largest x over all ranks (the job's time is the slowest rank's)."""
     if world == 1:
         return x
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def job_throughput(units_per_rank_step: float, steps: int, world: int, max_ms: float) -> float:
+    """Whole-job throughput: every rank's units over the slowest rank's time."""
+    return units_per_rank_step * steps * world / (max_ms / 1000.0)
 
 
 def timed(torch, world, fn, K, W, stream):
@@ -337,7 +344,7 @@ def main():
     if sata.sata_sync_status(stream) != 0:
         raise RuntimeError("device status after the timed prefill")
     tokens_per_step = w.B * w.N
-    value = tokens_per_step * args.steps * world / (ms / 1000.0)
+    value = job_throughput(tokens_per_step, args.steps, world, ms)
     launches = sum(n for n, _ in stats.values())
 
     # roofline of the dominant kernel
@@ -383,7 +390,7 @@ def main():
                 outh.copy_(out, non_blocking=True)
 
         ms_e2e = timed(torch, world, e2e_step, args.steps, 1, stream)
-        e2e = {"value": tokens_per_step * args.steps * world / (ms_e2e / 1000.0), "unit": "tokens/s",
+        e2e = {"value": job_throughput(tokens_per_step, args.steps, world, ms_e2e), "unit": "tokens/s",
                "h2d_bytes_per_step": in_bytes, "d2h_bytes_per_step": out_bytes,
                "ms_per_step": ms_e2e / args.steps}
 
@@ -450,7 +457,7 @@ def bench_decode(torch, sata, wl, args, world, dev, stream, peaks, peaks_src):
     sata.sata_set_option(sata.SATA_OPT_TIME_KERNELS, 0)
     if sata.sata_sync_status(stream) != 0:
         raise RuntimeError("device status after decode")
-    value = w.B * D * world / (ms / 1000.0)
+    value = job_throughput(w.B, D, world, ms)
     F = w.F
     state_bytes = 8 * F * (w.d_V + 1) * w.B * w.H          # read + write, fp32
     io_bytes = w.B * w.H * (2 * (2 * w.d_K + w.d_V) + 4 * w.d_V)
