@@ -164,6 +164,29 @@ SATA_API int sata_prefill_ex(const void *q, const void *k, const void *v, float 
  */
 SATA_API int sata_decode_step(sata_state *st, const void *q, const void *k, const void *v, float *out);
 
+/*
+ * sata_decode_step_static: the same decode step as sata_decode_step, for
+ * callers that may not allocate device memory.  The method's pages have no
+ * counterpart; this is a deployment variant.
+ *
+ * Some callers must not call cudaMalloc: a serving runtime that owns every
+ * byte of the GPU through a pre-allocated arena, a plugin inside a host
+ * application with its own allocator, or a process held to a memory budget.
+ * cudaMalloc allocates outside their accounting and can also synchronise the
+ * device.  sata_decode_step allocates on first use (its partial-sum workspace
+ * and basis tables).  This entry point allocates nothing: the caller passes the
+ * state, inputs and outputs, as above.  Its partial sums live in a 4 MiB static
+ * device array compiled into the library, and it derives the basis
+ * arithmetically instead of from tables.
+ *   Limit: B*H*ceil(F/1024)*(d_V+1) <= 1,048,576 fp32 values (about 1500 heads
+ *   at d_K = d_V = 32).  Beyond that it returns SATA_ENOMEM without launching.
+ *   The first call on each device looks up the array's device address (once);
+ *   make it before any stream capture.  All calls share the array: calls that
+ *   overlap on the GPU race.  Nothing in it needs clearing between calls.
+ * Returns SATA_OK or a negative status as sata_decode_step; st->tokens += 1.
+ */
+SATA_API int sata_decode_step_static(sata_state *st, const void *q, const void *k, const void *v, float *out);
+
 /* Tuning and test options (process-wide).  Keys: */
 enum sata_option {
     SATA_OPT_PREFILL_PATH = 1,   /* 0 auto, 1 CUDA-core path, 2 tensor-core path */

@@ -11,5 +11,5 @@ from .binding import (  # noqa: F401
     sata_state_init, sata_sync_status, sata_version, sata_workspace_bytes,
     SATA_OK, SATA_EINVAL, SATA_EUNSUPPORTED, SATA_ECUDA, SATA_ETIMEOUT, SATA_ENOMEM,
     SATA_ERANGE, SATA_EALIGN, SATA_OPT_PREFILL_PATH, SATA_OPT_WAIT_LIMIT, SATA_OPT_TEST_STALL,
-    SATA_OPT_TIME_KERNELS, sata_kernel_stats, sata_reset_kernel_stats,
+    SATA_OPT_TIME_KERNELS, sata_kernel_stats, sata_reset_kernel_stats, sata_decode_step_static,
 )

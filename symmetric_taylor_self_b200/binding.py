@@ -35,7 +35,7 @@ EXPORTED = (
     "sata_build_basis", "sata_set_stream", "sata_sync_status", "sata_shutdown",
     "sata_state_bytes", "sata_state_init", "sata_workspace_bytes", "sata_prefill",
     "sata_prefill_ex", "sata_decode_step", "sata_set_option", "sata_get_option",
-    "sata_kernel_stats", "sata_reset_kernel_stats",
+    "sata_kernel_stats", "sata_reset_kernel_stats", "sata_decode_step_static",
 )
 
 
@@ -94,6 +94,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "sata_get_option": (i32, [i32, P_i64]),
         "sata_kernel_stats": (i32, [ctypes.POINTER(sata_kernel_stat), i32, ctypes.POINTER(ctypes.c_int)]),
         "sata_reset_kernel_stats": (i32, []),
+        "sata_decode_step_static": (i32, [st_p, vp, vp, vp, vp]),
     }
     for name, (res, args) in sigs.items():
         fn = getattr(lib, name)
@@ -225,6 +226,12 @@ def sata_state_init(st, B, H, d_K, d_V, P, S, Z, stream=None):
 def sata_decode_step(st, q, k, v, out):
     _check(load().sata_decode_step(ctypes.byref(st), _ptr(q), _ptr(k), _ptr(v), _ptr(out)),
            "sata_decode_step")
+
+
+def sata_decode_step_static(st, q, k, v, out):
+    """The decode step that allocates no device memory (see include/sata.h)."""
+    _check(load().sata_decode_step_static(ctypes.byref(st), _ptr(q), _ptr(k), _ptr(v), _ptr(out)),
+           "sata_decode_step_static")
 
 
 # ------------------------------------------------- tensor-level wrappers ----

@@ -76,6 +76,8 @@ int current_device(cudaError_t *err) {
 
 }  // namespace
 
+int record_cuda_error(cudaError_t e) { return cuda_fail(e); }
+
 const DeviceBasis *device_basis(int d_K, int P, cudaError_t *err) {
     std::lock_guard<std::mutex> lk(g_mu);
     const int dev = current_device(err);

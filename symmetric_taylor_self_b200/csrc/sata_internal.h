@@ -45,6 +45,9 @@ struct DeviceBasis {
 // Device-side status words, one set per device: [0] timeout, [1] range.
 enum { kFlagTimeout = 0, kFlagRange = 1, kNumFlags = 4 };
 
+// Record a failed CUDA call for sata_last_cuda_error(); returns SATA_ECUDA.
+int record_cuda_error(cudaError_t e);
+
 // Library-owned per-device resources (basis cache, status flags, workspaces).
 const DeviceBasis *device_basis(int d_K, int P, cudaError_t *err);
 int *device_flags(cudaError_t *err);

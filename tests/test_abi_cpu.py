@@ -150,3 +150,22 @@ def test_product_path_does_not_touch_oracle():
                 src = open(os.path.join(dirpath, fn)).read()
                 assert "import oracle" not in src and "from oracle" not in src, fn
                 assert "sata_oracle" not in src and "liboracle" not in src, fn
+
+
+def test_static_decode_rejects_oversized_requests_before_any_cuda_call(lib):
+    """The no-allocation decode step rejects shapes whose partial sums exceed its
+    static scratch, before touching the GPU.  Run on the CPU suite only: the
+    pointers below are placeholders that must never reach a kernel."""
+    from symmetric_taylor_self_b200 import binding as bd
+    B, H, d = 64, 64, 64
+    F = math.comb(d + 3, 3)
+    G = (F + 1023) // 1024
+    assert B * H * G * (d + 1) > 2 ** 20          # oversized by construction
+    fake = ctypes.c_void_p(0x10000)
+    st = bd.sata_state(B=B, H=H, d_K=d, d_V=d, P=4, F=F, S=0x10000, Z=0x10000, stream=None, tokens=0)
+    assert lib.sata_decode_step_static(ctypes.byref(st), fake, fake, fake, fake) == bd.SATA_ENOMEM
+    assert st.tokens == 0
+    # invalid arguments are rejected the same way as by sata_decode_step
+    assert lib.sata_decode_step_static(None, fake, fake, fake, fake) == bd.SATA_EINVAL
+    st.F = 7
+    assert lib.sata_decode_step_static(ctypes.byref(st), fake, fake, fake, fake) == bd.SATA_EINVAL
