@@ -152,7 +152,7 @@ def ncu_traffic(kernel):
         return None
     if e.get("source_sha256_16") != kernel_source_hash(e.get("source", "")):
         return None
-    return e.get("dram_bytes_per_full_launch")
+    return e.get("dram_bytes_per_launch")
 
 
 def flops_per_token(d_K, d_V, P):
@@ -371,7 +371,7 @@ def main():
         roof["ms_per_launch"] = per_launch_ms
         roof["algorithmic_flops_per_launch"] = flops_per_launch
         tr = ncu_traffic(dom)
-        roof["traffic"] = None if tr is None else tr / (n_l / args.steps)
+        roof["traffic"] = tr
         if tr is None:
             roof["traffic_note"] = "no ncu capture of the current kernel source"
 

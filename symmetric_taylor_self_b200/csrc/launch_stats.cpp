@@ -26,7 +26,7 @@ thread_local cudaEvent_t t_start[kNumKernels] = {};
 
 const char *const kNames[kNumKernels] = {
     "decode_stream", "decode_finish", "simt_scan", "simt_finish",
-    "tc_prep", "tc_scan", "tc_finish",
+    "tc_prep", "tc_scan", "tc_finish", "tc_reduce",
 };
 
 void drain_locked() {

@@ -41,7 +41,7 @@ namespace sata {
 namespace {
 
 constexpr int kL = 128;               // chunk length (tokens)
-constexpr int kNS = 3;                // ring stages of generated operand tiles
+constexpr int kNQ = 2;                // ring stages of alpha*C*phi(q) tiles (shared memory)
 constexpr int kStageBytes = 128 * kL * 2;
 constexpr int kScanThreads = 448;     // 14 warps
 constexpr int kWarpProducer = 0, kWarpMma = 1, kWarpConv0 = 2, kWarpGen0 = 6;
@@ -53,26 +53,30 @@ template <int DK, int DV>
 struct Cfg {
     static constexpr int NV = DV + 16;                           // MMA N: [V | 1 | 0 pad]
     static constexpr int MT_MAX = DV == 64 ? 4 : (DV == 32 ? 8 : 12);
-    static constexpr int ROW = kL * 2;                           // one image row: 128 fp16
+    static constexpr int ROW = kL * 2;                           // one (q/c)^T row: 128 fp16
+    static constexpr int KROW = ROW + 16;                        // k^T rows padded so that 32 lanes
+                                                                 // reading 32 rows hit distinct banks
     static constexpr int IMG_V = NV * ROW;                       // [V|1]^T, K-major SW128
-    static constexpr int IMG_X = (DK + 1) * ROW;                 // k^T or (q/c)^T, row DK = 1
-    static constexpr int IMG = IMG_V + 2 * IMG_X;
+    static constexpr int OFF_IQ = IMG_V;                         // (q/c)^T, row DK = 1
+    static constexpr int OFF_IK = IMG_V + (DK + 1) * ROW;        // k^T, row DK = 1
+    static constexpr int IMG = OFF_IK + (DK + 1) * KROW;
     static constexpr int IMG_PAD = (IMG + 1023) / 1024 * 1024;
     static constexpr int OFF_RING = 2 * IMG_PAD;
-    static constexpr int OFF_BS = OFF_RING + kNS * kStageBytes;
+    static constexpr int OFF_BS = OFF_RING + kNQ * kStageBytes;
     static constexpr int BS_BYTES = 128 * NV * 2;
-    static constexpr int OFF_TAB = OFF_BS + BS_BYTES;
+    static constexpr int OFF_TAB = OFF_BS + 2 * BS_BYTES;
     static constexpr int OFF_MC = OFF_TAB + MT_MAX * 128 * 4;
     static constexpr int OFF_BAR = (OFF_MC + MT_MAX * 128 * 2 + 15) / 16 * 16;
-    // barrier indices
-    static constexpr int B_INF = 0, B_INE = 2, B_AF = 4, B_AE = 4 + kNS, B_BSF = 4 + 2 * kNS,
-                         B_BSE = B_BSF + 1, B_SD = B_BSE + 1, B_OF = B_SD + MT_MAX,
-                         B_OE = B_OF + 2, B_FIN = B_OE + 2, N_BAR = B_FIN + 1;
+    // barrier indices (pairs are double buffers)
+    static constexpr int B_INF = 0, B_INE = 2, B_QF = 4, B_QE = 6, B_KF = 8, B_KE = 10, B_BSF = 12,
+                         B_BSE = 14, B_SD = 16, B_OF = B_SD + MT_MAX, B_OE = B_OF + 1, B_FIN = B_OE + 1,
+                         N_BAR = B_FIN + 1;
     static constexpr int OFF_MISC = OFF_BAR + N_BAR * 8;
     static constexpr int SMEM = OFF_MISC + 16 + 1024;            // + base alignment slack
-    static constexpr int COL_O = MT_MAX * NV;                    // TMEM column of D_O[0]
+    static constexpr int COL_O = MT_MAX * NV;                    // TMEM: readout accumulator
+    static constexpr int COL_A = COL_O + NV;                     // TMEM: two phi(k) stages, 32 columns each
     static constexpr int LBO_BS = (NV / 8) * 128;
-    static_assert(COL_O + 2 * NV <= 512, "TMEM columns");
+    static_assert(COL_A + 64 <= 512, "TMEM columns");
     static_assert(SMEM <= 232448, "shared memory");
     static_assert(NV % 16 == 0, "MMA N");
 };
@@ -154,6 +158,14 @@ __device__ __forceinline__ void tc_mma(uint32_t d, uint64_t a, uint64_t b, uint3
         "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
         "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d),
         "l"(a), "l"(b), "r"(idesc), "r"(acc)
+        : "memory");
+}
+// A operand in TMEM (rows on lanes, two fp16 per 32-bit column, even K in the low half).
+__device__ __forceinline__ void tc_mma_ta(uint32_t d, uint32_t a_tmem, uint64_t b, uint32_t idesc, uint32_t acc) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}\n" ::"r"(d),
+        "r"(a_tmem), "l"(b), "r"(idesc), "r"(acc)
         : "memory");
 }
 __device__ __forceinline__ void tc_ld16(uint32_t taddr, uint32_t *r) {
@@ -253,8 +265,8 @@ __device__ __forceinline__ uint4 hmul4s(uint4 a, __half2 m) {
 // ----------------------------------------------------------------- prep ----
 
 // Per (head, chunk): write the chunk image [ [V|1]^T (K-major, 128-byte swizzle)
-// | k^T | (q/c)^T ], fp16, padded tokens zero (including their 1 entries), and
-// raise the per-head maxima of |q|, |k|, |v|.
+// | (q/c)^T | k^T (rows padded to 272 bytes) ], fp16, padded tokens zero
+// (including their 1 entries), and raise the per-head maxima of |q|, |k|, |v|.
 template <int DK, int DV>
 __global__ void __launch_bounds__(256)
 tc_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k,
@@ -329,9 +341,8 @@ tc_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restr
                 hk[j] = i < DK ? sk[t * PK + i] : (t < nt ? one : zero);
                 hq[j] = i < DK ? sq[t * PK + i] : (t < nt ? one : zero);
             }
-            *reinterpret_cast<uint4 *>(out + C::IMG_V + i * C::ROW + t8 * 16) = *reinterpret_cast<const uint4 *>(hk);
-            *reinterpret_cast<uint4 *>(out + C::IMG_V + C::IMG_X + i * C::ROW + t8 * 16) =
-                *reinterpret_cast<const uint4 *>(hq);
+            *reinterpret_cast<uint4 *>(out + C::OFF_IK + i * C::KROW + t8 * 16) = *reinterpret_cast<const uint4 *>(hk);
+            *reinterpret_cast<uint4 *>(out + C::OFF_IQ + i * C::ROW + t8 * 16) = *reinterpret_cast<const uint4 *>(hq);
         }
         // per-head maxima (non-negative floats order like their bit patterns)
 #pragma unroll
@@ -403,8 +414,8 @@ __global__ void __launch_bounds__(kScanThreads, 1) tc_scan_kernel(const ScanPara
         for (int i = 0; i < C::N_BAR; ++i) {
             uint32_t cnt = 1;
             if (i == C::B_INE || i == C::B_INE + 1) cnt = kGenWarps + 1;
-            else if (i >= C::B_AF && i < C::B_AF + kNS) cnt = kGenWarps;
-            else if (i == C::B_BSF || i == C::B_OE || i == C::B_OE + 1) cnt = 4;
+            else if ((i >= C::B_QF && i < C::B_QF + 2) || (i >= C::B_KF && i < C::B_KF + 2)) cnt = kGenWarps;
+            else if (i == C::B_BSF || i == C::B_BSF + 1 || i == C::B_OE) cnt = 4;
             mbar_init(BAR(i), cnt);
         }
         *abort_flag = 0;
@@ -453,47 +464,46 @@ __global__ void __launch_bounds__(kScanThreads, 1) tc_scan_kernel(const ScanPara
         if (lane == 0) {
             constexpr uint32_t id_upd = idesc_f16(128, NV, 0, 0);
             constexpr uint32_t id_rd = idesc_f16(128, NV, 1, 1);
-            int seq = 0;
+            int qa = 0, qk = 0;
             bool ok = true;
             for (int cl = 0; cl < p.nc && ok; ++cl) {
-                const int ib = cl & 1, ob = cl & 1;
-                ok = W.wait(BAR(C::B_INF + ib), (cl >> 1) & 1) && W.wait(BAR(C::B_OE + ob), ((cl >> 1) & 1) ^ 1);
-                if (!ok) break;
-                tc_after();
+                const int ib = cl & 1;
+                if (!(ok = W.wait(BAR(C::B_INF + ib), (cl >> 1) & 1))) break;
                 const uint32_t vimg = sb + ib * C::IMG_PAD;
-                const uint32_t d_o = tmem + C::COL_O + ob * NV;
                 for (int j = 0; j < p.MT; ++j) {
-                    const int qn = cl * p.MT + j;
-                    int s = seq % kNS;
-                    ok = W.wait(BAR(C::B_BSF), qn & 1) && W.wait(BAR(C::B_AF + s), (seq / kNS) & 1);
+                    const int qn = cl * p.MT + j, bsb = qn & 1, sa = qa & 1;
+                    ok = W.wait(BAR(C::B_BSF + bsb), (qn >> 1) & 1) && W.wait(BAR(C::B_QF + sa), (qa >> 1) & 1);
+                    if (ok && j == 0) ok = W.wait(BAR(C::B_OE), (cl & 1) ^ 1);   // epilogue of cl-1 done
                     if (!ok) break;
                     tc_after();
                     // readout: D_O += (alpha C phi(q)) [128 t x 128 f] . [S|Z]_j fp16 [128 f x NV]
-                    const uint32_t a_st = sb + C::OFF_RING + s * kStageBytes;
+                    const uint32_t a_st = sb + C::OFF_RING + sa * kStageBytes;
+                    const uint32_t b_s = sb + C::OFF_BS + bsb * C::BS_BYTES;
 #pragma unroll
                     for (int ks = 0; ks < 8; ++ks)
-                        tc_mma(d_o, sdesc(a_st + ks * 2048, 16384, 1024, 2),
-                               sdesc(sb + C::OFF_BS + ks * 2 * C::LBO_BS, C::LBO_BS, 128, 0), id_rd,
+                        tc_mma(tmem + C::COL_O, sdesc(a_st + ks * 2048, 16384, 1024, 2),
+                               sdesc(b_s + ks * 2 * C::LBO_BS, C::LBO_BS, 128, 0), id_rd,
                                (j > 0 || ks > 0) ? 1u : 0u);
-                    tc_commit(BAR(C::B_AE + s));
-                    tc_commit(BAR(C::B_BSE));
-                    ++seq;
-                    s = seq % kNS;
-                    ok = W.wait(BAR(C::B_AF + s), (seq / kNS) & 1);
-                    if (!ok) break;
-                    tc_after();
-                    // update: [S|Z]_j += phi(K)^T [128 f x 128 t] . [V|1] [128 t x NV]
-                    const uint32_t k_st = sb + C::OFF_RING + s * kStageBytes;
+                    tc_commit(BAR(C::B_QE + sa));
+                    tc_commit(BAR(C::B_BSE + bsb));
+                    if (j == p.MT - 1) tc_commit(BAR(C::B_OF));
+                    ++qa;
+                    // update: [S|Z]_j += phi(K)^T [128 f x 64 t] (TMEM) . [V|1] [64 t x NV], two halves
+                    for (int h = 0; h < 2 && ok; ++h) {
+                        const int sk = qk & 1;
+                        if (!(ok = W.wait(BAR(C::B_KF + sk), (qk >> 1) & 1))) break;
+                        tc_after();
 #pragma unroll
-                    for (int ks = 0; ks < 8; ++ks)
-                        tc_mma(tmem + j * NV, sdesc(k_st + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024, 2),
-                               sdesc(vimg + (ks >> 2) * (NV * 128) + (ks & 3) * 32, 16, 1024, 2), id_upd, 1u);
-                    tc_commit(BAR(C::B_AE + s));
+                        for (int ks = 0; ks < 4; ++ks)
+                            tc_mma_ta(tmem + j * NV, tmem + C::COL_A + sk * 32 + ks * 8,
+                                      sdesc(vimg + h * (NV * 128) + ks * 32, 16, 1024, 2), id_upd, 1u);
+                        tc_commit(BAR(C::B_KE + sk));
+                        ++qk;
+                    }
+                    if (!ok) break;
                     tc_commit(BAR(C::B_SD + j));
-                    ++seq;
                 }
                 if (!ok) break;
-                tc_commit(BAR(C::B_OF + ob));
                 tc_commit(BAR(C::B_INE + ib));
             }
             // every issued MMA completes before TMEM is released
@@ -523,15 +533,14 @@ __global__ void __launch_bounds__(kScanThreads, 1) tc_scan_kernel(const ScanPara
         tc_wait_st();
         int64_t part_base = ((int64_t)bh * p.G + g) * p.nc;
         auto epilogue = [&](int cl) -> bool {
-            const int ob = cl & 1;
-            if (!W.wait(BAR(C::B_OF + ob), (cl >> 1) & 1)) return false;
+            if (!W.wait(BAR(C::B_OF), cl & 1)) return false;
             tc_after();
 #pragma unroll
-            for (int c16 = 0; c16 < NV / 16; ++c16) tc_ld16(tmem + lane_off + C::COL_O + ob * NV + c16 * 16, r + c16 * 16);
+            for (int c16 = 0; c16 < NV / 16; ++c16) tc_ld16(tmem + lane_off + C::COL_O + c16 * 16, r + c16 * 16);
             tc_wait_ld();
             tc_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(BAR(C::B_OE + ob));
+            if (lane == 0) mbar_arrive(BAR(C::B_OE));
             const float up = pow2f(state_sigma(p.c0 + cl, mk, mv, ms, p.P));
             float *dst = p.part + ((part_base + cl) * (DV + 1)) * kL + row;
 #pragma unroll
@@ -542,15 +551,15 @@ __global__ void __launch_bounds__(kScanThreads, 1) tc_scan_kernel(const ScanPara
         for (int cl = 0; cl < p.nc && ok; ++cl) {
             const float down = pow2f(-state_sigma(p.c0 + cl, mk, mv, ms, p.P));
             for (int j = 0; j < p.MT; ++j) {
-                const int qn = cl * p.MT + j;
+                const int qn = cl * p.MT + j, bsb = qn & 1;
                 if (cl > 0 && !(ok = W.wait(BAR(C::B_SD + j), (cl - 1) & 1))) break;
                 tc_after();
 #pragma unroll
                 for (int c16 = 0; c16 < NV / 16; ++c16) tc_ld16(tmem + lane_off + j * NV + c16 * 16, r + c16 * 16);
                 tc_wait_ld();
-                if (!(ok = W.wait(BAR(C::B_BSE), (qn & 1) ^ 1))) break;
+                if (!(ok = W.wait(BAR(C::B_BSE + bsb), ((qn >> 1) & 1) ^ 1))) break;
                 // B_s: [S|Z]_j * 2^-sigma as fp16, K = feature rows, N-major core matrices
-                uint8_t *bs = smem + C::OFF_BS + (row / 8) * C::LBO_BS + (row % 8) * 16;
+                uint8_t *bs = smem + C::OFF_BS + bsb * C::BS_BYTES + (row / 8) * C::LBO_BS + (row % 8) * 16;
 #pragma unroll
                 for (int m = 0; m < NV / 8; ++m) {
                     __align__(16) __half2 h[4];
@@ -563,7 +572,7 @@ __global__ void __launch_bounds__(kScanThreads, 1) tc_scan_kernel(const ScanPara
                 fence_proxy_async();
                 tc_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(BAR(C::B_BSF));
+                if (lane == 0) mbar_arrive(BAR(C::B_BSF + bsb));
                 if (j == 0 && cl > 0 && !(ok = epilogue(cl - 1))) break;
             }
         }
@@ -587,33 +596,37 @@ __global__ void __launch_bounds__(kScanThreads, 1) tc_scan_kernel(const ScanPara
             }
         }
         tc_before();
-    } else {
+    } else if (warp >= kWarpGen0) {
         // ------------------------------------------------ feature generation
         const int gt = threadIdx.x - kWarpGen0 * 32;
+        // alpha*C*phi(q/c) tiles into shared memory: thread = 8 tokens x 8 features
         const int tg = gt & 15;            // tokens 8*tg .. 8*tg+7
         const int fgrp = gt >> 4;          // features 8*fgrp .. 8*fgrp+7 of the tile
         const int xoff = tg * 16;
         const int hoff = (tg >> 3) * 16384;
         const int cidx = tg & 7;
-        int seq = 0;
+        // phi(k) tiles into TMEM: lane = feature row of the tile, 32 tokens per warp
+        const int kq = warp & 3;                           // TMEM lane quarter of this warp
+        const int krow = kq * 32 + lane;
+        const int ksub = (warp - kWarpGen0) >> 2;          // which 32 tokens of a 64-token stage
+        const uint32_t k_lane_off = (uint32_t)(kq * 32) << 16;
+        int qa = 0, qk = 0;
         bool ok = true;
         for (int cl = 0; cl < p.nc && ok; ++cl) {
             const int ib = cl & 1;
             if (!(ok = W.wait(BAR(C::B_INF + ib), (cl >> 1) & 1))) break;
-            const uint8_t *xk = smem + ib * C::IMG_PAD + C::IMG_V;
-            const uint8_t *xq = xk + C::IMG_X;
+            const uint8_t *xq = smem + ib * C::IMG_PAD + C::OFF_IQ;
+            const uint8_t *xk = smem + ib * C::IMG_PAD + C::OFF_IK;
             for (int j = 0; j < p.MT && ok; ++j) {
-                for (int side = 0; side < 2; ++side, ++seq) {   // 0: alpha C phi(q/.) (readout), 1: phi(k)
-                    const int s = seq % kNS;
-                    if (!(ok = W.wait(BAR(C::B_AE + s), ((seq / kNS) & 1) ^ 1))) break;
-                    uint8_t *stage = smem + C::OFF_RING + s * kStageBytes + hoff;
-                    const uint8_t *x = side ? xk : xq;
+                {   // alpha*C*phi(q/c), shared memory, 128-byte swizzled [f][t]
+                    const int sa = qa & 1;
+                    if (!(ok = W.wait(BAR(C::B_QE + sa), ((qa >> 1) & 1) ^ 1))) break;
+                    uint8_t *stage = smem + C::OFF_RING + sa * kStageBytes + hoff;
                     const uint4 *tj4 = reinterpret_cast<const uint4 *>(tab + j * 128 + fgrp * 8);
                     const uint4 t_lo = tj4[0], t_hi = tj4[1];
                     const uint32_t tw[8] = {t_lo.x, t_lo.y, t_lo.z, t_lo.w, t_hi.x, t_hi.y, t_hi.z, t_hi.w};
                     __align__(16) __half mj[8];
-                    if (side == 0)
-                        *reinterpret_cast<uint4 *>(mj) = *reinterpret_cast<const uint4 *>(mc + j * 128 + fgrp * 8);
+                    *reinterpret_cast<uint4 *>(mj) = *reinterpret_cast<const uint4 *>(mc + j * 128 + fgrp * 8);
                     uint32_t prev = 0xFFFFFFFFu;
                     uint4 pre = make_uint4(0, 0, 0, 0);
 #pragma unroll
@@ -621,25 +634,55 @@ __global__ void __launch_bounds__(kScanThreads, 1) tc_scan_kernel(const ScanPara
                         const uint32_t w = tw[i];
                         if ((w & 0xFFFFu) != prev) {   // new prefix pair (a, b)
                             prev = w & 0xFFFFu;
-                            const uint4 xa = *reinterpret_cast<const uint4 *>(x + (w & 255u) * C::ROW + xoff);
-                            const uint4 xb = *reinterpret_cast<const uint4 *>(x + ((w >> 8) & 255u) * C::ROW + xoff);
+                            const uint4 xa = *reinterpret_cast<const uint4 *>(xq + (w & 255u) * C::ROW + xoff);
+                            const uint4 xb = *reinterpret_cast<const uint4 *>(xq + ((w >> 8) & 255u) * C::ROW + xoff);
                             pre = hmul4(xa, xb);
                         }
-                        const uint4 xl = *reinterpret_cast<const uint4 *>(x + ((w >> 16) & 255u) * C::ROW + xoff);
-                        uint4 val = hmul4(pre, xl);
-                        if (side == 0) val = hmul4s(val, __half2half2(mj[i]));
+                        const uint4 xl = *reinterpret_cast<const uint4 *>(xq + ((w >> 16) & 255u) * C::ROW + xoff);
+                        const uint4 val = hmul4s(hmul4(pre, xl), __half2half2(mj[i]));
                         const int fr = fgrp * 8 + i;
                         *reinterpret_cast<uint4 *>(stage + fr * 128 + ((cidx ^ i) << 4)) = val;
                     }
                     fence_proxy_async();
                     __syncwarp();
-                    if (lane == 0) mbar_arrive(BAR(C::B_AF + s));
+                    if (lane == 0) mbar_arrive(BAR(C::B_QF + sa));
+                    ++qa;
+                }
+                {   // phi(k), TMEM: this lane's feature over 32 tokens, per 64-token stage
+                    const uint32_t w = tab[j * 128 + krow];
+                    const uint8_t *ra = xk + (w & 255u) * C::KROW;
+                    const uint8_t *rb = xk + ((w >> 8) & 255u) * C::KROW;
+                    const uint8_t *rl = xk + ((w >> 16) & 255u) * C::KROW;
+                    for (int h = 0; h < 2; ++h) {
+                        const int sk = qk & 1;
+                        if (!(ok = W.wait(BAR(C::B_KE + sk), ((qk >> 1) & 1) ^ 1))) break;
+                        const int tb = (64 * h + 32 * ksub) * 2;   // byte offset of this warp's tokens
+                        uint32_t rr[16];
+#pragma unroll
+                        for (int g8 = 0; g8 < 4; ++g8) {
+                            const uint4 xa = *reinterpret_cast<const uint4 *>(ra + tb + g8 * 16);
+                            const uint4 xb = *reinterpret_cast<const uint4 *>(rb + tb + g8 * 16);
+                            const uint4 xl = *reinterpret_cast<const uint4 *>(rl + tb + g8 * 16);
+                            const uint4 val = hmul4(hmul4(xa, xb), xl);
+                            rr[4 * g8 + 0] = val.x;
+                            rr[4 * g8 + 1] = val.y;
+                            rr[4 * g8 + 2] = val.z;
+                            rr[4 * g8 + 3] = val.w;
+                        }
+                        tc_st16(tmem + k_lane_off + C::COL_A + sk * 32 + 16 * ksub, rr);
+                        tc_wait_st();
+                        tc_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(BAR(C::B_KF + sk));
+                        ++qk;
+                    }
                 }
             }
             if (!ok) break;
             __syncwarp();
             if (lane == 0) mbar_arrive(BAR(C::B_INE + ib));
         }
+        tc_before();
     }
 
     __syncthreads();
@@ -650,6 +693,36 @@ __global__ void __launch_bounds__(kScanThreads, 1) tc_scan_kernel(const ScanPara
 }
 
 // --------------------------------------------------------------- finish ----
+
+// Sum the G feature-group partials of every (head, chunk, column, token):
+// part [BH][G][nc][DV+1][128] -> red [BH][nc][DV+1][128].  A pure streaming
+// kernel (float4, eight loads in flight per thread, fixed summation order).
+template <int DV>
+__global__ void __launch_bounds__(256)
+tc_reduce_kernel(const float4 *__restrict__ part, float4 *__restrict__ red, int BH, int G, int nc) {
+    const int64_t per_head = (int64_t)nc * (DV + 1) * (kL / 4);
+    const int64_t total = (int64_t)BH * per_head;
+    for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < total; e += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t bh = e / per_head, rem = e % per_head;
+        const float4 *src = part + bh * G * per_head + rem;
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        int gg = 0;
+        for (; gg + 8 <= G; gg += 8) {
+            float4 x[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) x[u] = src[(int64_t)(gg + u) * per_head];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                acc.x += x[u].x; acc.y += x[u].y; acc.z += x[u].z; acc.w += x[u].w;
+            }
+        }
+        for (; gg < G; ++gg) {
+            const float4 x = src[(int64_t)gg * per_head];
+            acc.x += x.x; acc.y += x.y; acc.z += x.z; acc.w += x.w;
+        }
+        red[e] = acc;
+    }
+}
 
 // Per (head, chunk): sum the feature tiles' inter-chunk partials, add the
 // intra-chunk block sum_{s<=t} w_ts [v_s | 1] (fp32 from the bf16 inputs) and
@@ -793,7 +866,7 @@ tc_finish_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__res
 
 struct Plan {
     int MT = 1, G = 1, nchunks = 0, nc_seg = 0;
-    size_t off_stats = 0, off_img = 0, off_part = 0, off_state = 0, total = 0;
+    size_t off_stats = 0, off_img = 0, off_part = 0, off_red = 0, off_state = 0, total = 0;
 };
 
 size_t align256(size_t x) { return (x + 255) / 256 * 256; }
@@ -817,7 +890,8 @@ Plan make_plan(int BH, int64_t N, int64_t F, bool need_state) {
     pl.off_stats = 0;
     pl.off_img = align256((size_t)BH * 4 * sizeof(float));
     pl.off_part = pl.off_img + align256((size_t)BH * pl.nchunks * C::IMG);
-    pl.off_state = pl.off_part + align256(per_chunk * pl.nc_seg);
+    pl.off_red = pl.off_part + align256(per_chunk * pl.nc_seg);
+    pl.off_state = pl.off_red + align256((size_t)BH * (DV + 1) * kL * sizeof(float) * pl.nc_seg);
     pl.total = pl.off_state + (need_state ? align256((size_t)BH * F * (DV + 1) * sizeof(float)) : 0);
     return pl;
 }
@@ -897,10 +971,17 @@ cudaError_t run(const DeviceBasis &basis, int BH, int64_t N, const void *q, cons
         tc_scan_kernel<DK, DV><<<BH * pl.G, kScanThreads, C::SMEM, stream>>>(sp);
         launch_end(kTcScan, stream);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        float *red = (float *)(w + pl.off_red);
+        const int64_t rwork = (int64_t)BH * sp.nc * (DV + 1) * (kL / 4);
+        launch_begin(kTcReduce, stream);
+        tc_reduce_kernel<DV><<<(int)((rwork + 255) / 256 < 148 * 32 ? (rwork + 255) / 256 : 148 * 32), 256, 0, stream>>>(
+            (const float4 *)part, (float4 *)red, BH, pl.G, sp.nc);
+        launch_end(kTcReduce, stream);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
         const int64_t fwork = (int64_t)BH * sp.nc;
         launch_begin(kTcFinish, stream);
         tc_finish_kernel<DK, DV><<<(int)(fwork < 148 * 16 ? fwork : 148 * 16), 256, fin_smem, stream>>>(
-            qb, kb, vb, part, out, BH, pl.G, sp.c0, sp.nc, N, basis.P, inv_c);
+            qb, kb, vb, red, out, BH, 1, sp.c0, sp.nc, N, basis.P, inv_c);
         launch_end(kTcFinish, stream);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }

@@ -55,7 +55,7 @@ void *device_workspace(int slot, size_t bytes, cudaError_t *err);
 
 // Kernel identities for launch statistics.
 enum KernelId {
-    kDecodeStream = 0, kDecodeFinish, kSimtScan, kSimtFinish, kTcPrep, kTcScan, kTcFinish,
+    kDecodeStream = 0, kDecodeFinish, kSimtScan, kSimtFinish, kTcPrep, kTcScan, kTcFinish, kTcReduce,
     kNumKernels
 };
 const char *kernel_name(int id);
