@@ -48,6 +48,8 @@ def parse():
     ap.add_argument("--decode-workload", default="decode_d32")
     ap.add_argument("--decode-steps", type=int, default=256)
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--only", choices=["all", "prefill", "decode"], default="all",
+                    help="run one part only (reduced workloads for profiler captures)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--path", choices=["auto", "cuda_core", "tensor_core"], default="auto")
@@ -305,6 +307,8 @@ def main():
     from symmetric_taylor_self_b200 import workloads as wl
 
     rank, world, local = dist_setup(torch)
+    if args.only != "all":
+        return run_part(torch, sata, wl, args, world)
     dev = torch.device("cuda", torch.cuda.current_device())
     sata.load()
     sata.sata_set_option(sata.SATA_OPT_PREFILL_PATH, {"auto": 0, "cuda_core": 1, "tensor_core": 2}[args.path])
@@ -421,6 +425,32 @@ def main():
         import torch.distributed as dist
         dist.destroy_process_group()
     return 0
+
+
+def run_part(torch, sata, wl, args, world):
+    """One part alone, no JSON line: the command profiler captures run."""
+    dev = torch.device("cuda", torch.cuda.current_device())
+    stream = torch.cuda.Stream()
+    if args.only == "prefill":
+        w = wl.WORKLOADS[args.workload]
+        (q, k, v), _ = wl.make_inputs(w)
+        qd, kd, vd = q.to(dev), k.to(dev), v.to(dev)
+        out = torch.empty((w.B, w.H, w.N, w.d_V), dtype=torch.float32, device=dev)
+        for _ in range(args.warmup + args.steps):
+            sata.sata_prefill_ex(qd, kd, vd, out, w.B, w.H, w.N, w.d_K, w.d_V, w.P, None, None, stream)
+    else:
+        w = wl.WORKLOADS[args.decode_workload]
+        (q, k, v), (qs, ks, vs) = wl.make_inputs(w)
+        st = sata.State(w.B, w.H, w.d_K, w.d_V, w.P, device=dev, stream=stream)
+        with torch.cuda.stream(stream):
+            sata.prefill(q.to(dev), k.to(dev), v.to(dev), P=w.P, state=st, stream=stream)
+        qs, ks, vs = qs.to(dev), ks.to(dev), vs.to(dev)
+        for i in range(min(args.warmup + args.steps, w.steps)):
+            sata.decode_step(st, qs[i], ks[i], vs[i])
+    torch.cuda.synchronize()
+    status = sata.sata_sync_status(stream)
+    print(json.dumps({"part": args.only, "status": status}), flush=True)
+    return 0 if status == 0 else 1
 
 
 def bench_decode(torch, sata, wl, args, world, dev, stream, peaks, peaks_src):

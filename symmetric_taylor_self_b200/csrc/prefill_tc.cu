@@ -35,62 +35,90 @@
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
+#include <algorithm>
+#include <utility>
+#include <cstring>
+#include <map>
+#include <mutex>
+#include <tuple>
+#include <vector>
+
 #include "sata_internal.h"
 
 namespace sata {
 namespace {
 
 constexpr int kL = 128;               // chunk length (tokens)
-constexpr int kNQ = 2;                // ring stages of alpha*C*phi(q) tiles (shared memory)
-constexpr int kStageBytes = 128 * kL * 2;
-constexpr int kScanThreads = 448;     // 14 warps
-constexpr int kWarpProducer = 0, kWarpMma = 1, kWarpConv0 = 2, kWarpGen0 = 6;
-constexpr int kGenWarps = 8;
+constexpr int kScanThreads = 480;     // 15 warps
+// warp roles: chunk-image producer, readout MMA issuer, state conversion (4), q side (4),
+// k side (4), update MMA issuer
+constexpr int kWarpProducer = 0, kWarpMmaRd = 1, kWarpConv0 = 2, kWarpQ0 = 6, kWarpK0 = 10, kWarpMmaUp = 14;
+constexpr int kKStages = 3;           // ring of (P2k . x_l) operand stages, 32 tokens each
 constexpr int64_t kDefaultWaitNs = 2000000000LL;   // 2 s per wait
 constexpr size_t kPartialBudget = size_t(4) << 30;
 
+// Feature organisation.  With x~ = (x, 1) (index D is the constant 1), the P=4
+// basis is exactly the nondecreasing triples (a <= b <= l) over 0..D: F =
+// binom(D+3, 3).  State rows are grouped by their pair (a, b) and their last
+// index l: a CTA ("unit") owns one tile of 128 pairs (pairs sorted by b, then a)
+// and up to MT values of l.  With P2(x) = x~_a x~_b per pair:
+//   update:  [S|Z]_(pairs, l) += (P2(k) (.) k~_l)^T [V|1]
+//   readout: R += (P2(q) (.) q~_l) . (C/p! * [S|Z]_(pairs, l)),   summed over the unit's l
+// Both feature operands live in TMEM: the pair products are formed once per chunk
+// in registers (one pair row, resp. one token row, per thread) and only scaled by
+// the l column before each store, so no feature tile passes through shared memory.
 template <int DK, int DV>
 struct Cfg {
+    static_assert(DK == DV, "square heads");
+    static constexpr int D = DK;
     static constexpr int NV = DV + 16;                           // MMA N: [V | 1 | 0 pad]
-    static constexpr int MT_MAX = DV == 64 ? 4 : (DV == 32 ? 8 : 12);
-    static constexpr int ROW = kL * 2;                           // one (q/c)^T row: 128 fp16
+    // TMEM: MT state tiles (NV columns each), R (NV), q-side operand (64), k-side ring
+    static constexpr int MT_MAX = (512 - NV - 64 - 16 * kKStages) / NV;
+    static constexpr int ROW = kL * 2;                           // 128 fp16
     static constexpr int KROW = ROW + 16;                        // k^T rows padded so that 32 lanes
                                                                  // reading 32 rows hit distinct banks
+    static constexpr int QS = (D + 1 + 7) / 8 * 8;               // token-major q~ row: D+1 fp16, padded
     static constexpr int IMG_V = NV * ROW;                       // [V|1]^T, K-major SW128
-    static constexpr int OFF_IQ = IMG_V;                         // (q/c)^T, row DK = 1
-    static constexpr int OFF_IK = IMG_V + (DK + 1) * ROW;        // k^T, row DK = 1
-    static constexpr int IMG = OFF_IK + (DK + 1) * KROW;
+    static constexpr int OFF_IQ = IMG_V;                         // q~ = (q/c, 1) token-major [128][QS]
+    static constexpr int OFF_IK = IMG_V + kL * QS * 2;           // k~^T = (k, 1)^T [D+1][KROW]
+    static constexpr int IMG = OFF_IK + (D + 1) * KROW;
     static constexpr int IMG_PAD = (IMG + 1023) / 1024 * 1024;
-    static constexpr int OFF_RING = 2 * IMG_PAD;
-    static constexpr int OFF_BS = OFF_RING + kNQ * kStageBytes;
+    static constexpr int OFF_BS = 2 * IMG_PAD;                   // two fp16 state operands
     static constexpr int BS_BYTES = 128 * NV * 2;
-    static constexpr int OFF_TAB = OFF_BS + 2 * BS_BYTES;
-    static constexpr int OFF_MC = OFF_TAB + MT_MAX * 128 * 4;
-    static constexpr int OFF_BAR = (OFF_MC + MT_MAX * 128 * 2 + 15) / 16 * 16;
-    // barrier indices (pairs are double buffers)
-    static constexpr int B_INF = 0, B_INE = 2, B_QF = 4, B_QE = 6, B_KF = 8, B_KE = 10, B_BSF = 12,
-                         B_BSE = 14, B_SD = 16, B_OF = B_SD + MT_MAX, B_OE = B_OF + 1, B_FIN = B_OE + 1,
-                         N_BAR = B_FIN + 1;
+    static constexpr int OFF_PAIR = OFF_BS + 2 * BS_BYTES;       // uint16 [128]
+    static constexpr int OFF_COEF = OFF_PAIR + 256;              // float [MT_MAX][128]
+    static constexpr int OFF_LV = OFF_COEF + MT_MAX * 128 * 4;   // int [MT_MAX]
+    static constexpr int OFF_BAR = OFF_LV + 64;
+    // barrier indices
+    static constexpr int B_INF = 0, B_INE = 2, B_AQF = 4, B_AQE = 5, B_BSF = 6, B_BSE = 8, B_RE = 10,
+                         B_FIN = 11, B_KF = 12, B_KE = B_KF + kKStages, B_SD = B_KE + kKStages,
+                         B_SR = B_SD + MT_MAX, N_BAR = B_SR + MT_MAX;
     static constexpr int OFF_MISC = OFF_BAR + N_BAR * 8;
     static constexpr int SMEM = OFF_MISC + 16 + 1024;            // + base alignment slack
-    static constexpr int COL_O = MT_MAX * NV;                    // TMEM: readout accumulator
-    static constexpr int COL_A = COL_O + NV;                     // TMEM: two phi(k) stages, 32 columns each
+    static constexpr int COL_R = MT_MAX * NV;                    // TMEM: readout accumulator
+    static constexpr int COL_AQ = COL_R + NV;                    // TMEM: P2(q) (.) q~_l, 64 columns
+    static constexpr int COL_AK = COL_AQ + 64;                   // TMEM: (P2(k) (.) k~_l) ring
     static constexpr int LBO_BS = (NV / 8) * 128;
-    static_assert(COL_A + 64 <= 512, "TMEM columns");
+    static_assert(MT_MAX >= 1 && MT_MAX <= 16, "unit l table");
+    static_assert(COL_AK + 16 * kKStages <= 512, "TMEM columns");
     static_assert(SMEM <= 232448, "shared memory");
     static_assert(NV % 16 == 0, "MMA N");
 };
 
 struct ScanParams {
-    const uint8_t *img;       // [BH][nchunks][IMG]
-    const float *stats;       // [BH][4] max|q|, max|k|, max|v|, max|state|
-    const uint32_t *packed;   // basis: a | b<<8 | l<<16 | p<<24
-    const float *mcoef;       // C/p!
-    float *S, *Z;             // state in/out
-    float *part;              // [BH][G][nc][DV+1][128]
+    const uint8_t *img;         // [BH][nchunks][IMG]
+    const float *stats;         // [BH][4] max|q|, max|k|, max|v|, max|state|
+    const uint16_t *pairs;      // [NPT][128]  a | b << 8
+    const int32_t *unit_k;      // [G] pair tile of each unit
+    const int32_t *unit_nl;     // [G] number of l values
+    const int32_t *unit_l;      // [G][MT_MAX]
+    const float *unit_coef;     // [G][MT_MAX][128] C/p! of feature (pair, l), 0 if none
+    const int32_t *unit_fidx;   // [G][MT_MAX][128] basis index of feature (pair, l), -1 if none
+    float *S, *Z;               // state in/out
+    float *part;                // [BH][G][nc][DV+1][128]
     int *flags;
     int64_t F, N;
-    int BH, G, MT, c0, nc, nchunks, P;
+    int BH, G, c0, nc, nchunks, P;
     int load_state, store_state, stall_chunk;
     float inv_c;
     int64_t wait_ns;
@@ -152,13 +180,6 @@ __device__ __forceinline__ void tc_after() { asm volatile("tcgen05.fence::after_
 __device__ __forceinline__ void tc_commit(uint32_t bar) {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
                  : "memory");
-}
-__device__ __forceinline__ void tc_mma(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d),
-        "l"(a), "l"(b), "r"(idesc), "r"(acc)
-        : "memory");
 }
 // A operand in TMEM (rows on lanes, two fp16 per 32-bit column, even K in the low half).
 __device__ __forceinline__ void tc_mma_ta(uint32_t d, uint32_t a_tmem, uint64_t b, uint32_t idesc, uint32_t acc) {
@@ -246,20 +267,50 @@ struct Waiter {
     }
 };
 
-__device__ __forceinline__ uint4 hmul4(uint4 a, uint4 b) {
-    uint4 r;
-    __half2 *ra = reinterpret_cast<__half2 *>(&a), *rb = reinterpret_cast<__half2 *>(&b),
-            *rr = reinterpret_cast<__half2 *>(&r);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) rr[i] = __hmul2(ra[i], rb[i]);
+// Packed fp16 products on 32-bit registers (round to nearest).
+__device__ __forceinline__ uint32_t hmul2u(uint32_t a, uint32_t b) {
+    uint32_t r;
+    asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
     return r;
 }
-__device__ __forceinline__ uint4 hmul4s(uint4 a, __half2 m) {
-    uint4 r;
-    __half2 *ra = reinterpret_cast<__half2 *>(&a), *rr = reinterpret_cast<__half2 *>(&r);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) rr[i] = __hmul2(ra[i], m);
-    return r;
+// Pair (a, b), a <= b <= D, sorted by b then a: index b (b + 1) / 2 + a; indices
+// past the last pair stand for (D, D).  The host plan uses the same order.
+template <int D>
+struct Pairs {
+    static constexpr int N = (D + 1) * (D + 2) / 2;
+    static constexpr int NT = (N + 127) / 128;
+    __host__ __device__ static constexpr int b(int idx) {
+        if (idx >= N) return D;
+        int v = 0;
+        while ((v + 1) * (v + 2) / 2 <= idx) ++v;
+        return v;
+    }
+    __host__ __device__ static constexpr int a(int idx) { return idx >= N ? D : idx - b(idx) * (b(idx) + 1) / 2; }
+};
+
+// Two fp16 values x~_i0, x~_i1 (indices into a token row held as packed half2
+// registers) as one half2, i0 in the low half.
+template <int I0, int I1, int NX>
+__device__ __forceinline__ uint32_t pick2(const uint32_t (&x)[NX]) {
+    if constexpr (I0 % 2 == 0 && I1 == I0 + 1) {
+        return x[I0 / 2];
+    } else {
+        constexpr uint32_t s0 = (I0 % 2) * 2, s2 = 4 + (I1 % 2) * 2;
+        return __byte_perm(x[I0 / 2], x[I1 / 2], s0 | ((s0 + 1) << 4) | (s2 << 8) | ((s2 + 1) << 12));
+    }
+}
+// P2(q) of one token for pair tile K: pq[m] = (x~_a x~_b) of pairs 2m, 2m+1.
+template <int D, int K, int NX, int... M>
+__device__ __forceinline__ void p2q_tile(const uint32_t (&x)[NX], uint32_t (&pq)[64], std::integer_sequence<int, M...>) {
+    using PT = Pairs<D>;
+    ((pq[M] = hmul2u(pick2<PT::a(K * 128 + 2 * M), PT::a(K * 128 + 2 * M + 1)>(x),
+                     pick2<PT::b(K * 128 + 2 * M), PT::b(K * 128 + 2 * M + 1)>(x))),
+     ...);
+}
+template <int D, int NX, int... K>
+__device__ __forceinline__ void p2q_dispatch(int k, const uint32_t (&x)[NX], uint32_t (&pq)[64],
+                                             std::integer_sequence<int, K...>) {
+    ((k == K ? (p2q_tile<D, K>(x, pq, std::make_integer_sequence<int, 64>{}), 0) : 0), ...);
 }
 
 // ----------------------------------------------------------------- prep ----
@@ -331,18 +382,27 @@ tc_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restr
             const int off = (t8 / 8) * (C::NV * 128) + n * 128 + (((t8 % 8) ^ (n % 8)) * 16);
             *reinterpret_cast<uint4 *>(out + off) = *reinterpret_cast<const uint4 *>(h);
         }
-        // k^T and (q/c)^T: row i holds tokens 0..127; row DK is 1 (0 for padded tokens)
+        // k~^T: row i holds tokens 0..127; row DK is 1 (0 for padded tokens)
         for (int e = tid; e < (DK + 1) * 16; e += 256) {
             const int i = e / 16, t8 = e % 16;
-            __align__(16) __half hk[8], hq[8];
+            __align__(16) __half hk[8];
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
                 const int t = t8 * 8 + j;
                 hk[j] = i < DK ? sk[t * PK + i] : (t < nt ? one : zero);
-                hq[j] = i < DK ? sq[t * PK + i] : (t < nt ? one : zero);
             }
             *reinterpret_cast<uint4 *>(out + C::OFF_IK + i * C::KROW + t8 * 16) = *reinterpret_cast<const uint4 *>(hk);
-            *reinterpret_cast<uint4 *>(out + C::OFF_IQ + i * C::ROW + t8 * 16) = *reinterpret_cast<const uint4 *>(hq);
+        }
+        // q~ token-major: row t holds (q_t / c, 1) then zeros (all zero for padded tokens)
+        for (int e = tid; e < kL * (C::QS / 8); e += 256) {
+            const int t = e / (C::QS / 8), i8 = (e % (C::QS / 8)) * 8;
+            __align__(16) __half hq[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const int i = i8 + j;
+                hq[j] = i < DK ? sq[t * PK + i] : ((i == DK && t < nt) ? one : zero);
+            }
+            *reinterpret_cast<uint4 *>(out + C::OFF_IQ + (t * C::QS + i8) * 2) = *reinterpret_cast<const uint4 *>(hq);
         }
         // per-head maxima (non-negative floats order like their bit patterns)
 #pragma unroll
@@ -388,6 +448,7 @@ template <int DK, int DV>
 __global__ void __launch_bounds__(kScanThreads, 1) tc_scan_kernel(const ScanParams p) {
     using C = Cfg<DK, DV>;
     constexpr int NV = C::NV;
+    constexpr int D = C::D;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sb = smem_u32(smem);
@@ -395,13 +456,16 @@ __global__ void __launch_bounds__(kScanThreads, 1) tc_scan_kernel(const ScanPara
     auto BAR = [bar0](int i) { return bar0 + 8u * (uint32_t)i; };
     volatile uint32_t *tmem_slot = reinterpret_cast<volatile uint32_t *>(smem + C::OFF_MISC);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + C::OFF_MISC + 4);
-    uint32_t *tab = reinterpret_cast<uint32_t *>(smem + C::OFF_TAB);
-    __half *mc = reinterpret_cast<__half *>(smem + C::OFF_MC);
+    uint16_t *sp_pair = reinterpret_cast<uint16_t *>(smem + C::OFF_PAIR);
+    float *sp_coef = reinterpret_cast<float *>(smem + C::OFF_COEF);
+    int *sp_l = reinterpret_cast<int *>(smem + C::OFF_LV);
 
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-    const int64_t bh = blockIdx.x / p.G;
-    const int g = blockIdx.x % p.G;
-    const int64_t f0 = (int64_t)g * p.MT * 128;
+    // unit-major order: every head's largest units are scheduled first
+    const int64_t bh = blockIdx.x % p.BH;
+    const int u = blockIdx.x / p.BH;
+    const int ktile = p.unit_k[u];
+    const int nl = p.unit_nl[u];
     const float mq = p.stats[bh * 4 + 0], mk = p.stats[bh * 4 + 1], mv = p.stats[bh * 4 + 2],
                 ms = p.stats[bh * 4 + 3];
     // fp16 operand range (uniform over the CTA: exit before any barrier or TMEM use)
@@ -413,9 +477,11 @@ __global__ void __launch_bounds__(kScanThreads, 1) tc_scan_kernel(const ScanPara
     if (threadIdx.x == 0) {
         for (int i = 0; i < C::N_BAR; ++i) {
             uint32_t cnt = 1;
-            if (i == C::B_INE || i == C::B_INE + 1) cnt = kGenWarps + 1;
-            else if ((i >= C::B_QF && i < C::B_QF + 2) || (i >= C::B_KF && i < C::B_KF + 2)) cnt = kGenWarps;
-            else if (i == C::B_BSF || i == C::B_BSF + 1 || i == C::B_OE) cnt = 4;
+            if (i == C::B_INE || i == C::B_INE + 1) cnt = 1 + 4 + 4;   // MMA commit, q-side, k-side warps
+            else if (i == C::B_AQF || i == C::B_RE || i == C::B_BSF || i == C::B_BSF + 1) cnt = 4;
+            else if (i >= C::B_KF && i < C::B_KF + kKStages) cnt = 4;
+            else if (i >= C::B_SR && i < C::B_SR + C::MT_MAX) cnt = 4;
+            else if (i == C::B_FIN) cnt = 2;                             // both MMA issuers
             mbar_init(BAR(i), cnt);
         }
         *abort_flag = 0;
@@ -429,15 +495,10 @@ __global__ void __launch_bounds__(kScanThreads, 1) tc_scan_kernel(const ScanPara
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
         tc_before();
     }
-    if (warp >= kWarpGen0) {   // this CTA's feature descriptors
-        const uint32_t pad = (uint32_t)DK | ((uint32_t)DK << 8) | ((uint32_t)DK << 16);
-        for (int i = threadIdx.x - kWarpGen0 * 32; i < C::MT_MAX * 128; i += kGenWarps * 32) {
-            const int64_t f = f0 + i;
-            const bool ok = i < p.MT * 128 && f < p.F;
-            tab[i] = ok ? (p.packed[f] & 0xFFFFFFu) : pad;
-            mc[i] = __float2half_rn(ok ? p.mcoef[f] : 0.f);
-        }
-    }
+    for (int i = threadIdx.x; i < 128; i += blockDim.x) sp_pair[i] = p.pairs[ktile * 128 + i];
+    for (int i = threadIdx.x; i < C::MT_MAX * 128; i += blockDim.x)
+        sp_coef[i] = p.unit_coef[(int64_t)u * C::MT_MAX * 128 + i];
+    for (int i = threadIdx.x; i < C::MT_MAX; i += blockDim.x) sp_l[i] = p.unit_l[u * C::MT_MAX + i];
     __syncthreads();
     tc_after();
     const uint32_t tmem = *tmem_slot;
@@ -459,67 +520,85 @@ __global__ void __launch_bounds__(kScanThreads, 1) tc_scan_kernel(const ScanPara
             for (int ib = 0; ib < 2; ++ib)   // no copy may still be landing at exit
                 if (last[ib] >= 0) W.drain(BAR(C::B_INF + ib), (last[ib] >> 1) & 1);
         }
-    } else if (warp == kWarpMma) {
-        // ------------------------------------------------ MMA issue (one thread)
+    } else if (warp == kWarpMmaRd) {
+        // ------------------------------------------------ readout MMA issue (one thread)
         if (lane == 0) {
-            constexpr uint32_t id_upd = idesc_f16(128, NV, 0, 0);
-            constexpr uint32_t id_rd = idesc_f16(128, NV, 1, 1);
-            int qa = 0, qk = 0;
+            constexpr uint32_t id_rd = idesc_f16(128, NV, 0, 1);    // A TMEM, B MN-major
+            int qa = 0;
             bool ok = true;
             for (int cl = 0; cl < p.nc && ok; ++cl) {
-                const int ib = cl & 1;
-                if (!(ok = W.wait(BAR(C::B_INF + ib), (cl >> 1) & 1))) break;
-                const uint32_t vimg = sb + ib * C::IMG_PAD;
-                for (int j = 0; j < p.MT; ++j) {
-                    const int qn = cl * p.MT + j, bsb = qn & 1, sa = qa & 1;
-                    ok = W.wait(BAR(C::B_BSF + bsb), (qn >> 1) & 1) && W.wait(BAR(C::B_QF + sa), (qa >> 1) & 1);
-                    if (ok && j == 0) ok = W.wait(BAR(C::B_OE), (cl & 1) ^ 1);   // epilogue of cl-1 done
+                for (int j = 0; j < nl; ++j) {
+                    const int bsb = qa & 1;
+                    ok = W.wait(BAR(C::B_BSF + bsb), (qa >> 1) & 1) && W.wait(BAR(C::B_AQF), qa & 1);
+                    if (ok && j == 0 && cl > 0) ok = W.wait(BAR(C::B_RE), (cl - 1) & 1);   // R of cl-1 read
                     if (!ok) break;
                     tc_after();
-                    // readout: D_O += (alpha C phi(q)) [128 t x 128 f] . [S|Z]_j fp16 [128 f x NV]
-                    const uint32_t a_st = sb + C::OFF_RING + sa * kStageBytes;
+                    // R (+)= (P2(q) (.) q~_lj) [128 t x 128 pairs] . (C/p! 2^-s [S|Z])_(pairs, lj) [128 pairs x NV]
                     const uint32_t b_s = sb + C::OFF_BS + bsb * C::BS_BYTES;
 #pragma unroll
                     for (int ks = 0; ks < 8; ++ks)
-                        tc_mma(tmem + C::COL_O, sdesc(a_st + ks * 2048, 16384, 1024, 2),
-                               sdesc(b_s + ks * 2 * C::LBO_BS, C::LBO_BS, 128, 0), id_rd,
-                               (j > 0 || ks > 0) ? 1u : 0u);
-                    tc_commit(BAR(C::B_QE + sa));
+                        tc_mma_ta(tmem + C::COL_R, tmem + C::COL_AQ + ks * 8,
+                                  sdesc(b_s + ks * 2 * C::LBO_BS, C::LBO_BS, 128, 0), id_rd,
+                                  (j > 0 || ks > 0) ? 1u : 0u);
                     tc_commit(BAR(C::B_BSE + bsb));
-                    if (j == p.MT - 1) tc_commit(BAR(C::B_OF));
+                    tc_commit(BAR(C::B_AQE));
                     ++qa;
-                    // update: [S|Z]_j += phi(K)^T [128 f x 64 t] (TMEM) . [V|1] [64 t x NV], two halves
-                    for (int h = 0; h < 2 && ok; ++h) {
-                        const int sk = qk & 1;
-                        if (!(ok = W.wait(BAR(C::B_KF + sk), (qk >> 1) & 1))) break;
-                        tc_after();
-#pragma unroll
-                        for (int ks = 0; ks < 4; ++ks)
-                            tc_mma_ta(tmem + j * NV, tmem + C::COL_A + sk * 32 + ks * 8,
-                                      sdesc(vimg + h * (NV * 128) + ks * 32, 16, 1024, 2), id_upd, 1u);
-                        tc_commit(BAR(C::B_KE + sk));
-                        ++qk;
-                    }
-                    if (!ok) break;
-                    tc_commit(BAR(C::B_SD + j));
                 }
-                if (!ok) break;
-                tc_commit(BAR(C::B_INE + ib));
             }
             // every issued MMA completes before TMEM is released
             tc_commit(BAR(C::B_FIN));
             W.drain(BAR(C::B_FIN), 0);
         }
-    } else if (warp >= kWarpConv0 && warp < kWarpGen0) {
-        // ------------------------------------------------ state conversion + epilogue
+    } else if (warp == kWarpMmaUp) {
+        // ------------------------------------------------ update MMA issue (one thread)
+        if (lane == 0) {
+            constexpr uint32_t id_upd = idesc_f16(128, NV, 0, 0);   // A TMEM, B K-major
+            int st = 0, sph = 0;                                    // k-side ring stage and its phase
+            bool ok = true;
+            for (int cl = 0; cl < p.nc && ok; ++cl) {
+                const int ib = cl & 1;
+                if (!(ok = W.wait(BAR(C::B_INF + ib), (cl >> 1) & 1))) break;
+                const uint32_t vimg = sb + ib * C::IMG_PAD;
+                // [S|Z]_(pairs, lj) += (P2(k) (.) k~_lj) [128 pairs x 32 t] . [V|1] [32 t x NV], by token
+                // quarter qq; tile j is final for this chunk after its last quarter
+                for (int h = 0; h < 2 && ok; ++h) {
+                    for (int j = 0; j < nl && ok; ++j) {
+                        // the state conversion has read tile j before it changes
+                        if (h == 0 && !(ok = W.wait(BAR(C::B_SR + j), cl & 1))) break;
+                        for (int qh = 0; qh < 2; ++qh) {
+                            const int qq = 2 * h + qh;
+                            if (!(ok = W.wait(BAR(C::B_KF + st), sph))) break;
+                            tc_after();
+                            tc_mma_ta(tmem + j * NV, tmem + C::COL_AK + st * 16,
+                                      sdesc(vimg + h * (NV * 128) + qh * 64, 16, 1024, 2), id_upd, 1u);
+                            tc_mma_ta(tmem + j * NV, tmem + C::COL_AK + st * 16 + 8,
+                                      sdesc(vimg + h * (NV * 128) + qh * 64 + 32, 16, 1024, 2), id_upd, 1u);
+                            tc_commit(BAR(C::B_KE + st));
+                            (void)qq;
+                            if (++st == kKStages) {
+                                st = 0;
+                                sph ^= 1;
+                            }
+                        }
+                        if (ok && h == 1) tc_commit(BAR(C::B_SD + j));
+                    }
+                }
+                if (!ok) break;
+                tc_commit(BAR(C::B_INE + ib));
+            }
+            tc_commit(BAR(C::B_FIN));
+            W.drain(BAR(C::B_FIN), 0);
+        }
+    } else if (warp >= kWarpConv0 && warp < kWarpQ0) {
+        // ------------------------------------------------ state -> fp16 readout operand
         const int quarter = warp & 3;
-        const int row = quarter * 32 + lane;
+        const int row = quarter * 32 + lane;            // pair row of the tile = TMEM lane
         const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
         uint32_t r[NV];
         // initial state -> TMEM (zeros for a fresh sequence)
-        for (int j = 0; j < p.MT; ++j) {
-            const int64_t f = f0 + j * 128 + row;
-            const bool have = p.load_state && f < p.F;
+        for (int j = 0; j < nl; ++j) {
+            const int f = p.unit_fidx[((int64_t)u * C::MT_MAX + j) * 128 + row];
+            const bool have = p.load_state && f >= 0;
 #pragma unroll
             for (int col = 0; col < NV; ++col) {
                 float x = 0.f;
@@ -531,61 +610,46 @@ __global__ void __launch_bounds__(kScanThreads, 1) tc_scan_kernel(const ScanPara
             for (int c16 = 0; c16 < NV / 16; ++c16) tc_st16(tmem + lane_off + j * NV + c16 * 16, r + c16 * 16);
         }
         tc_wait_st();
-        int64_t part_base = ((int64_t)bh * p.G + g) * p.nc;
-        auto epilogue = [&](int cl) -> bool {
-            if (!W.wait(BAR(C::B_OF), cl & 1)) return false;
-            tc_after();
-#pragma unroll
-            for (int c16 = 0; c16 < NV / 16; ++c16) tc_ld16(tmem + lane_off + C::COL_O + c16 * 16, r + c16 * 16);
-            tc_wait_ld();
-            tc_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(BAR(C::B_OE));
-            const float up = pow2f(state_sigma(p.c0 + cl, mk, mv, ms, p.P));
-            float *dst = p.part + ((part_base + cl) * (DV + 1)) * kL + row;
-#pragma unroll
-            for (int col = 0; col <= DV; ++col) dst[col * kL] = __uint_as_float(r[col]) * up;
-            return true;
-        };
         bool ok = true;
         for (int cl = 0; cl < p.nc && ok; ++cl) {
             const float down = pow2f(-state_sigma(p.c0 + cl, mk, mv, ms, p.P));
-            for (int j = 0; j < p.MT; ++j) {
-                const int qn = cl * p.MT + j, bsb = qn & 1;
+            for (int j = 0; j < nl; ++j) {
+                const int qn = cl * nl + j, bsb = qn & 1;
                 if (cl > 0 && !(ok = W.wait(BAR(C::B_SD + j), (cl - 1) & 1))) break;
                 tc_after();
 #pragma unroll
                 for (int c16 = 0; c16 < NV / 16; ++c16) tc_ld16(tmem + lane_off + j * NV + c16 * 16, r + c16 * 16);
                 tc_wait_ld();
+                tc_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(BAR(C::B_SR + j));   // tile j read: the update may proceed
                 if (!(ok = W.wait(BAR(C::B_BSE + bsb), ((qn >> 1) & 1) ^ 1))) break;
-                // B_s: [S|Z]_j * 2^-sigma as fp16, K = feature rows, N-major core matrices
+                const float cf = sp_coef[j * 128 + row] * down;
                 uint8_t *bs = smem + C::OFF_BS + bsb * C::BS_BYTES + (row / 8) * C::LBO_BS + (row % 8) * 16;
 #pragma unroll
                 for (int m = 0; m < NV / 8; ++m) {
                     __align__(16) __half2 h[4];
 #pragma unroll
-                    for (int u = 0; u < 4; ++u)
-                        h[u] = __floats2half2_rn(__uint_as_float(r[m * 8 + 2 * u]) * down,
-                                                 __uint_as_float(r[m * 8 + 2 * u + 1]) * down);
+                    for (int w = 0; w < 4; ++w)
+                        h[w] = __floats2half2_rn(__uint_as_float(r[m * 8 + 2 * w]) * cf,
+                                                 __uint_as_float(r[m * 8 + 2 * w + 1]) * cf);
                     *reinterpret_cast<uint4 *>(bs + m * 128) = *reinterpret_cast<const uint4 *>(h);
                 }
                 fence_proxy_async();
                 tc_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(BAR(C::B_BSF + bsb));
-                if (j == 0 && cl > 0 && !(ok = epilogue(cl - 1))) break;
             }
         }
-        if (ok) ok = epilogue(p.nc - 1);
         if (ok && p.store_state) {
-            for (int j = 0; j < p.MT && ok; ++j) {
+            for (int j = 0; j < nl && ok; ++j) {
                 if (!(ok = W.wait(BAR(C::B_SD + j), (p.nc - 1) & 1))) break;
                 tc_after();
 #pragma unroll
                 for (int c16 = 0; c16 < NV / 16; ++c16) tc_ld16(tmem + lane_off + j * NV + c16 * 16, r + c16 * 16);
                 tc_wait_ld();
-                const int64_t f = f0 + j * 128 + row;
-                if (f < p.F) {
+                const int f = p.unit_fidx[((int64_t)u * C::MT_MAX + j) * 128 + row];
+                if (f >= 0) {
                     float4 *dS = reinterpret_cast<float4 *>(p.S + (bh * p.F + f) * DV);
 #pragma unroll
                     for (int c4 = 0; c4 < DV / 4; ++c4)
@@ -596,84 +660,122 @@ __global__ void __launch_bounds__(kScanThreads, 1) tc_scan_kernel(const ScanPara
             }
         }
         tc_before();
-    } else if (warp >= kWarpGen0) {
-        // ------------------------------------------------ feature generation
-        const int gt = threadIdx.x - kWarpGen0 * 32;
-        // alpha*C*phi(q/c) tiles into shared memory: thread = 8 tokens x 8 features
-        const int tg = gt & 15;            // tokens 8*tg .. 8*tg+7
-        const int fgrp = gt >> 4;          // features 8*fgrp .. 8*fgrp+7 of the tile
-        const int xoff = tg * 16;
-        const int hoff = (tg >> 3) * 16384;
-        const int cidx = tg & 7;
-        // phi(k) tiles into TMEM: lane = feature row of the tile, 32 tokens per warp
-        const int kq = warp & 3;                           // TMEM lane quarter of this warp
-        const int krow = kq * 32 + lane;
-        const int ksub = (warp - kWarpGen0) >> 2;          // which 32 tokens of a 64-token stage
+    } else if (warp >= kWarpQ0 && warp < kWarpK0) {
+        // ------------------------------------------------ q side: operand per l, partial per chunk
+        const int quarter = warp & 3;
+        const int t = quarter * 32 + lane;               // token row of the chunk = TMEM lane
+        const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+        const int64_t part_base = ((int64_t)bh * p.G + u) * p.nc;
+        int qa = 0;
+        bool ok = true;
+        // R of chunk cl -> partial (x 2^sigma_cl); the caller has seen the completion of the
+        // chunk's last readout
+        auto drain = [&](int cl) -> bool {
+            tc_after();
+            const float up = pow2f(state_sigma(p.c0 + cl, mk, mv, ms, p.P));
+            float *dst = p.part + ((part_base + cl) * (DV + 1)) * kL + t;
+#pragma unroll
+            for (int c16 = 0; c16 * 16 <= D; ++c16) {
+                uint32_t rr[16];
+                tc_ld16(tmem + lane_off + C::COL_R + c16 * 16, rr);
+                tc_wait_ld();
+#pragma unroll
+                for (int i = 0; i < 16; ++i)
+                    if (c16 * 16 + i <= D) dst[(c16 * 16 + i) * kL] = __uint_as_float(rr[i]) * up;
+            }
+            tc_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(BAR(C::B_RE));
+            return true;
+        };
+        for (int cl = 0; cl < p.nc && ok; ++cl) {
+            const int ib = cl & 1;
+            if (!(ok = W.wait(BAR(C::B_INF + ib), (cl >> 1) & 1))) break;
+            const __half *xq = reinterpret_cast<const __half *>(smem + ib * C::IMG_PAD + C::OFF_IQ) + t * C::QS;
+            // P2(q) of this token for the tile's 128 pairs (even pair in the low half), from
+            // the token's q~ row in registers; pair indices are compile-time per tile
+            uint32_t pq[64];
+            {
+                uint32_t x[C::QS / 2];
+#pragma unroll
+                for (int i = 0; i < C::QS / 8; ++i) {
+                    const uint4 v = reinterpret_cast<const uint4 *>(xq)[i];
+                    x[4 * i] = v.x; x[4 * i + 1] = v.y; x[4 * i + 2] = v.z; x[4 * i + 3] = v.w;
+                }
+                p2q_dispatch<D>(ktile, x, pq, std::make_integer_sequence<int, Pairs<D>::NT>{});
+            }
+            for (int j = 0; j < nl; ++j) {
+                const __half2 ql2 = __half2half2(xq[sp_l[j]]);   // q~_l of this token
+                uint32_t qlb = *reinterpret_cast<const uint32_t *>(&ql2);
+                if (!(ok = W.wait(BAR(C::B_AQE), (qa & 1) ^ 1))) break;
+#pragma unroll
+                for (int c16 = 0; c16 < 4; ++c16) {
+                    // keeps each group's products behind the previous group's store
+                    asm volatile("" : "+r"(qlb));
+                    uint32_t o[16];
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) o[i] = hmul2u(pq[c16 * 16 + i], qlb);
+                    tc_st16(tmem + lane_off + C::COL_AQ + c16 * 16, o);
+                }
+                tc_wait_st();
+                tc_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(BAR(C::B_AQF));
+                ++qa;
+                // R of the previous chunk is complete once this chunk's first operand is out
+                if (j == 0 && cl > 0 && !(ok = drain(cl - 1))) break;
+            }
+            if (!ok) break;
+            __syncwarp();
+            if (lane == 0) mbar_arrive(BAR(C::B_INE + ib));
+        }
+        if (ok && p.nc > 0 && W.wait(BAR(C::B_AQE), (qa & 1) ^ 1)) drain(p.nc - 1);
+        tc_before();
+    } else if (warp >= kWarpK0) {
+        // ------------------------------------------------ k side: (P2(k) (.) k~_l) stages
+        const int kq = warp & 3;
+        const int prow = kq * 32 + lane;                  // pair row of the tile = TMEM lane
         const uint32_t k_lane_off = (uint32_t)(kq * 32) << 16;
-        int qa = 0, qk = 0;
+        const uint32_t pw = sp_pair[prow];
+        const int pa = pw & 255, pb = pw >> 8;
+        int qk = 0;
         bool ok = true;
         for (int cl = 0; cl < p.nc && ok; ++cl) {
             const int ib = cl & 1;
             if (!(ok = W.wait(BAR(C::B_INF + ib), (cl >> 1) & 1))) break;
-            const uint8_t *xq = smem + ib * C::IMG_PAD + C::OFF_IQ;
             const uint8_t *xk = smem + ib * C::IMG_PAD + C::OFF_IK;
-            for (int j = 0; j < p.MT && ok; ++j) {
-                {   // alpha*C*phi(q/c), shared memory, 128-byte swizzled [f][t]
-                    const int sa = qa & 1;
-                    if (!(ok = W.wait(BAR(C::B_QE + sa), ((qa >> 1) & 1) ^ 1))) break;
-                    uint8_t *stage = smem + C::OFF_RING + sa * kStageBytes + hoff;
-                    const uint4 *tj4 = reinterpret_cast<const uint4 *>(tab + j * 128 + fgrp * 8);
-                    const uint4 t_lo = tj4[0], t_hi = tj4[1];
-                    const uint32_t tw[8] = {t_lo.x, t_lo.y, t_lo.z, t_lo.w, t_hi.x, t_hi.y, t_hi.z, t_hi.w};
-                    __align__(16) __half mj[8];
-                    *reinterpret_cast<uint4 *>(mj) = *reinterpret_cast<const uint4 *>(mc + j * 128 + fgrp * 8);
-                    uint32_t prev = 0xFFFFFFFFu;
-                    uint4 pre = make_uint4(0, 0, 0, 0);
+            for (int h = 0; h < 2 && ok; ++h) {
+                uint32_t pk[32];   // P2(k) of this pair over tokens 64h .. 64h+63
 #pragma unroll
-                    for (int i = 0; i < 8; ++i) {
-                        const uint32_t w = tw[i];
-                        if ((w & 0xFFFFu) != prev) {   // new prefix pair (a, b)
-                            prev = w & 0xFFFFu;
-                            const uint4 xa = *reinterpret_cast<const uint4 *>(xq + (w & 255u) * C::ROW + xoff);
-                            const uint4 xb = *reinterpret_cast<const uint4 *>(xq + ((w >> 8) & 255u) * C::ROW + xoff);
-                            pre = hmul4(xa, xb);
-                        }
-                        const uint4 xl = *reinterpret_cast<const uint4 *>(xq + ((w >> 16) & 255u) * C::ROW + xoff);
-                        const uint4 val = hmul4s(hmul4(pre, xl), __half2half2(mj[i]));
-                        const int fr = fgrp * 8 + i;
-                        *reinterpret_cast<uint4 *>(stage + fr * 128 + ((cidx ^ i) << 4)) = val;
-                    }
-                    fence_proxy_async();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(BAR(C::B_QF + sa));
-                    ++qa;
+                for (int g = 0; g < 8; ++g) {
+                    const uint4 xa = *reinterpret_cast<const uint4 *>(xk + pa * C::KROW + (8 * h + g) * 16);
+                    const uint4 xb = *reinterpret_cast<const uint4 *>(xk + pb * C::KROW + (8 * h + g) * 16);
+                    pk[4 * g] = hmul2u(xa.x, xb.x);
+                    pk[4 * g + 1] = hmul2u(xa.y, xb.y);
+                    pk[4 * g + 2] = hmul2u(xa.z, xb.z);
+                    pk[4 * g + 3] = hmul2u(xa.w, xb.w);
                 }
-                {   // phi(k), TMEM: this lane's feature over 32 tokens, per 64-token stage
-                    const uint32_t w = tab[j * 128 + krow];
-                    const uint8_t *ra = xk + (w & 255u) * C::KROW;
-                    const uint8_t *rb = xk + ((w >> 8) & 255u) * C::KROW;
-                    const uint8_t *rl = xk + ((w >> 16) & 255u) * C::KROW;
-                    for (int h = 0; h < 2; ++h) {
-                        const int sk = qk & 1;
-                        if (!(ok = W.wait(BAR(C::B_KE + sk), ((qk >> 1) & 1) ^ 1))) break;
-                        const int tb = (64 * h + 32 * ksub) * 2;   // byte offset of this warp's tokens
-                        uint32_t rr[16];
+                for (int j = 0; j < nl && ok; ++j) {
+                    const uint8_t *xl = xk + sp_l[j] * C::KROW + h * 128;
 #pragma unroll
-                        for (int g8 = 0; g8 < 4; ++g8) {
-                            const uint4 xa = *reinterpret_cast<const uint4 *>(ra + tb + g8 * 16);
-                            const uint4 xb = *reinterpret_cast<const uint4 *>(rb + tb + g8 * 16);
-                            const uint4 xl = *reinterpret_cast<const uint4 *>(rl + tb + g8 * 16);
-                            const uint4 val = hmul4(hmul4(xa, xb), xl);
-                            rr[4 * g8 + 0] = val.x;
-                            rr[4 * g8 + 1] = val.y;
-                            rr[4 * g8 + 2] = val.z;
-                            rr[4 * g8 + 3] = val.w;
+                    for (int qh = 0; qh < 2; ++qh) {
+                        const int st = qk % kKStages;
+                        if (!(ok = W.wait(BAR(C::B_KE + st), ((qk / kKStages) & 1) ^ 1))) break;
+                        uint32_t o[16];
+#pragma unroll
+                        for (int g = 0; g < 4; ++g) {
+                            const int gg = 4 * qh + g;                     // 8-token group of the half
+                            const uint4 x4 = *reinterpret_cast<const uint4 *>(xl + gg * 16);
+                            o[4 * g] = hmul2u(pk[4 * gg], x4.x);
+                            o[4 * g + 1] = hmul2u(pk[4 * gg + 1], x4.y);
+                            o[4 * g + 2] = hmul2u(pk[4 * gg + 2], x4.z);
+                            o[4 * g + 3] = hmul2u(pk[4 * gg + 3], x4.w);
                         }
-                        tc_st16(tmem + k_lane_off + C::COL_A + sk * 32 + 16 * ksub, rr);
+                        tc_st16(tmem + k_lane_off + C::COL_AK + st * 16, o);
                         tc_wait_st();
                         tc_before();
                         __syncwarp();
-                        if (lane == 0) mbar_arrive(BAR(C::B_KF + sk));
+                        if (lane == 0) mbar_arrive(BAR(C::B_KF + st));
                         ++qk;
                     }
                 }
@@ -691,8 +793,6 @@ __global__ void __launch_bounds__(kScanThreads, 1) tc_scan_kernel(const ScanPara
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(512) : "memory");
     }
 }
-
-// --------------------------------------------------------------- finish ----
 
 // Sum the G feature-group partials of every (head, chunk, column, token):
 // part [BH][G][nc][DV+1][128] -> red [BH][nc][DV+1][128].  A pure streaming
@@ -864,24 +964,139 @@ tc_finish_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__res
 
 // ------------------------------------------------------------------ host ----
 
-struct Plan {
-    int MT = 1, G = 1, nchunks = 0, nc_seg = 0;
-    size_t off_stats = 0, off_img = 0, off_part = 0, off_red = 0, off_state = 0, total = 0;
+// Unit plan: which (pair tile, l values) each CTA owns, and per (unit, l slot,
+// row) the basis index and C/p! of feature (a, b, l), or -1 / 0 where the row
+// is no feature (b > l, degree >= P, or a padding pair).
+struct UnitPlan {
+    int D = 0, P = 0, MT = 0, MT_MAX = 0, NPT = 0, G = 0;
+    std::vector<uint16_t> pairs;       // [NPT*128]
+    std::vector<int32_t> unit_k, unit_nl, unit_l;   // [G], [G], [G*MT_MAX]
+    std::vector<float> coef;           // [G*MT_MAX*128]
+    std::vector<int32_t> fidx;         // [G*MT_MAX*128]
+    size_t off_k = 0, off_nl = 0, off_l = 0, off_coef = 0, off_fidx = 0, bytes = 0;
 };
 
 size_t align256(size_t x) { return (x + 255) / 256 * 256; }
 
+bool build_unit_plan(int D, int P, int MT, int MT_MAX, UnitPlan &up) {
+    HostBasis hb;
+    if (!build_basis_host(D, P, hb)) return false;
+    // basis index of each sorted tuple of real indices (indices < D), keyed a | b << 8 | l << 16
+    std::map<uint32_t, int32_t> index_of;
+    for (size_t f = 0; f < hb.tuples.size(); ++f) {
+        uint32_t idx[3] = {(uint32_t)D, (uint32_t)D, (uint32_t)D};
+        for (size_t m = 0; m < hb.tuples[f].size(); ++m) idx[m] = hb.tuples[f][m];
+        index_of[idx[0] | (idx[1] << 8) | (idx[2] << 16)] = (int32_t)f;
+    }
+    up.D = D;
+    up.P = P;
+    up.MT = MT;
+    up.MT_MAX = MT_MAX;
+    const int npair = (D + 1) * (D + 2) / 2;
+    up.NPT = (npair + 127) / 128;
+    up.pairs.assign((size_t)up.NPT * 128, (uint16_t)(D | (D << 8)));
+    std::vector<int> pa(npair), pb(npair);
+    {
+        int i = 0;
+        for (int b = 0; b <= D; ++b)
+            for (int a = 0; a <= b; ++a, ++i) {
+                pa[i] = a;
+                pb[i] = b;
+                up.pairs[i] = (uint16_t)(a | (b << 8));
+            }
+    }
+    struct Unit {
+        int k, nl;
+        int l[16];
+    };
+    std::vector<Unit> units;
+    int64_t covered = 0;
+    for (int k = 0; k < up.NPT; ++k) {
+        std::vector<int> ls;
+        for (int l = 0; l <= D; ++l) {
+            bool any = false;
+            for (int r = 0; r < 128 && !any; ++r) {
+                const int i = k * 128 + r;
+                if (i >= npair || pb[i] > l) continue;
+                const int p = (pa[i] < D) + (pb[i] < D) + (l < D);
+                any = p < P;
+            }
+            if (any) ls.push_back(l);
+        }
+        for (size_t s = 0; s < ls.size(); s += MT) {
+            Unit u{k, 0, {}};
+            for (size_t j = s; j < ls.size() && j < s + MT; ++j) u.l[u.nl++] = ls[j];
+            units.push_back(u);
+        }
+    }
+    std::stable_sort(units.begin(), units.end(), [](const Unit &x, const Unit &y) { return x.nl > y.nl; });
+    up.G = (int)units.size();
+    up.unit_k.resize(up.G);
+    up.unit_nl.resize(up.G);
+    up.unit_l.assign((size_t)up.G * MT_MAX, D);
+    up.coef.assign((size_t)up.G * MT_MAX * 128, 0.f);
+    up.fidx.assign((size_t)up.G * MT_MAX * 128, -1);
+    for (int g = 0; g < up.G; ++g) {
+        const Unit &u = units[g];
+        up.unit_k[g] = u.k;
+        up.unit_nl[g] = u.nl;
+        for (int j = 0; j < u.nl; ++j) {
+            const int l = u.l[j];
+            up.unit_l[(size_t)g * MT_MAX + j] = l;
+            for (int r = 0; r < 128; ++r) {
+                const int i = u.k * 128 + r;
+                if (i >= npair || pb[i] > l) continue;
+                const int p = (pa[i] < D) + (pb[i] < D) + (l < D);
+                if (p >= P) continue;
+                auto it = index_of.find((uint32_t)pa[i] | ((uint32_t)pb[i] << 8) | ((uint32_t)l << 16));
+                if (it == index_of.end()) return false;
+                const size_t at = ((size_t)g * MT_MAX + j) * 128 + r;
+                up.fidx[at] = it->second;
+                // C_p / p! = 1 / prod over runs of equal real indices of (run length)!
+                up.coef[at] = (float)((double)hb.mult[it->second] / (p == 3 ? 6.0 : (p == 2 ? 2.0 : 1.0)));
+                ++covered;
+            }
+        }
+    }
+    if (covered != (int64_t)hb.tuples.size()) return false;   // every feature exactly once
+    up.off_k = align256((size_t)up.NPT * 128 * sizeof(uint16_t));
+    up.off_nl = up.off_k + align256((size_t)up.G * 4);
+    up.off_l = up.off_nl + align256((size_t)up.G * 4);
+    up.off_coef = up.off_l + align256((size_t)up.G * MT_MAX * 4);
+    up.off_fidx = up.off_coef + align256(up.coef.size() * 4);
+    up.bytes = up.off_fidx + align256(up.fidx.size() * 4);
+    return true;
+}
+
+std::mutex g_plan_mu;
+std::map<std::tuple<int, int, int>, UnitPlan> g_plans;
+
+const UnitPlan *unit_plan(int D, int P, int MT, int MT_MAX) {
+    std::lock_guard<std::mutex> lk(g_plan_mu);
+    const auto key = std::make_tuple(D, P, MT);
+    auto it = g_plans.find(key);
+    if (it != g_plans.end()) return &it->second;
+    UnitPlan up;
+    if (!build_unit_plan(D, P, MT, MT_MAX, up)) return nullptr;
+    return &g_plans.emplace(key, std::move(up)).first->second;
+}
+
+struct Plan {
+    const UnitPlan *up = nullptr;
+    int G = 1, nchunks = 0, nc_seg = 0;
+    size_t off_stats = 0, off_img = 0, off_part = 0, off_red = 0, off_state = 0, total = 0;
+};
+
 template <int DK, int DV>
-Plan make_plan(int BH, int64_t N, int64_t F, bool need_state) {
+bool make_plan(int BH, int64_t N, int64_t F, int P, bool need_state, Plan &pl) {
     using C = Cfg<DK, DV>;
-    Plan pl;
-    const int ftiles = (int)((F + 127) / 128);
-    // feature tiles per CTA: as many as fit, unless that leaves fewer than two
-    // CTAs per SM of work
+    // l values per CTA: as many as fit, unless that leaves the SMs without a full wave
     int mt = C::MT_MAX;
-    while (mt > 1 && (int64_t)BH * ((ftiles + mt - 1) / mt) < 2 * 148) --mt;
-    pl.G = (ftiles + mt - 1) / mt;
-    pl.MT = (ftiles + pl.G - 1) / pl.G;
+    const UnitPlan *up = unit_plan(DK, P, mt, C::MT_MAX);
+    while (up && mt > 1 && (int64_t)BH * up->G < 148) up = unit_plan(DK, P, --mt, C::MT_MAX);
+    if (!up) return false;
+    pl.up = up;
+    pl.G = up->G;
     pl.nchunks = (int)((N + kL - 1) / kL);
     const size_t per_chunk = (size_t)BH * pl.G * (DV + 1) * kL * sizeof(float);
     int64_t seg = (int64_t)(kPartialBudget / per_chunk);
@@ -893,7 +1108,8 @@ Plan make_plan(int BH, int64_t N, int64_t F, bool need_state) {
     pl.off_red = pl.off_part + align256(per_chunk * pl.nc_seg);
     pl.off_state = pl.off_red + align256((size_t)BH * (DV + 1) * kL * sizeof(float) * pl.nc_seg);
     pl.total = pl.off_state + (need_state ? align256((size_t)BH * F * (DV + 1) * sizeof(float)) : 0);
-    return pl;
+    (void)F;
+    return true;
 }
 
 template <int DK, int DV>
@@ -903,8 +1119,25 @@ cudaError_t run(const DeviceBasis &basis, int BH, int64_t N, const void *q, cons
     using C = Cfg<DK, DV>;
     const int64_t F = basis.F;
     const bool own_state = (S == nullptr);
-    const Plan pl = make_plan<DK, DV>(BH, N, F, true);
-    if (ws_bytes < make_plan<DK, DV>(BH, N, F, own_state).total) return cudaErrorInvalidValue;
+    Plan pl, need;
+    if (!make_plan<DK, DV>(BH, N, F, basis.P, true, pl) ||
+        !make_plan<DK, DV>(BH, N, F, basis.P, own_state, need))
+        return cudaErrorInvalidValue;
+    if (ws_bytes < need.total) return cudaErrorInvalidValue;
+    const UnitPlan &up = *pl.up;
+    cudaError_t e = cudaSuccess;
+    const uint8_t *tab = (const uint8_t *)device_table(
+        ((uint64_t)DK << 32) | ((uint64_t)basis.P << 16) | (uint64_t)up.MT, up.bytes,
+        [&up](uint8_t *h) {
+            std::memcpy(h, up.pairs.data(), up.pairs.size() * sizeof(uint16_t));
+            std::memcpy(h + up.off_k, up.unit_k.data(), up.unit_k.size() * 4);
+            std::memcpy(h + up.off_nl, up.unit_nl.data(), up.unit_nl.size() * 4);
+            std::memcpy(h + up.off_l, up.unit_l.data(), up.unit_l.size() * 4);
+            std::memcpy(h + up.off_coef, up.coef.data(), up.coef.size() * 4);
+            std::memcpy(h + up.off_fidx, up.fidx.data(), up.fidx.size() * 4);
+        },
+        &e);
+    if (!tab) return e != cudaSuccess ? e : cudaErrorMemoryAllocation;
     uint8_t *w = (uint8_t *)ws;
     float *stats = (float *)(w + pl.off_stats);
     uint8_t *img = w + pl.off_img;
@@ -917,7 +1150,7 @@ cudaError_t run(const DeviceBasis &basis, int BH, int64_t N, const void *q, cons
     const float inv_c = 1.0f / sqrtf((float)DK);
     const auto *qb = (const __nv_bfloat16 *)q, *kb = (const __nv_bfloat16 *)k, *vb = (const __nv_bfloat16 *)v;
 
-    cudaError_t e = cudaMemsetAsync(stats, 0, (size_t)BH * 4 * sizeof(float), stream);
+    e = cudaMemsetAsync(stats, 0, (size_t)BH * 4 * sizeof(float), stream);
     if (e != cudaSuccess) return e;
     const size_t prep_smem = sizeof(__half) * kL * (2 * (DK + 2) + (DV + 2));
     e = cudaFuncSetAttribute(tc_prep_kernel<DK, DV>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)prep_smem);
@@ -947,8 +1180,12 @@ cudaError_t run(const DeviceBasis &basis, int BH, int64_t N, const void *q, cons
         ScanParams sp;
         sp.img = img;
         sp.stats = stats;
-        sp.packed = basis.packed;
-        sp.mcoef = basis.mcoef;
+        sp.pairs = (const uint16_t *)tab;
+        sp.unit_k = (const int32_t *)(tab + up.off_k);
+        sp.unit_nl = (const int32_t *)(tab + up.off_nl);
+        sp.unit_l = (const int32_t *)(tab + up.off_l);
+        sp.unit_coef = (const float *)(tab + up.off_coef);
+        sp.unit_fidx = (const int32_t *)(tab + up.off_fidx);
         sp.S = S;
         sp.Z = Z;
         sp.part = part;
@@ -957,7 +1194,6 @@ cudaError_t run(const DeviceBasis &basis, int BH, int64_t N, const void *q, cons
         sp.N = N;
         sp.BH = BH;
         sp.G = pl.G;
-        sp.MT = pl.MT;
         sp.c0 = s * pl.nc_seg;
         sp.nc = (pl.nchunks - sp.c0 < pl.nc_seg) ? pl.nchunks - sp.c0 : pl.nc_seg;
         sp.nchunks = pl.nchunks;
@@ -994,13 +1230,16 @@ bool prefill_tc_supported(int d_K, int d_V, int P) {
     return d_K == d_V && (d_K == 16 || d_K == 32 || d_K == 64) && P >= 1 && P <= 4;
 }
 
-size_t prefill_tc_workspace_bytes(int BH, int64_t N, int64_t F, int d_K, int d_V, bool need_state) {
+size_t prefill_tc_workspace_bytes(int BH, int64_t N, int64_t F, int d_K, int d_V, int P, bool need_state) {
+    Plan pl;
+    bool ok = false;
     switch (d_K * 1000 + d_V) {
-        case 16016: return make_plan<16, 16>(BH, N, F, need_state).total;
-        case 32032: return make_plan<32, 32>(BH, N, F, need_state).total;
-        case 64064: return make_plan<64, 64>(BH, N, F, need_state).total;
-        default: return 0;
+        case 16016: ok = make_plan<16, 16>(BH, N, F, P, need_state, pl); break;
+        case 32032: ok = make_plan<32, 32>(BH, N, F, P, need_state, pl); break;
+        case 64064: ok = make_plan<64, 64>(BH, N, F, P, need_state, pl); break;
+        default: break;
     }
+    return ok ? pl.total : 0;
 }
 
 cudaError_t launch_prefill_tc(const DeviceBasis &basis, int BH, int64_t N, int d_V, const void *q,

@@ -30,6 +30,7 @@ struct DeviceRes {
     int *flags = nullptr;
     void *ws[4] = {nullptr, nullptr, nullptr, nullptr};
     size_t ws_bytes[4] = {0, 0, 0, 0};
+    std::map<uint64_t, void *> tables;
 };
 std::map<int, DeviceRes> g_dev;
 std::map<std::pair<int, int>, HostBasis> g_host_bases;
@@ -170,6 +171,27 @@ void *device_workspace(int slot, size_t bytes, cudaError_t *err) {
     return r.ws[slot];
 }
 
+const void *device_table(uint64_t key, size_t bytes, const std::function<void(uint8_t *)> &fill,
+                         cudaError_t *err) {
+    std::lock_guard<std::mutex> lk(g_mu);
+    const int dev = current_device(err);
+    if (*err != cudaSuccess) return nullptr;
+    DeviceRes &r = g_dev[dev];
+    auto it = r.tables.find(key);
+    if (it != r.tables.end()) return it->second;
+    std::vector<uint8_t> host(bytes, 0);
+    fill(host.data());
+    void *d = nullptr;
+    *err = cudaMalloc(&d, bytes);
+    if (*err == cudaSuccess) *err = cudaMemcpy(d, host.data(), bytes, cudaMemcpyHostToDevice);
+    if (*err != cudaSuccess) {
+        cudaFree(d);
+        return nullptr;
+    }
+    r.tables[key] = d;
+    return d;
+}
+
 namespace {
 
 size_t prefill_ws_bytes(int BH, int64_t N, int d_K, int d_V, int P, bool need_state, bool *use_tc) {
@@ -178,7 +200,7 @@ size_t prefill_ws_bytes(int BH, int64_t N, int d_K, int d_V, int P, bool need_st
     if (g_opt_prefill_path == 2) tc = true;
     else if (g_opt_prefill_path == 0) tc = prefill_tc_supported(d_K, d_V, P);
     if (use_tc) *use_tc = tc;
-    return tc ? prefill_tc_workspace_bytes(BH, N, F, d_K, d_V, need_state)
+    return tc ? prefill_tc_workspace_bytes(BH, N, F, d_K, d_V, P, need_state)
               : prefill_simt_workspace_bytes(BH, N, F, d_V, need_state);
 }
 
@@ -274,6 +296,7 @@ void sata_shutdown(void) {
         }
         cudaFree(kv.second.flags);
         for (int s = 0; s < 4; ++s) cudaFree(kv.second.ws[s]);
+        for (auto &t : kv.second.tables) cudaFree(t.second);
     }
     g_dev.clear();
     cudaSetDevice(cur);

@@ -2,6 +2,7 @@
 #pragma once
 
 #include <cstdint>
+#include <functional>
 #include <vector>
 
 #include <cuda_runtime.h>
@@ -52,6 +53,10 @@ int record_cuda_error(cudaError_t e);
 const DeviceBasis *device_basis(int d_K, int P, cudaError_t *err);
 int *device_flags(cudaError_t *err);
 void *device_workspace(int slot, size_t bytes, cudaError_t *err);
+// Immutable device table of `bytes` bytes, built once per (device, key): `fill`
+// writes the host image, which is copied to the device.  Freed by sata_shutdown.
+const void *device_table(uint64_t key, size_t bytes, const std::function<void(uint8_t *)> &fill,
+                         cudaError_t *err);
 
 // Kernel identities for launch statistics.
 enum KernelId {
@@ -85,7 +90,7 @@ cudaError_t launch_prefill_simt(const DeviceBasis &basis, int BH, int64_t N, int
 
 // ---- prefill, tensor-core path (prefill_tc.cu) ----
 bool prefill_tc_supported(int d_K, int d_V, int P);
-size_t prefill_tc_workspace_bytes(int BH, int64_t N, int64_t F, int d_K, int d_V, bool need_state);
+size_t prefill_tc_workspace_bytes(int BH, int64_t N, int64_t F, int d_K, int d_V, int P, bool need_state);
 cudaError_t launch_prefill_tc(const DeviceBasis &basis, int BH, int64_t N, int d_V,
                               const void *q, const void *k, const void *v, float *out,
                               float *S, float *Z, bool state_in, void *ws, size_t ws_bytes,

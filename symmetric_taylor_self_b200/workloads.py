@@ -54,6 +54,10 @@ WORKLOADS = {
                             oracle_heads=((0, 0),), oracle_tokens=2048),
     "decode_d32": Workload("decode_d32", B=64, H=32, N=8192, d_K=32, d_V=32, P=4, seed=4,
                            steps=1024, oracle_heads=((0, 0), (63, 31), (17, 5), (40, 22))),
+    # reduced sizes of the two benchmark workloads, for ncu captures
+    "prefill_d64_small": Workload("prefill_d64_small", B=1, H=8, N=8192, d_K=64, d_V=64, P=4, seed=3),
+    "decode_d32_small": Workload("decode_d32_small", B=8, H=32, N=256, d_K=32, d_V=32, P=4, seed=4,
+                                 steps=16),
 }
 
 
