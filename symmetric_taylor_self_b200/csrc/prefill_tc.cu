@@ -181,6 +181,13 @@ __device__ __forceinline__ void tc_commit(uint32_t bar) {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
                  : "memory");
 }
+__device__ __forceinline__ void tc_mma(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d),
+        "l"(a), "l"(b), "r"(idesc), "r"(acc)
+        : "memory");
+}
 // A operand in TMEM (rows on lanes, two fp16 per 32-bit column, even K in the low half).
 __device__ __forceinline__ void tc_mma_ta(uint32_t d, uint32_t a_tmem, uint64_t b, uint32_t idesc, uint32_t acc) {
     asm volatile(
@@ -824,141 +831,223 @@ tc_reduce_kernel(const float4 *__restrict__ part, float4 *__restrict__ red, int 
     }
 }
 
-// Per (head, chunk): sum the feature tiles' inter-chunk partials, add the
-// intra-chunk block sum_{s<=t} w_ts [v_s | 1] (fp32 from the bf16 inputs) and
-// divide.  Partial sums stream with float4 loads, several in flight per thread.
+// Per (head, chunk): the intra-chunk block on tensor cores, plus the division.
+//   S = Q K^T          fp16 operands (the bf16 inputs, exactly), fp32 accumulate in TMEM
+//   W[t][s] = sum_{p<P} (S_ts / c)^p / p!  for s <= t, row t scaled by 2^-e_t, split into two
+//                      fp16 parts W_hi + W_lo (about 22 significant bits: the polynomial's terms can
+//                      cancel, so one fp16 rounding of W is not accurate enough)
+//   O = W_hi [V|1] + W_lo [V|1]   TMEM
+//   out[t] = (2^e_t O_num + num_t) / (2^e_t O_den + den_t), num/den the summed inter-chunk partials
+// One CTA (4 warps, thread = token row) per (head, chunk).
 template <int DK, int DV>
-__global__ void __launch_bounds__(256)
+struct FinCfg {
+    static constexpr int NV = DV + 16;
+    static constexpr int OFF_Q = 0;                // [128 t][64 d] K-major SW128 (d >= DK zero)
+    static constexpr int OFF_K = 16384;            // [128 s][64 d] K-major SW128
+    static constexpr int OFF_W = 32768;            // W_hi [128 t][128 s] K-major SW128, two 64-wide K blocks
+    static constexpr int OFF_WLO = 0;              // W_lo, same layout, over Q and K once S is done
+    static constexpr int OFF_V = 65536;            // [128 s][NV n] MN-major, no swizzle
+    static constexpr int LBO_V = (NV / 8) * 128;
+    static constexpr int OFF_BAR = OFF_V + 128 * NV * 2;
+    static constexpr int SMEM = OFF_BAR + 64 + 1024;
+    static constexpr int STG = DV + 4;             // staging row stride (floats), over Q, K, W
+    static_assert(128 * STG * 4 <= OFF_V, "staging");
+    static_assert(DK <= 64, "head size");
+};
+
+template <int DK, int DV>
+__global__ void __launch_bounds__(128)
 tc_finish_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k,
-                 const __nv_bfloat16 *__restrict__ v, const float *__restrict__ part,
-                 float *__restrict__ out, int BH, int G, int c0, int nc, int64_t N, int P, float inv_c) {
-    constexpr int VP = DV + 1, WP = kL + 1, HW = DV / 2;
-    constexpr int ITEMS = VP * (kL / 4);            // float4 items of one chunk's partial
-    constexpr int PER = (ITEMS + 255) / 256;
-    extern __shared__ float fsm[];
-    float *Ps = fsm;                 // [VP][128]  summed partials (col-major by token)
-    float *fqT = Ps + VP * kL;       // [DK][128]  q^T  (later: staging [128][DV])
-    float *fkT = fqT + DK * kL;      // [DK][128]  k^T  (later: v [128][DV])
-    float *Wt = fkT + DK * kL;       // [128][WP]
-    const int tid = threadIdx.x;
-    const float4 *p4 = reinterpret_cast<const float4 *>(part);
-    for (int64_t idx = blockIdx.x; idx < (int64_t)BH * nc; idx += gridDim.x) {
-        const int64_t bh = idx / nc;
-        const int cl = (int)(idx % nc);
-        const int64_t t0 = (int64_t)(c0 + cl) * kL;
-        const int nt = (int)(N - t0 < kL ? N - t0 : kL);
-        // (1) sum over the G feature-tile groups
-        {
-            const int64_t gstride = (int64_t)nc * ITEMS;
-            const int64_t base = ((int64_t)bh * G * nc + cl) * ITEMS;
-            float4 acc[PER];
+                 const __nv_bfloat16 *__restrict__ v, const float *__restrict__ red, float *__restrict__ out,
+                 int c0, int nc, int64_t N, int P, float inv_c, int *flags, int64_t wait_ns) {
+    using F = FinCfg<DK, DV>;
+    constexpr int NV = F::NV;
+    extern __shared__ uint8_t fraw[];
+    uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(fraw) + 1023) & ~uintptr_t(1023));
+    const uint32_t sb = smem_u32(sm);
+    const uint32_t bar = sb + F::OFF_BAR;
+    volatile uint32_t *tmem_slot = reinterpret_cast<volatile uint32_t *>(sm + F::OFF_BAR + 16);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + F::OFF_BAR + 20);
+    const int tid = threadIdx.x, warp = tid / 32;
+    const int64_t bh = blockIdx.x / nc;
+    const int cl = blockIdx.x % nc;
+    const int64_t t0 = (int64_t)(c0 + cl) * kL;
+    const int nt = (int)(N - t0 < kL ? N - t0 : kL);
+    if (tid == 0) {
+        mbar_init(bar, 1);
+        *abort_flag = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (warp == 0) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                         smem_u32((const void *)tmem_slot)),
+                     "r"(256)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    // ---- operands: bf16 -> fp16 (exact for the accepted input range), swizzled
+    const __half one = __float2half(1.f);
+    for (int e = tid; e < kL * 8; e += 128) {      // Q and K: 8 chunks of 8 d per row
+        const int r = e / 8, c = e % 8;
+        uint4 hq = make_uint4(0, 0, 0, 0), hk = make_uint4(0, 0, 0, 0);
+        if (r < nt && c < DK / 8) {
+            const uint4 bq = *reinterpret_cast<const uint4 *>(q + (bh * N + t0 + r) * DK + c * 8);
+            const uint4 bk = *reinterpret_cast<const uint4 *>(k + (bh * N + t0 + r) * DK + c * 8);
+            const __nv_bfloat16 *pq = reinterpret_cast<const __nv_bfloat16 *>(&bq);
+            const __nv_bfloat16 *pk = reinterpret_cast<const __nv_bfloat16 *>(&bk);
+            __half *oq = reinterpret_cast<__half *>(&hq), *ok2 = reinterpret_cast<__half *>(&hk);
 #pragma unroll
-            for (int u = 0; u < PER; ++u) acc[u] = make_float4(0.f, 0.f, 0.f, 0.f);
-            for (int gg = 0; gg < G; ++gg) {
-                const float4 *src = p4 + base + gg * gstride;
+            for (int i = 0; i < 8; ++i) {
+                oq[i] = __float2half_rn(__bfloat162float(pq[i]));
+                ok2[i] = __float2half_rn(__bfloat162float(pk[i]));
+            }
+        }
+        const int off = r * 128 + ((c ^ (r & 7)) << 4);
+        *reinterpret_cast<uint4 *>(sm + F::OFF_Q + off) = hq;
+        *reinterpret_cast<uint4 *>(sm + F::OFF_K + off) = hk;
+    }
+    for (int e = tid; e < kL * (NV / 8); e += 128) {   // [V|1]: row s, 8 n per 16-byte core row
+        const int r = e / (NV / 8), c = e % (NV / 8);
+        uint4 hv = make_uint4(0, 0, 0, 0);
+        __half *ov = reinterpret_cast<__half *>(&hv);
+        if (r < nt) {
+            if (c < DV / 8) {
+                const uint4 bv = *reinterpret_cast<const uint4 *>(v + (bh * N + t0 + r) * DV + c * 8);
+                const __nv_bfloat16 *pv = reinterpret_cast<const __nv_bfloat16 *>(&bv);
 #pragma unroll
-                for (int u = 0; u < PER; ++u) {
-                    const int item = tid + u * 256;
-                    if (item < ITEMS) {
-                        const float4 x = src[item];
-                        acc[u].x += x.x; acc[u].y += x.y; acc[u].z += x.z; acc[u].w += x.w;
-                    }
+                for (int i = 0; i < 8; ++i) ov[i] = __float2half_rn(__bfloat162float(pv[i]));
+            } else if (c == DV / 8) {
+                ov[0] = one;
+            }
+        }
+        *reinterpret_cast<uint4 *>(sm + F::OFF_V + (r / 8) * F::LBO_V + c * 128 + (r % 8) * 16) = hv;
+    }
+    fence_proxy_async();
+    tc_before();
+    __syncthreads();
+    tc_after();
+    const uint32_t tmem = *tmem_slot;
+    const Waiter W{abort_flag, flags + kFlagTimeout, wait_ns};
+    // ---- S = Q K^T  [128 t x 128 s], K = 64
+    if (tid == 0) {
+        constexpr uint32_t id_s = idesc_f16(128, 128, 0, 0);
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks)
+            tc_mma(tmem, sdesc(sb + F::OFF_Q + ks * 32, 16, 1024, 2), sdesc(sb + F::OFF_K + ks * 32, 16, 1024, 2),
+                   id_s, ks > 0 ? 1u : 0u);
+        tc_commit(bar);
+    }
+    __syncwarp();
+    bool ok = W.wait(bar, 0);
+    tc_after();
+    const int t = tid;                               // token row = TMEM lane
+    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+    // ---- W row t: polynomial, causal mask, power-of-two scale into the fp16 range
+    auto wval = [&](float sv, int s) -> float {
+        const float x = sv * inv_c;
+        float h = 1.f;   // Horner form of sum_{p<P} x^p / p!
+        for (int pp = P - 1; pp >= 1; --pp) h = fmaf(h, x / (float)pp, 1.f);
+        return (s <= t && t < nt) ? h : 0.f;
+    };
+    float wmax = 0.f;
+    if (ok) {
+#pragma unroll 1
+        for (int c16 = 0; c16 < 8; ++c16) {
+            uint32_t rr[16];
+            tc_ld16(tmem + lane_off + c16 * 16, rr);
+            tc_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 16; ++i) wmax = fmaxf(wmax, fabsf(wval(__uint_as_float(rr[i]), c16 * 16 + i)));
+        }
+    }
+    // e_t: 2^-e_t wmax < 2^15
+    const int ebits = (int)((__float_as_uint(wmax) >> 23) & 255) - 127;
+    const int e_t = ebits > 14 ? ebits - 14 : 0;
+    const float down = pow2f(-e_t);
+    if (ok) {
+#pragma unroll 1
+        for (int c16 = 0; c16 < 8; ++c16) {
+            uint32_t rr[16];
+            tc_ld16(tmem + lane_off + c16 * 16, rr);
+            tc_wait_ld();
+#pragma unroll
+            for (int h8 = 0; h8 < 2; ++h8) {
+                __align__(16) __half2 hw[4], lw[4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const int s0 = c16 * 16 + h8 * 8 + 2 * i;
+                    const float w0 = wval(__uint_as_float(rr[h8 * 8 + 2 * i]), s0) * down;
+                    const float w1 = wval(__uint_as_float(rr[h8 * 8 + 2 * i + 1]), s0 + 1) * down;
+                    hw[i] = __floats2half2_rn(w0, w1);
+                    lw[i] = __floats2half2_rn(w0 - __low2float(hw[i]), w1 - __high2float(hw[i]));
                 }
-            }
-#pragma unroll
-            for (int u = 0; u < PER; ++u) {
-                const int item = tid + u * 256;
-                if (item < ITEMS) reinterpret_cast<float4 *>(Ps)[item] = acc[u];
+                const int s8 = c16 * 2 + h8;                                // 8-wide s group 0..15
+                const int off = (s8 / 8) * 16384 + t * 128 + (((s8 % 8) ^ (t & 7)) << 4);
+                *reinterpret_cast<uint4 *>(sm + F::OFF_W + off) = *reinterpret_cast<const uint4 *>(hw);
+                *reinterpret_cast<uint4 *>(sm + F::OFF_WLO + off) = *reinterpret_cast<const uint4 *>(lw);
             }
         }
-        // (2) q^T, k^T in fp32
-        for (int e = tid; e < kL * DK; e += 256) {
-            const int t = e / DK, i = e % DK;
-            float a = 0.f, b = 0.f;
-            if (t < nt) {
-                a = __bfloat162float(q[(bh * N + t0 + t) * DK + i]);
-                b = __bfloat162float(k[(bh * N + t0 + t) * DK + i]);
-            }
-            fqT[i * kL + t] = a;
-            fkT[i * kL + t] = b;
+    }
+    fence_proxy_async();
+    tc_before();
+    __syncthreads();
+    tc_after();
+    // ---- O = (W_hi + W_lo) [V|1]  [128 t x NV], K = 128
+    if (tid == 0 && ok) {
+        constexpr uint32_t id_o = idesc_f16(128, NV, 0, 1);
+#pragma unroll
+        for (int part = 0; part < 2; ++part)
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks)
+                tc_mma(tmem + 128,
+                       sdesc(sb + (part ? F::OFF_WLO : F::OFF_W) + (ks / 4) * 16384 + (ks % 4) * 32, 16, 1024, 2),
+                       sdesc(sb + F::OFF_V + ks * 2 * F::LBO_V, F::LBO_V, 128, 0), id_o, (part | ks) ? 1u : 0u);
+        tc_commit(bar);
+    }
+    __syncwarp();
+    ok = ok && W.wait(bar, 1);
+    tc_after();
+    // ---- epilogue: add the inter-chunk partials, divide, stage the row
+    float *stg = reinterpret_cast<float *>(sm);
+    if (ok) {
+        const float up = pow2f(e_t);
+        const float *rp = red + ((bh * nc + cl) * (DV + 1)) * kL + t;
+        float inv;
+        {   // denominator: column DV
+            uint32_t rr[16];
+            tc_ld16(tmem + 128 + lane_off + DV, rr);
+            tc_wait_ld();
+            inv = 1.f / fmaf(__uint_as_float(rr[0]), up, rp[DV * kL]);
         }
-        __syncthreads();
-        // (3) W[t][s] = sum_{p<P} (q_t.k_s / c)^p / p! for s <= t, by 8x8 blocks
-        {
-            const int tb = tid / 16, sbk = tid % 16;
-            float acc[8][8];
 #pragma unroll
-            for (int a = 0; a < 8; ++a)
+        for (int c16 = 0; c16 < DV / 16; ++c16) {
+            uint32_t rr[16];
+            tc_ld16(tmem + 128 + lane_off + c16 * 16, rr);
+            tc_wait_ld();
 #pragma unroll
-                for (int b = 0; b < 8; ++b) acc[a][b] = 0.f;
-            if (sbk <= tb) {
-                for (int i = 0; i < DK; ++i) {
-                    const float4 qa0 = *reinterpret_cast<const float4 *>(fqT + i * kL + tb * 8);
-                    const float4 qa1 = *reinterpret_cast<const float4 *>(fqT + i * kL + tb * 8 + 4);
-                    const float4 kb0 = *reinterpret_cast<const float4 *>(fkT + i * kL + sbk * 8);
-                    const float4 kb1 = *reinterpret_cast<const float4 *>(fkT + i * kL + sbk * 8 + 4);
-                    const float xa[8] = {qa0.x, qa0.y, qa0.z, qa0.w, qa1.x, qa1.y, qa1.z, qa1.w};
-                    const float xb[8] = {kb0.x, kb0.y, kb0.z, kb0.w, kb1.x, kb1.y, kb1.z, kb1.w};
+            for (int i4 = 0; i4 < 4; ++i4) {
+                float o[4];
 #pragma unroll
-                    for (int a = 0; a < 8; ++a)
-#pragma unroll
-                        for (int b = 0; b < 8; ++b) acc[a][b] = fmaf(xa[a], xb[b], acc[a][b]);
+                for (int i = 0; i < 4; ++i) {
+                    const int j = c16 * 16 + 4 * i4 + i;
+                    o[i] = fmaf(__uint_as_float(rr[4 * i4 + i]), up, rp[j * kL]) * inv;
                 }
+                *reinterpret_cast<float4 *>(stg + t * F::STG + c16 * 16 + 4 * i4) = make_float4(o[0], o[1], o[2], o[3]);
             }
-#pragma unroll
-            for (int a = 0; a < 8; ++a)
-#pragma unroll
-                for (int b = 0; b < 8; ++b) {
-                    const int t = tb * 8 + a, s2 = sbk * 8 + b;
-                    float w = 0.f;
-                    if (s2 <= t && t < nt) {
-                        const float x = acc[a][b] * inv_c;
-                        float h = 1.f;   // Horner form of sum_{p<P} x^p / p!
-                        for (int pp = P - 1; pp >= 1; --pp) h = fmaf(h, x / (float)pp, 1.f);
-                        w = h;
-                    }
-                    Wt[t * WP + s2] = w;
-                }
         }
-        __syncthreads();
-        // (4) v rows (fp32) over k^T's space
-        float *fv = fkT;   // [128][DV]
-        for (int e = tid; e < kL * DV; e += 256) {
-            const int t = e / DV;
-            fv[e] = t < nt ? __bfloat162float(v[(bh * N + t0) * DV + e]) : 0.f;
+    }
+    tc_before();
+    __syncthreads();
+    if (ok) {
+        float4 *o4 = reinterpret_cast<float4 *>(out + (bh * N + t0) * DV);
+        for (int e = tid; e < nt * (DV / 4); e += 128) {
+            const int r = e / (DV / 4), c4 = e % (DV / 4);
+            o4[e] = *reinterpret_cast<const float4 *>(stg + r * F::STG + 4 * c4);
         }
-        __syncthreads();
-        // (5) out[t][j] = (partial num + sum_s W[t][s] v[s][j]) / (partial den + sum_s W[t][s])
-        {
-            const int t = tid % kL, h = tid / kL;
-            float num[HW];
-#pragma unroll
-            for (int jj = 0; jj < HW; ++jj) num[jj] = Ps[(h * HW + jj) * kL + t];
-            float den = Ps[DV * kL + t];
-            for (int s2 = 0; s2 < kL; ++s2) {
-                const float w = Wt[t * WP + s2];
-                den += w;
-                const float *vr = fv + s2 * DV + h * HW;
-#pragma unroll
-                for (int jj = 0; jj < HW; jj += 4) {
-                    const float4 x = *reinterpret_cast<const float4 *>(vr + jj);
-                    num[jj] = fmaf(w, x.x, num[jj]);
-                    num[jj + 1] = fmaf(w, x.y, num[jj + 1]);
-                    num[jj + 2] = fmaf(w, x.z, num[jj + 2]);
-                    num[jj + 3] = fmaf(w, x.w, num[jj + 3]);
-                }
-            }
-            float *stage = fqT;   // [128][DV]
-#pragma unroll
-            for (int jj = 0; jj < HW; ++jj) stage[t * DV + h * HW + jj] = num[jj] / den;
-        }
-        __syncthreads();
-        {
-            const float4 *st4 = reinterpret_cast<const float4 *>(fqT);
-            float4 *o4 = reinterpret_cast<float4 *>(out + (bh * N + t0) * DV);
-            for (int e = tid; e < nt * DV / 4; e += 256) o4[e] = st4[e];
-        }
-        __syncthreads();
+    }
+    if (warp == 0) {
+        tc_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(256) : "memory");
     }
 }
 
@@ -1167,8 +1256,8 @@ cudaError_t run(const DeviceBasis &basis, int BH, int64_t N, const void *q, cons
     }
     e = cudaFuncSetAttribute(tc_scan_kernel<DK, DV>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
     if (e != cudaSuccess) return e;
-    const size_t fin_smem = sizeof(float) * ((size_t)(DV + 1) * kL + (size_t)2 * DK * kL + (size_t)kL * (kL + 1));
-    e = cudaFuncSetAttribute(tc_finish_kernel<DK, DV>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)fin_smem);
+    e = cudaFuncSetAttribute(tc_finish_kernel<DK, DV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             FinCfg<DK, DV>::SMEM);
     if (e != cudaSuccess) return e;
     int stall = -1;
     if (g_opt_test_stall) {
@@ -1214,10 +1303,9 @@ cudaError_t run(const DeviceBasis &basis, int BH, int64_t N, const void *q, cons
             (const float4 *)part, (float4 *)red, BH, pl.G, sp.nc);
         launch_end(kTcReduce, stream);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
-        const int64_t fwork = (int64_t)BH * sp.nc;
         launch_begin(kTcFinish, stream);
-        tc_finish_kernel<DK, DV><<<(int)(fwork < 148 * 16 ? fwork : 148 * 16), 256, fin_smem, stream>>>(
-            qb, kb, vb, red, out, BH, 1, sp.c0, sp.nc, N, basis.P, inv_c);
+        tc_finish_kernel<DK, DV><<<(int)((int64_t)BH * sp.nc), 128, FinCfg<DK, DV>::SMEM, stream>>>(
+            qb, kb, vb, red, out, sp.c0, sp.nc, N, basis.P, inv_c, flags, wait_ns);
         launch_end(kTcFinish, stream);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
