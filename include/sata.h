@@ -155,6 +155,30 @@ SATA_API int sata_prefill_ex(const void *q, const void *k, const void *v, float 
                     sata_state *st, void *workspace, size_t ws_bytes, void *stream);
 
 /*
+ * As sata_prefill_ex, with q, k, v and out in HOST memory (same layouts and
+ * dtypes) and a library-owned workspace.  The same computation as
+ * sata_prefill_ex, so the output is the same; the difference is the transfers:
+ * the call copies the inputs to the device in token segments (at least four
+ * for the tensor-core path) on a library copy stream, starts each segment as
+ * soon as its rows have landed, and copies each segment's output back on a
+ * second copy stream while later segments compute.  Everything is enqueued
+ * behind the work already on `stream`, and `stream` completes only after the
+ * last output row is in host memory.
+ *   q, k, v, out: host pointers, owned by the caller, valid and unmodified
+ *                 until `stream` completes.  Page-locked (pinned) memory lets
+ *                 the copies overlap the kernels; pageable memory works, but
+ *                 the CUDA runtime then stages the copies synchronously.
+ *   st, stream:   as in sata_prefill_ex (st, when given, is device memory).
+ * Device memory: the library keeps device copies of the inputs and the output
+ * (reused by later calls) besides the usual workspace; SATA_ENOMEM if they
+ * cannot be allocated.  Errors otherwise as sata_prefill_ex (no SATA_EALIGN for
+ * the host pointers).
+ */
+SATA_API int sata_prefill_host(const void *q, const void *k, const void *v, float *out,
+                    int B, int H, int64_t N, int d_K, int d_V, int P,
+                    sata_state *st, void *stream);
+
+/*
  * One decode step for every head of `st`, on st->stream: the state absorbs
  * (k, v) and the output is read with q ([CC-TAYLOR] "Feature maps and linear
  * attention": Z_T = Z_{T-1} + phi(k_T), S_T = S_{T-1} + phi(k_T) v_T^T, then

@@ -35,7 +35,7 @@ EXPORTED = (
     "sata_build_basis", "sata_set_stream", "sata_sync_status", "sata_shutdown",
     "sata_state_bytes", "sata_state_init", "sata_workspace_bytes", "sata_prefill",
     "sata_prefill_ex", "sata_decode_step", "sata_set_option", "sata_get_option",
-    "sata_kernel_stats", "sata_reset_kernel_stats", "sata_decode_step_static",
+    "sata_kernel_stats", "sata_reset_kernel_stats", "sata_decode_step_static", "sata_prefill_host",
 )
 
 
@@ -95,6 +95,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "sata_kernel_stats": (i32, [ctypes.POINTER(sata_kernel_stat), i32, ctypes.POINTER(ctypes.c_int)]),
         "sata_reset_kernel_stats": (i32, []),
         "sata_decode_step_static": (i32, [st_p, vp, vp, vp, vp]),
+        "sata_prefill_host": (i32, [vp, vp, vp, vp, i32, i32, i64, i32, i32, i32, st_p, vp]),
     }
     for name, (res, args) in sigs.items():
         fn = getattr(lib, name)
@@ -216,6 +217,17 @@ def sata_prefill_ex(q, k, v, out, B, H, N, d_K, d_V, P, st=None, workspace=None,
     _check(load().sata_prefill_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(out), B, H, N, d_K, d_V, P,
                                   None if st is None else ctypes.byref(st), _ptr(workspace),
                                   ws_bytes, _stream(stream)), "sata_prefill_ex")
+
+
+def sata_prefill_host(q, k, v, out, B, H, N, d_K, d_V, P, st=None, stream=None):
+    """q, k, v, out: CPU tensors (pinned for overlap); the library copies them in
+    and out segment by segment around the kernels (see include/sata.h)."""
+    for t in (q, k, v, out):
+        if t.is_cuda:
+            raise ValueError("sata_prefill_host takes host tensors")
+    _check(load().sata_prefill_host(_ptr(q), _ptr(k), _ptr(v), _ptr(out), B, H, N, d_K, d_V, P,
+                                    None if st is None else ctypes.byref(st), _stream(stream)),
+           "sata_prefill_host")
 
 
 def sata_state_init(st, B, H, d_K, d_V, P, S, Z, stream=None):

@@ -329,7 +329,7 @@ template <int DK, int DV>
 __global__ void __launch_bounds__(256)
 tc_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k,
                const __nv_bfloat16 *__restrict__ v, uint8_t *__restrict__ img,
-               float *__restrict__ stats, int BH, int64_t N, int nchunks, float inv_c) {
+               float *__restrict__ stats, int BH, int64_t N, int nchunks, int cbeg, int ccount, float inv_c) {
     using C = Cfg<DK, DV>;
     constexpr int PK = DK + 2, PV = DV + 2;
     extern __shared__ __half psm[];
@@ -339,9 +339,9 @@ tc_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restr
     __shared__ float red[3][8];
     const int tid = threadIdx.x;
     const __half one = __float2half(1.f), zero = __float2half(0.f);
-    for (int64_t idx = blockIdx.x; idx < (int64_t)BH * nchunks; idx += gridDim.x) {
-        const int64_t bh = idx / nchunks;
-        const int c = (int)(idx % nchunks);
+    for (int64_t idx = blockIdx.x; idx < (int64_t)BH * ccount; idx += gridDim.x) {
+        const int64_t bh = idx / ccount;
+        const int c = cbeg + (int)(idx % ccount);
         const int64_t t0 = (int64_t)c * kL;
         const int nt = (int)(N - t0 < kL ? N - t0 : kL);
         float mq = 0.f, mk = 0.f, mv = 0.f;
@@ -376,7 +376,7 @@ tc_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restr
             }
         }
         __syncthreads();
-        uint8_t *out = img + idx * (int64_t)C::IMG;
+        uint8_t *out = img + (bh * nchunks + c) * (int64_t)C::IMG;
         // [V|1]^T: element (n, t) at (t/64)*(NV*128) + n*128 + ((((t%64)/8) ^ (n%8))*16) + (t%8)*2
         for (int e = tid; e < C::NV * 16; e += 256) {
             const int n = e / 16, t8 = e % 16;
@@ -1177,7 +1177,7 @@ struct Plan {
 };
 
 template <int DK, int DV>
-bool make_plan(int BH, int64_t N, int64_t F, int P, bool need_state, Plan &pl) {
+bool make_plan(int BH, int64_t N, int64_t F, int P, bool need_state, int min_segments, Plan &pl) {
     using C = Cfg<DK, DV>;
     // l values per CTA: as many as fit, unless that leaves the SMs without a full wave
     int mt = C::MT_MAX;
@@ -1190,7 +1190,11 @@ bool make_plan(int BH, int64_t N, int64_t F, int P, bool need_state, Plan &pl) {
     const size_t per_chunk = (size_t)BH * pl.G * (DV + 1) * kL * sizeof(float);
     int64_t seg = (int64_t)(kPartialBudget / per_chunk);
     if (seg < 1) seg = 1;
-    pl.nc_seg = (int)(seg < pl.nchunks ? seg : pl.nchunks);
+    // segments of equal length: as few as the partial budget allows, at least min_segments
+    int64_t nseg = (pl.nchunks + seg - 1) / seg;
+    if (nseg < min_segments) nseg = min_segments < pl.nchunks ? min_segments : pl.nchunks;
+    if (nseg < 1) nseg = 1;
+    pl.nc_seg = (int)((pl.nchunks + nseg - 1) / nseg);
     pl.off_stats = 0;
     pl.off_img = align256((size_t)BH * 4 * sizeof(float));
     pl.off_part = pl.off_img + align256((size_t)BH * pl.nchunks * C::IMG);
@@ -1201,16 +1205,25 @@ bool make_plan(int BH, int64_t N, int64_t F, int P, bool need_state, Plan &pl) {
     return true;
 }
 
+// Enqueue the copy of token rows [t0, t1) of a [BH][N][width] tensor (elem bytes each).
+cudaError_t copy_rows(void *dst, const void *src, int BH, int64_t N, int64_t t0, int64_t t1, int width, int elem,
+                      cudaMemcpyKind kind, cudaStream_t s) {
+    const size_t pitch = (size_t)N * width * elem, off = (size_t)t0 * width * elem;
+    return cudaMemcpy2DAsync((uint8_t *)dst + off, pitch, (const uint8_t *)src + off, pitch,
+                             (size_t)(t1 - t0) * width * elem, BH, kind, s);
+}
+
 template <int DK, int DV>
 cudaError_t run(const DeviceBasis &basis, int BH, int64_t N, const void *q, const void *k, const void *v,
                 float *out, float *S, float *Z, bool state_in, void *ws, size_t ws_bytes, int *flags,
-                cudaStream_t stream) {
+                cudaStream_t stream, const HostIO *io) {
     using C = Cfg<DK, DV>;
     const int64_t F = basis.F;
     const bool own_state = (S == nullptr);
+    const int min_seg = io ? kHostSegments : 1;
     Plan pl, need;
-    if (!make_plan<DK, DV>(BH, N, F, basis.P, true, pl) ||
-        !make_plan<DK, DV>(BH, N, F, basis.P, own_state, need))
+    if (!make_plan<DK, DV>(BH, N, F, basis.P, true, min_seg, pl) ||
+        !make_plan<DK, DV>(BH, N, F, basis.P, own_state, min_seg, need))
         return cudaErrorInvalidValue;
     if (ws_bytes < need.total) return cudaErrorInvalidValue;
     const UnitPlan &up = *pl.up;
@@ -1244,16 +1257,6 @@ cudaError_t run(const DeviceBasis &basis, int BH, int64_t N, const void *q, cons
     const size_t prep_smem = sizeof(__half) * kL * (2 * (DK + 2) + (DV + 2));
     e = cudaFuncSetAttribute(tc_prep_kernel<DK, DV>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)prep_smem);
     if (e != cudaSuccess) return e;
-    const int64_t nwork = (int64_t)BH * pl.nchunks;
-    const int prep_grid = (int)(nwork < 148 * 8 ? nwork : 148 * 8);
-    launch_begin(kTcPrep, stream);
-    tc_prep_kernel<DK, DV><<<prep_grid, 256, prep_smem, stream>>>(qb, kb, vb, img, stats, BH, N, pl.nchunks, inv_c);
-    launch_end(kTcPrep, stream);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    if (state_in) {
-        tc_state_stats_kernel<<<dim3(BH, 8), 256, 0, stream>>>(S, Z, stats, F, DV);
-        if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    }
     e = cudaFuncSetAttribute(tc_scan_kernel<DK, DV>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
     if (e != cudaSuccess) return e;
     e = cudaFuncSetAttribute(tc_finish_kernel<DK, DV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -1265,7 +1268,42 @@ cudaError_t run(const DeviceBasis &basis, int BH, int64_t N, const void *q, cons
         g_opt_test_stall = 0;
     }
     const int64_t wait_ns = g_opt_wait_limit > 0 ? g_opt_wait_limit : kDefaultWaitNs;
+    // events of the host-buffer pipeline; released once enqueued (they live until they complete)
+    std::vector<cudaEvent_t> events;
+    auto new_event = [&events](cudaEvent_t *ev) {
+        cudaError_t r = cudaEventCreateWithFlags(ev, cudaEventDisableTiming);
+        if (r == cudaSuccess) events.push_back(*ev);
+        return r;
+    };
+    struct Release {
+        std::vector<cudaEvent_t> &ev;
+        ~Release() { for (cudaEvent_t x : ev) cudaEventDestroy(x); }
+    } release{events};
     for (int s = 0; s < nseg; ++s) {
+        const int c0s = s * pl.nc_seg;
+        const int ncs = (pl.nchunks - c0s < pl.nc_seg) ? pl.nchunks - c0s : pl.nc_seg;
+        const int64_t tok0 = (int64_t)c0s * kL, tok1 = (int64_t)(c0s + ncs) * kL < N ? (int64_t)(c0s + ncs) * kL : N;
+        if (io) {   // this segment's inputs: host -> device on the copy stream, compute waits for them
+            cudaEvent_t ev;
+            if ((e = copy_rows((void *)q, io->q, BH, N, tok0, tok1, DK, 2, cudaMemcpyHostToDevice, io->h2d)) ||
+                (e = copy_rows((void *)k, io->k, BH, N, tok0, tok1, DK, 2, cudaMemcpyHostToDevice, io->h2d)) ||
+                (e = copy_rows((void *)v, io->v, BH, N, tok0, tok1, DV, 2, cudaMemcpyHostToDevice, io->h2d)) ||
+                (e = new_event(&ev)) || (e = cudaEventRecord(ev, io->h2d)) || (e = cudaStreamWaitEvent(stream, ev, 0)))
+                return e;
+        }
+        {   // chunk images and per-head maxima of this segment (maxima accumulate over segments)
+            const int64_t nwork = (int64_t)BH * ncs;
+            const int prep_grid = (int)(nwork < 148 * 8 ? nwork : 148 * 8);
+            launch_begin(kTcPrep, stream);
+            tc_prep_kernel<DK, DV><<<prep_grid, 256, prep_smem, stream>>>(qb, kb, vb, img, stats, BH, N, pl.nchunks,
+                                                                           c0s, ncs, inv_c);
+            launch_end(kTcPrep, stream);
+            if ((e = cudaGetLastError()) != cudaSuccess) return e;
+            if (s == 0 && state_in) {
+                tc_state_stats_kernel<<<dim3(BH, 8), 256, 0, stream>>>(S, Z, stats, F, DV);
+                if ((e = cudaGetLastError()) != cudaSuccess) return e;
+            }
+        }
         ScanParams sp;
         sp.img = img;
         sp.stats = stats;
@@ -1308,6 +1346,17 @@ cudaError_t run(const DeviceBasis &basis, int BH, int64_t N, const void *q, cons
             qb, kb, vb, red, out, sp.c0, sp.nc, N, basis.P, inv_c, flags, wait_ns);
         launch_end(kTcFinish, stream);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        if (io) {   // this segment's output: device -> host on the second copy stream
+            cudaEvent_t ev;
+            if ((e = new_event(&ev)) || (e = cudaEventRecord(ev, stream)) || (e = cudaStreamWaitEvent(io->d2h, ev, 0)) ||
+                (e = copy_rows(io->out, out, BH, N, tok0, tok1, DV, 4, cudaMemcpyDeviceToHost, io->d2h)))
+                return e;
+        }
+    }
+    if (io) {   // the caller's stream completes after the last copy back
+        cudaEvent_t ev;
+        if ((e = new_event(&ev)) || (e = cudaEventRecord(ev, io->d2h)) || (e = cudaStreamWaitEvent(stream, ev, 0)))
+            return e;
     }
     return cudaSuccess;
 }
@@ -1318,13 +1367,15 @@ bool prefill_tc_supported(int d_K, int d_V, int P) {
     return d_K == d_V && (d_K == 16 || d_K == 32 || d_K == 64) && P >= 1 && P <= 4;
 }
 
-size_t prefill_tc_workspace_bytes(int BH, int64_t N, int64_t F, int d_K, int d_V, int P, bool need_state) {
+size_t prefill_tc_workspace_bytes(int BH, int64_t N, int64_t F, int d_K, int d_V, int P, bool need_state,
+                                  bool host_io) {
     Plan pl;
     bool ok = false;
+    const int ms = host_io ? kHostSegments : 1;
     switch (d_K * 1000 + d_V) {
-        case 16016: ok = make_plan<16, 16>(BH, N, F, P, need_state, pl); break;
-        case 32032: ok = make_plan<32, 32>(BH, N, F, P, need_state, pl); break;
-        case 64064: ok = make_plan<64, 64>(BH, N, F, P, need_state, pl); break;
+        case 16016: ok = make_plan<16, 16>(BH, N, F, P, need_state, ms, pl); break;
+        case 32032: ok = make_plan<32, 32>(BH, N, F, P, need_state, ms, pl); break;
+        case 64064: ok = make_plan<64, 64>(BH, N, F, P, need_state, ms, pl); break;
         default: break;
     }
     return ok ? pl.total : 0;
@@ -1332,11 +1383,11 @@ size_t prefill_tc_workspace_bytes(int BH, int64_t N, int64_t F, int d_K, int d_V
 
 cudaError_t launch_prefill_tc(const DeviceBasis &basis, int BH, int64_t N, int d_V, const void *q,
                               const void *k, const void *v, float *out, float *S, float *Z, bool state_in,
-                              void *ws, size_t ws_bytes, int *flags, cudaStream_t stream) {
+                              void *ws, size_t ws_bytes, int *flags, cudaStream_t stream, const HostIO *io) {
     switch (basis.d_K * 1000 + d_V) {
-        case 16016: return run<16, 16>(basis, BH, N, q, k, v, out, S, Z, state_in, ws, ws_bytes, flags, stream);
-        case 32032: return run<32, 32>(basis, BH, N, q, k, v, out, S, Z, state_in, ws, ws_bytes, flags, stream);
-        case 64064: return run<64, 64>(basis, BH, N, q, k, v, out, S, Z, state_in, ws, ws_bytes, flags, stream);
+        case 16016: return run<16, 16>(basis, BH, N, q, k, v, out, S, Z, state_in, ws, ws_bytes, flags, stream, io);
+        case 32032: return run<32, 32>(basis, BH, N, q, k, v, out, S, Z, state_in, ws, ws_bytes, flags, stream, io);
+        case 64064: return run<64, 64>(basis, BH, N, q, k, v, out, S, Z, state_in, ws, ws_bytes, flags, stream, io);
         default: return cudaErrorNotSupported;
     }
 }

@@ -31,6 +31,7 @@ struct DeviceRes {
     void *ws[4] = {nullptr, nullptr, nullptr, nullptr};
     size_t ws_bytes[4] = {0, 0, 0, 0};
     std::map<uint64_t, void *> tables;
+    cudaStream_t h2d = nullptr, d2h = nullptr;
 };
 std::map<int, DeviceRes> g_dev;
 std::map<std::pair<int, int>, HostBasis> g_host_bases;
@@ -171,6 +172,19 @@ void *device_workspace(int slot, size_t bytes, cudaError_t *err) {
     return r.ws[slot];
 }
 
+cudaError_t device_copy_streams(cudaStream_t *h2d, cudaStream_t *d2h) {
+    std::lock_guard<std::mutex> lk(g_mu);
+    cudaError_t err = cudaSuccess;
+    const int dev = current_device(&err);
+    if (err != cudaSuccess) return err;
+    DeviceRes &r = g_dev[dev];
+    if (!r.h2d && (err = cudaStreamCreateWithFlags(&r.h2d, cudaStreamNonBlocking)) != cudaSuccess) return err;
+    if (!r.d2h && (err = cudaStreamCreateWithFlags(&r.d2h, cudaStreamNonBlocking)) != cudaSuccess) return err;
+    *h2d = r.h2d;
+    *d2h = r.d2h;
+    return cudaSuccess;
+}
+
 const void *device_table(uint64_t key, size_t bytes, const std::function<void(uint8_t *)> &fill,
                          cudaError_t *err) {
     std::lock_guard<std::mutex> lk(g_mu);
@@ -194,14 +208,32 @@ const void *device_table(uint64_t key, size_t bytes, const std::function<void(ui
 
 namespace {
 
-size_t prefill_ws_bytes(int BH, int64_t N, int d_K, int d_V, int P, bool need_state, bool *use_tc) {
+size_t prefill_ws_bytes(int BH, int64_t N, int d_K, int d_V, int P, bool need_state, bool *use_tc,
+                        bool host_io = false) {
     const int64_t F = num_features(d_K, P);
     bool tc = false;
     if (g_opt_prefill_path == 2) tc = true;
     else if (g_opt_prefill_path == 0) tc = prefill_tc_supported(d_K, d_V, P);
     if (use_tc) *use_tc = tc;
-    return tc ? prefill_tc_workspace_bytes(BH, N, F, d_K, d_V, P, need_state)
+    return tc ? prefill_tc_workspace_bytes(BH, N, F, d_K, d_V, P, need_state, host_io)
               : prefill_simt_workspace_bytes(BH, N, F, d_V, need_state);
+}
+
+// Shared argument checks of the prefill entry points (pointers excepted).
+int check_prefill_args(int B, int H, int64_t N, int d_K, int d_V, int P, const sata_state *st, int *BH) {
+    int rc = check_heads(B, H, BH);
+    if (rc) return rc;
+    if (N < 0) return SATA_EINVAL;
+    rc = check_shape(d_K, d_V, P);
+    if (rc) return rc;
+    if (st) {
+        if (st->B != B || st->H != H || st->d_K != d_K || st->d_V != d_V || st->P != P)
+            return SATA_EINVAL;
+        if (!st->S || !st->Z) return SATA_EINVAL;
+        if (!aligned16(st->S) || !aligned16(st->Z)) return SATA_EALIGN;
+    }
+    if (g_opt_prefill_path == 2 && !prefill_tc_supported(d_K, d_V, P)) return SATA_EUNSUPPORTED;
+    return SATA_OK;
 }
 
 }  // namespace
@@ -297,6 +329,8 @@ void sata_shutdown(void) {
         cudaFree(kv.second.flags);
         for (int s = 0; s < 4; ++s) cudaFree(kv.second.ws[s]);
         for (auto &t : kv.second.tables) cudaFree(t.second);
+        if (kv.second.h2d) cudaStreamDestroy(kv.second.h2d);
+        if (kv.second.d2h) cudaStreamDestroy(kv.second.d2h);
     }
     g_dev.clear();
     cudaSetDevice(cur);
@@ -355,22 +389,12 @@ int sata_prefill_ex(const void *q, const void *k, const void *v, float *out, int
                     int64_t N, int d_K, int d_V, int P, sata_state *st, void *workspace,
                     size_t ws_bytes, void *stream) {
     int BH = 0;
-    int rc = check_heads(B, H, &BH);
+    int rc = check_prefill_args(B, H, N, d_K, d_V, P, st, &BH);
     if (rc) return rc;
-    if (N < 0) return SATA_EINVAL;
-    rc = check_shape(d_K, d_V, P);
-    if (rc) return rc;
-    if (st) {
-        if (st->B != B || st->H != H || st->d_K != d_K || st->d_V != d_V || st->P != P)
-            return SATA_EINVAL;
-        if (!st->S || !st->Z) return SATA_EINVAL;
-        if (!aligned16(st->S) || !aligned16(st->Z)) return SATA_EALIGN;
-    }
     if (N == 0 || BH == 0) return SATA_OK;
     if (!q || !k || !v || !out) return SATA_EINVAL;
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return SATA_EALIGN;
     if (workspace && !aligned16(workspace)) return SATA_EALIGN;
-    if (g_opt_prefill_path == 2 && !prefill_tc_supported(d_K, d_V, P)) return SATA_EUNSUPPORTED;
 
     bool use_tc = false;
     const size_t need = prefill_ws_bytes(BH, N, d_K, d_V, P, st == nullptr, &use_tc);
@@ -394,9 +418,61 @@ int sata_prefill_ex(const void *q, const void *k, const void *v, float *out, int
     float *Z = st ? st->Z : nullptr;
     const bool state_in = st != nullptr;
     e = use_tc ? launch_prefill_tc(*basis, BH, N, d_V, q, k, v, out, S, Z, state_in, workspace,
-                                   ws_bytes, flags, s)
+                                   ws_bytes, flags, s, nullptr)
                : launch_prefill_simt(*basis, BH, N, d_V, q, k, v, out, S, Z, state_in, workspace,
                                      ws_bytes, s);
+    if (e != cudaSuccess) return cuda_fail(e);
+    if (st) st->tokens += N;
+    return SATA_OK;
+}
+
+int sata_prefill_host(const void *q, const void *k, const void *v, float *out, int B, int H, int64_t N,
+                      int d_K, int d_V, int P, sata_state *st, void *stream) {
+    int BH = 0;
+    int rc = check_prefill_args(B, H, N, d_K, d_V, P, st, &BH);
+    if (rc) return rc;
+    if (N == 0 || BH == 0) return SATA_OK;
+    if (!q || !k || !v || !out) return SATA_EINVAL;
+    bool use_tc = false;
+    const size_t need = prefill_ws_bytes(BH, N, d_K, d_V, P, st == nullptr, &use_tc, true);
+    cudaError_t e = cudaSuccess;
+    const DeviceBasis *basis = device_basis(d_K, P, &e);
+    if (!basis) return cuda_fail(e);
+    int *flags = device_flags(&e);
+    if (!flags) return cuda_fail(e);
+    // device copies of the inputs and the output (slot 2), then the prefill workspace (slot 0)
+    const size_t nq = (size_t)BH * N * d_K * 2, nv = (size_t)BH * N * d_V * 2, no = (size_t)BH * N * d_V * 4;
+    const size_t a16 = 256;
+    const size_t oq = 0, ok_ = (oq + nq + a16 - 1) / a16 * a16, ov = (ok_ + nq + a16 - 1) / a16 * a16,
+                 oo = (ov + nv + a16 - 1) / a16 * a16, nio = oo + no;
+    uint8_t *io_buf = (uint8_t *)device_workspace(2, nio, &e);
+    if (!io_buf) {
+        g_last_cuda = (int)e;
+        return SATA_ENOMEM;
+    }
+    void *workspace = device_workspace(0, need, &e);
+    if (!workspace) {
+        g_last_cuda = (int)e;
+        return SATA_ENOMEM;
+    }
+    cudaStream_t s = (cudaStream_t)stream;
+    float *S = st ? st->S : nullptr;
+    float *Z = st ? st->Z : nullptr;
+    const bool state_in = st != nullptr;
+    void *dq = io_buf + oq, *dk = io_buf + ok_, *dv = io_buf + ov;
+    float *dout = (float *)(io_buf + oo);
+    if (use_tc) {
+        HostIO io{q, k, v, out, nullptr, nullptr};
+        if ((e = device_copy_streams(&io.h2d, &io.d2h)) != cudaSuccess) return cuda_fail(e);
+        e = launch_prefill_tc(*basis, BH, N, d_V, dq, dk, dv, dout, S, Z, state_in, workspace, need, flags, s, &io);
+    } else {   // CUDA-core path: whole copies around the call
+        if ((e = cudaMemcpyAsync(dq, q, nq, cudaMemcpyHostToDevice, s)) == cudaSuccess &&
+            (e = cudaMemcpyAsync(dk, k, nq, cudaMemcpyHostToDevice, s)) == cudaSuccess &&
+            (e = cudaMemcpyAsync(dv, v, nv, cudaMemcpyHostToDevice, s)) == cudaSuccess &&
+            (e = launch_prefill_simt(*basis, BH, N, d_V, dq, dk, dv, dout, S, Z, state_in, workspace, need, s)) ==
+                cudaSuccess)
+            e = cudaMemcpyAsync(out, dout, no, cudaMemcpyDeviceToHost, s);
+    }
     if (e != cudaSuccess) return cuda_fail(e);
     if (st) st->tokens += N;
     return SATA_OK;

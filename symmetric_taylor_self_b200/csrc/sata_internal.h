@@ -89,11 +89,23 @@ cudaError_t launch_prefill_simt(const DeviceBasis &basis, int BH, int64_t N, int
                                 cudaStream_t stream);
 
 // ---- prefill, tensor-core path (prefill_tc.cu) ----
+// Host-buffer prefill: the kernels read and write the device copies passed as q, k, v, out;
+// each token segment's inputs are copied in on h2d, and its output copied back on d2h,
+// so transfers overlap the other segments' compute.
+struct HostIO {
+    const void *q, *k, *v;   // host [BH][N][d] bf16
+    float *out;              // host [BH][N][d_V] fp32
+    cudaStream_t h2d, d2h;
+};
+constexpr int kHostSegments = 4;   // at least this many segments when copies are pipelined
 bool prefill_tc_supported(int d_K, int d_V, int P);
-size_t prefill_tc_workspace_bytes(int BH, int64_t N, int64_t F, int d_K, int d_V, int P, bool need_state);
+size_t prefill_tc_workspace_bytes(int BH, int64_t N, int64_t F, int d_K, int d_V, int P, bool need_state,
+                                  bool host_io);
 cudaError_t launch_prefill_tc(const DeviceBasis &basis, int BH, int64_t N, int d_V,
                               const void *q, const void *k, const void *v, float *out,
                               float *S, float *Z, bool state_in, void *ws, size_t ws_bytes,
-                              int *flags, cudaStream_t stream);
+                              int *flags, cudaStream_t stream, const HostIO *io);
+// Library-owned copy streams of the current device (non-blocking), created once.
+cudaError_t device_copy_streams(cudaStream_t *h2d, cudaStream_t *d2h);
 
 }  // namespace sata

@@ -119,6 +119,10 @@ def test_argument_validation_needs_no_gpu(lib):
     # state mismatch
     st = bd.sata_state(B=1, H=1, d_K=8, d_V=8, P=3, F=120, S=0x10000, Z=0x10000, stream=None, tokens=0)
     assert lib.sata_prefill_ex(fake, fake, fake, fake, 1, 1, 8, 8, 8, 4, ctypes.byref(st), None, 0, None) == bd.SATA_EINVAL
+    # host-buffer prefill: the same shape checks, host pointers required
+    assert lib.sata_prefill_host(fake, fake, fake, fake, 1, 1, 8, 8, 12, 4, None, None) == bd.SATA_EUNSUPPORTED
+    assert lib.sata_prefill_host(None, fake, fake, fake, 1, 1, 8, 8, 8, 4, None, None) == bd.SATA_EINVAL
+    assert lib.sata_prefill_host(None, None, None, None, 1, 1, 0, 8, 8, 4, None, None) == bd.SATA_OK
     # decode
     assert lib.sata_decode_step(None, fake, fake, fake, fake) == bd.SATA_EINVAL
     st = bd.sata_state(B=1, H=1, d_K=8, d_V=8, P=4, F=999, S=0x10000, Z=0x10000, stream=None, tokens=0)

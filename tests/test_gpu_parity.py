@@ -227,6 +227,52 @@ def test_tensor_core_path_selected_and_multi_segment_state(sata, oracle_mod, d):
     sata.sata_set_option(sata.SATA_OPT_PREFILL_PATH, 0)
 
 
+@pytest.mark.parametrize("path,d,N", [("auto", 64, 1000), ("auto", 32, 300), ("auto", 16, 129),
+                                      ("cuda_core", 8, 300)])
+def test_prefill_host_matches_device_and_oracle(sata, oracle_mod, path, d, N):
+    """sata_prefill_host (host buffers, copies pipelined by token segment) gives
+    the device entry point's result and passes the oracle."""
+    _set_path(sata, path)
+    B, H = 1, 2
+    q, k, v = wl.random_inputs(B, H, N, d, d, seed=700 + d + N)
+    y_dev = sata.prefill(q.cuda(), k.cuda(), v.cuda(), P=4)
+    qh, kh, vh = q.pin_memory(), k.pin_memory(), v.pin_memory()
+    yh = torch.full((B, H, N, d), float("nan"), dtype=torch.float32).pin_memory()
+    stream = torch.cuda.Stream()
+    sata.sata_prefill_host(qh, kh, vh, yh, B, H, N, d, d, 4, None, stream)
+    stream.synchronize()
+    torch.cuda.synchronize()
+    assert sata.sata_sync_status() == 0
+    assert torch.isfinite(yh).all()
+    scale = y_dev.abs().max().item()
+    assert (yh - y_dev.cpu()).abs().max().item() <= 1e-6 * scale
+    _check_heads(yh, _oracle_heads(oracle_mod, q, k, v, 4, [(0, 1)]), what=f"host d={d} N={N}")
+
+
+def test_prefill_host_carries_state(sata, oracle_mod):
+    """Two host-buffer calls on one state equal one call over the whole sequence."""
+    _set_path(sata, "auto")
+    B, H, N, d = 1, 2, 700, 64
+    q, k, v = wl.random_inputs(B, H, N, d, d, seed=77)
+    st = sata.State(B, H, d, d, 4)
+    stream = torch.cuda.Stream()
+    st.set_stream(stream)
+    parts = []
+    for a, b in ((0, 300), (300, N)):
+        yh = torch.empty((B, H, b - a, d), dtype=torch.float32).pin_memory()
+        sata.sata_prefill_host(q[:, :, a:b].contiguous().pin_memory(), k[:, :, a:b].contiguous().pin_memory(),
+                               v[:, :, a:b].contiguous().pin_memory(), yh, B, H, b - a, d, d, 4, st.st, stream)
+        stream.synchronize()
+        parts.append(yh)
+    assert sata.sata_sync_status(stream) == 0
+    assert st.tokens == N
+    y = torch.cat(parts, dim=2)
+    for (b, h), (yr, _, S, Z) in oracle_mod.prefill(q, k, v, 4).items():
+        err, _, _ = token_rel_err(y[b, h].double().numpy(), yr)
+        assert err <= TOL, f"head {h}: {err:.3e}"
+        assert np.abs(st.S[b, h].double().cpu().numpy() - S).max() / np.abs(S).max() <= TOL
+
+
 def test_bounded_wait_reports_timeout(sata):
     """A producer signal withheld on purpose: every wait gives up after the
     limit, the kernel exits cleanly, and the status comes back as SATA_ETIMEOUT;
