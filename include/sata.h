@@ -36,8 +36,14 @@
  *     the cudaError_t).  Device-side conditions (a bounded wait that gave up, an
  *     input outside the prefill's operand range) set a per-device flag that
  *     sata_sync_status() reports.
- *   - Supported: 1 <= d_K <= 128, d_V in {4, 8, 16, 32, 64, 128}, 1 <= P <= 4.
- *     Other values return SATA_EUNSUPPORTED.  There is no CPU fallback.
+ *   - Supported: 1 <= d_K <= 128, d_V in {4, 8, 16, 32, 64, 128}, 1 <= P <= 8
+ *     (P is a tunable hyperparameter: [CC-TAYLOR] "Precision and efficiency
+ *     trade-off" (精度与效率的权衡); [CC-HW] "Taylor-expansion trade-off between
+ *     precision and efficiency" (精度与效率的泰勒展开权衡) weighs P = 8).  The
+ *     tensor-core prefill serves d_K = d_V in
+ *     {16, 32, 64} with P <= 4; every other supported shape runs on the CUDA-core
+ *     prefill (fp32).  sata_decode_step_static takes P <= 4.  Other values return
+ *     SATA_EUNSUPPORTED.  There is no CPU fallback.
  *   - The library-owned workspaces are shared by all calls on a device: calls
  *     that may overlap on different streams must pass their own workspace
  *     (sata_prefill_ex) or be ordered by the caller.

@@ -33,8 +33,8 @@ __global__ void __launch_bounds__(kThreads)
 decode_stream_kernel(float *__restrict__ S, float *__restrict__ Z,
                      const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k,
                      const __nv_bfloat16 *__restrict__ v, const uint32_t *__restrict__ packed,
-                     const float *__restrict__ coef, int d_K, int64_t F,
-                     float *__restrict__ partials) {
+                     const uint32_t *__restrict__ packed_hi, const float *__restrict__ coef, int d_K,
+                     int64_t F, float *__restrict__ partials) {
     constexpr int TPR = DV / 4;              // threads per state row, one float4 each
     constexpr int RPI = kThreads / TPR;      // rows per block iteration
     constexpr int kWarps = kThreads / 32;
@@ -48,7 +48,7 @@ decode_stream_kernel(float *__restrict__ S, float *__restrict__ Z,
     const int nf = (int)(F - f0 < (int64_t)kFG ? F - f0 : (int64_t)kFG);
     const int tid = threadIdx.x;
 
-    // x[d_K] = 1 is the padding index of the packed basis (degree < 3).
+    // x[d_K] = 1 is the padding index of the packed basis.
     for (int i = tid; i <= d_K; i += kThreads) {
         xq[i] = i < d_K ? __bfloat162float(q[bh * d_K + i]) : 1.0f;
         xk[i] = i < d_K ? __bfloat162float(k[bh * d_K + i]) : 1.0f;
@@ -58,8 +58,18 @@ decode_stream_kernel(float *__restrict__ S, float *__restrict__ Z,
     for (int f = tid; f < nf; f += kThreads) {
         const uint32_t pk = packed[f0 + f];
         const int a = pk & 255, b = (pk >> 8) & 255, l = (pk >> 16) & 255;
-        phik[f] = xk[a] * xk[b] * xk[l];
-        aq[f] = coef[f0 + f] * (xq[a] * xq[b] * xq[l]);
+        float fk = xk[a] * xk[b] * xk[l], fq = xq[a] * xq[b] * xq[l];
+        if (packed_hi) {   // degrees above 3: the leading indices
+            const uint32_t ph = packed_hi[f0 + f];
+#pragma unroll
+            for (int m = 0; m < 4; ++m) {
+                const int i = (ph >> (8 * m)) & 255;
+                fk *= xk[i];
+                fq *= xq[i];
+            }
+        }
+        phik[f] = fk;
+        aq[f] = coef[f0 + f] * fq;
     }
     __syncthreads();
 
@@ -147,7 +157,7 @@ cudaError_t launch_dv(const DeviceBasis &basis, int BH, float *S, float *Z, cons
     launch_begin(kDecodeStream, stream);
     decode_stream_kernel<DV><<<grid, kThreads, 0, stream>>>(
         S, Z, (const __nv_bfloat16 *)q, (const __nv_bfloat16 *)k, (const __nv_bfloat16 *)v,
-        basis.packed, basis.coef, basis.d_K, basis.F, partials);
+        basis.packed, basis.packed_hi, basis.coef, basis.d_K, basis.F, partials);
     launch_end(kDecodeStream, stream);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;

@@ -256,7 +256,7 @@ extern "C" int sata_decode_step_static(sata_state *st, const void *q, const void
     if (st->B < 0 || st->H < 0 || st->d_K < 1 || st->d_V < 1 || st->P < 1) return SATA_EINVAL;
     const int64_t bh64 = (int64_t)st->B * st->H;
     const int d_V = st->d_V;
-    if (bh64 > INT32_MAX || st->d_K > kMaxDK || st->P > kMaxP ||
+    if (bh64 > INT32_MAX || st->d_K > kMaxDK || st->P > kMaxPStatic ||
         !(d_V == 4 || d_V == 8 || d_V == 16 || d_V == 32 || d_V == 64 || d_V == 128))
         return SATA_EUNSUPPORTED;
     const int64_t F = num_features(st->d_K, st->P);

@@ -44,7 +44,8 @@ __global__ void __launch_bounds__(kThreads)
 simt_scan_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k,
                  const __nv_bfloat16 *__restrict__ v, float *__restrict__ S,
                  float *__restrict__ Z, const uint32_t *__restrict__ packed,
-                 const float *__restrict__ coef, int d_K, int d_V, int64_t F, int64_t N,
+                 const uint32_t *__restrict__ packed_hi, const float *__restrict__ coef, int d_K, int d_V,
+                 int64_t F, int64_t N,
                  int64_t t0, int T, int Tseg, int load_state, float *__restrict__ partials) {
     extern __shared__ float smem[];
     const int DK1 = d_K + 1, DV1 = d_V + 1;
@@ -98,7 +99,17 @@ simt_scan_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__res
                 const uint32_t w = packed[f0 + f];
                 const int a = w & 255, b = (w >> 8) & 255, l = (w >> 16) & 255;
                 pk = xk[t * DK1 + a] * xk[t * DK1 + b] * xk[t * DK1 + l];
-                pq = coef[f0 + f] * (xq[t * DK1 + a] * xq[t * DK1 + b] * xq[t * DK1 + l]);
+                float fq = xq[t * DK1 + a] * xq[t * DK1 + b] * xq[t * DK1 + l];
+                if (packed_hi) {   // degrees above 3: the leading indices
+                    const uint32_t wh = packed_hi[f0 + f];
+#pragma unroll
+                    for (int m = 0; m < 4; ++m) {
+                        const int i = (wh >> (8 * m)) & 255;
+                        pk *= xk[t * DK1 + i];
+                        fq *= xq[t * DK1 + i];
+                    }
+                }
+                pq = coef[f0 + f] * fq;
             }
             phik[e] = pk;
             aq[e] = pq;
@@ -253,7 +264,7 @@ cudaError_t launch_prefill_simt(const DeviceBasis &basis, int BH, int64_t N, int
         launch_begin(kSimtScan, stream);
         simt_scan_kernel<<<dim3(BH, ntiles), kThreads, smemA, stream>>>(
             (const __nv_bfloat16 *)q, (const __nv_bfloat16 *)k, (const __nv_bfloat16 *)v, S, Z,
-            basis.packed, basis.coef, d_K, d_V, F, N, t0, T, (int)Tseg, load, partials);
+            basis.packed, basis.packed_hi, basis.coef, d_K, d_V, F, N, t0, T, (int)Tseg, load, partials);
         launch_end(kSimtScan, stream);
         e = cudaGetLastError();
         if (e != cudaSuccess) return e;

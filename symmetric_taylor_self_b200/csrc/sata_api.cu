@@ -94,16 +94,22 @@ const DeviceBasis *device_basis(int d_K, int P, cudaError_t *err) {
         return nullptr;
     }
     const int64_t F = hb->offsets[P];
-    std::vector<uint32_t> packed(F);
+    std::vector<uint32_t> packed(F), packed_hi(P > 4 ? F : 0);
     std::vector<float> coef(F), mcoef(F);
     const double c = std::sqrt((double)d_K);
     for (int64_t f = 0; f < F; ++f) {
         const auto &t = hb->tuples[f];
         const int p = (int)t.size();
-        // left-pad to three slots with the index d_K, which the kernels read as 1
+        // last three indices, left-padded with d_K (read as the constant 1)
         uint32_t idx[3] = {(uint32_t)d_K, (uint32_t)d_K, (uint32_t)d_K};
-        for (int m = 0; m < p; ++m) idx[3 - p + m] = t[m];
+        const int lo = p > 3 ? p - 3 : 0;
+        for (int m = lo; m < p; ++m) idx[3 - (p - m)] = t[m];
         packed[f] = idx[0] | (idx[1] << 8) | (idx[2] << 16) | ((uint32_t)p << 24);
+        if (P > 4) {   // leading indices of a degree > 3 tuple
+            uint32_t hi[4] = {(uint32_t)d_K, (uint32_t)d_K, (uint32_t)d_K, (uint32_t)d_K};
+            for (int m = 0; m < lo; ++m) hi[m] = t[m];
+            packed_hi[f] = hi[0] | (hi[1] << 8) | (hi[2] << 16) | (hi[3] << 24);
+        }
         double pf = 1.0;
         for (int i = 2; i <= p; ++i) pf *= i;
         mcoef[f] = (float)((double)hb->mult[f] / pf);
@@ -115,6 +121,9 @@ const DeviceBasis *device_basis(int d_K, int P, cudaError_t *err) {
     db.F = F;
     for (int p = 0; p <= P; ++p) db.offsets[p] = hb->offsets[p];
     *err = cudaMalloc(&db.packed, F * sizeof(uint32_t));
+    if (*err == cudaSuccess && P > 4) *err = cudaMalloc(&db.packed_hi, F * sizeof(uint32_t));
+    if (*err == cudaSuccess && P > 4)
+        *err = cudaMemcpy(db.packed_hi, packed_hi.data(), F * sizeof(uint32_t), cudaMemcpyHostToDevice);
     if (*err == cudaSuccess) *err = cudaMalloc(&db.coef, F * sizeof(float));
     if (*err == cudaSuccess) *err = cudaMalloc(&db.mcoef, F * sizeof(float));
     if (*err == cudaSuccess)
@@ -125,6 +134,7 @@ const DeviceBasis *device_basis(int d_K, int P, cudaError_t *err) {
         *err = cudaMemcpy(db.mcoef, mcoef.data(), F * sizeof(float), cudaMemcpyHostToDevice);
     if (*err != cudaSuccess) {
         cudaFree(db.packed);
+        cudaFree(db.packed_hi);
         cudaFree(db.coef);
         cudaFree(db.mcoef);
         return nullptr;
@@ -323,6 +333,7 @@ void sata_shutdown(void) {
         cudaDeviceSynchronize();
         for (auto &b : kv.second.bases) {
             cudaFree(b.second.packed);
+            cudaFree(b.second.packed_hi);
             cudaFree(b.second.coef);
             cudaFree(b.second.mcoef);
         }

@@ -13,7 +13,8 @@ namespace sata {
 
 constexpr int kMaxDK = 128;
 constexpr int kMaxDV = 128;
-constexpr int kMaxP = 4;      // degrees 0..3: packed tables hold three indices
+constexpr int kMaxP = 8;      // degrees 0..7: a feature is at most seven indices (two packed words)
+constexpr int kMaxPStatic = 4;   // the allocation-free decode step derives its basis for P <= 4
 
 // Host copy of the basis (sata_build_basis serves from it).
 struct HostBasis {
@@ -29,16 +30,21 @@ int64_t num_features(int d_K, int P);
 bool build_basis_host(int d_K, int P, HostBasis &hb);
 
 // Device copy of the basis for the kernels, cached per (device, d_K, P).
-//   packed[f] = a | b << 8 | l << 16 | p << 24: feature f is x[a] * x[b] * x[l]
-//   where index d_K stands for the constant 1 (degree-p tuples are left-padded
-//   with it, so every feature is a "prefix pair (a, b) times a last index l").
+//   packed[f] = a | b << 8 | l << 16 | p << 24: the feature's last three indices,
+//   where index d_K stands for the constant 1 (tuples of degree < 3 are
+//   left-padded with it, so every feature is a "prefix pair (a, b) times a last
+//   index l");
+//   packed_hi[f] (only when P > 4, else null) = its leading indices i0..i3 of a
+//   degree-p tuple, p > 3 (i0 | i1 << 8 | i2 << 16 | i3 << 24, padded with d_K):
+//   feature f = x[packed_hi] * x[a] * x[b] * x[l].
 //   coef[f]  = alpha_p * C_p[f] = C_p[f] / (p! c^p), c = sqrt(d_K)  (fp32)
 //   mcoef[f] = C_p[f] / p! = 1 / prod(mult!)                     (fp32)
 struct DeviceBasis {
     int d_K = 0, P = 0;
     int64_t F = 0;
-    int64_t offsets[kMaxP + 1] = {0, 0, 0, 0, 0};
+    int64_t offsets[kMaxP + 1] = {0, 0, 0, 0, 0, 0, 0, 0, 0};
     uint32_t *packed = nullptr;
+    uint32_t *packed_hi = nullptr;
     float *coef = nullptr;
     float *mcoef = nullptr;
 };

@@ -61,13 +61,15 @@ def test_status_strings(lib):
     assert lib.sata_version() >= 10000
 
 
-@pytest.mark.parametrize("d,P", [(1, 1), (1, 4), (2, 3), (8, 4), (16, 4), (32, 4), (64, 4), (128, 4), (5, 6)])
+@pytest.mark.parametrize("d,P", [(1, 1), (1, 4), (2, 3), (8, 4), (16, 4), (32, 4), (64, 4), (128, 4), (5, 6),
+                                 (8, 8), (16, 6)])
 def test_num_features(lib, d, P):
     from symmetric_taylor_self_b200 import sata_num_features
     assert sata_num_features(d, P) == math.comb(d + P - 1, P - 1)
 
 
-@pytest.mark.parametrize("d,P", [(1, 4), (2, 2), (3, 4), (8, 4), (16, 4), (32, 4), (64, 4), (7, 5)])
+@pytest.mark.parametrize("d,P", [(1, 4), (2, 2), (3, 4), (8, 4), (16, 4), (32, 4), (64, 4), (7, 5), (4, 8),
+                                 (8, 6)])
 def test_basis_matches_oracle_bit_exact(lib, oracle_mod, d, P):
     from symmetric_taylor_self_b200 import sata_build_basis
     M, C, off = sata_build_basis(d, P)
@@ -104,7 +106,7 @@ def test_argument_validation_needs_no_gpu(lib):
     fake = vp(0x10000)           # never dereferenced: checks fail before any launch
     # unsupported shapes
     assert lib.sata_prefill_ex(fake, fake, fake, fake, 1, 1, 8, 8, 12, 4, None, None, 0, None) == bd.SATA_EUNSUPPORTED
-    assert lib.sata_prefill_ex(fake, fake, fake, fake, 1, 1, 8, 8, 8, 5, None, None, 0, None) == bd.SATA_EUNSUPPORTED
+    assert lib.sata_prefill_ex(fake, fake, fake, fake, 1, 1, 8, 8, 8, 9, None, None, 0, None) == bd.SATA_EUNSUPPORTED
     assert lib.sata_prefill_ex(fake, fake, fake, fake, 1, 1, 8, 256, 8, 4, None, None, 0, None) == bd.SATA_EUNSUPPORTED
     # invalid values
     assert lib.sata_prefill_ex(fake, fake, fake, fake, -1, 1, 8, 8, 8, 4, None, None, 0, None) == bd.SATA_EINVAL
@@ -169,6 +171,9 @@ def test_static_decode_rejects_oversized_requests_before_any_cuda_call(lib):
     st = bd.sata_state(B=B, H=H, d_K=d, d_V=d, P=4, F=F, S=0x10000, Z=0x10000, stream=None, tokens=0)
     assert lib.sata_decode_step_static(ctypes.byref(st), fake, fake, fake, fake) == bd.SATA_ENOMEM
     assert st.tokens == 0
+    # the allocation-free step derives its basis for P <= 4 only
+    st5 = bd.sata_state(B=1, H=1, d_K=8, d_V=8, P=5, F=math.comb(12, 4), S=0x10000, Z=0x10000, stream=None, tokens=0)
+    assert lib.sata_decode_step_static(ctypes.byref(st5), fake, fake, fake, fake) == bd.SATA_EUNSUPPORTED
     # invalid arguments are rejected the same way as by sata_decode_step
     assert lib.sata_decode_step_static(None, fake, fake, fake, fake) == bd.SATA_EINVAL
     st.F = 7

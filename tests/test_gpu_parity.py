@@ -69,6 +69,24 @@ def test_prefill_lower_P(sata, oracle_mod, P):
     _check_heads(y, ref, what=f"P={P}")
 
 
+@pytest.mark.parametrize("d,P,N", [(4, 5, 200), (8, 6, 150), (4, 8, 130), (8, 8, 40)])
+def test_prefill_and_decode_higher_P(sata, oracle_mod, d, P, N):
+    """P > 4 (seven-index features): CUDA-core prefill over N tokens, then three
+    decode steps, against the oracle's recurrence over all N + 3 tokens."""
+    _set_path(sata, "auto")
+    B, H, steps = 1, 2, 3
+    q, k, v = wl.random_inputs(B, H, N + steps, d, d, seed=900 + 10 * d + P)
+    st = sata.State(B, H, d, d, P)
+    y = sata.prefill(q[:, :, :N].contiguous().cuda(), k[:, :, :N].contiguous().cuda(),
+                     v[:, :, :N].contiguous().cuda(), P=P, state=st)
+    ys = [sata.decode_step(st, q[:, :, N + i].contiguous().cuda(), k[:, :, N + i].contiguous().cuda(),
+                           v[:, :, N + i].contiguous().cuda()) for i in range(steps)]
+    torch.cuda.synchronize()
+    assert sata.sata_sync_status() == 0
+    yall = torch.cat([y, torch.stack(ys, dim=2)], dim=2)
+    _check_heads(yall, _oracle_heads(oracle_mod, q, k, v, P, [(0, 0), (0, 1)]), what=f"d={d} P={P}")
+
+
 @pytest.mark.parametrize("name", ["tiny_d8", "prefill_d16"])
 def test_prefill_workload_all_heads(sata, oracle_mod, name):
     _set_path(sata, "auto")
