@@ -87,6 +87,24 @@ def test_prefill_and_decode_higher_P(sata, oracle_mod, d, P, N):
     _check_heads(yall, _oracle_heads(oracle_mod, q, k, v, P, [(0, 0), (0, 1)]), what=f"d={d} P={P}")
 
 
+@pytest.mark.parametrize("d_K,d_V,N", [(32, 64, 150), (64, 16, 140), (128, 128, 20), (12, 8, 90)])
+def test_prefill_and_decode_other_head_sizes(sata, oracle_mod, d_K, d_V, N):
+    """Head sizes outside the tensor-core set (d_K != d_V, d = 128, odd d_K) run on
+    the CUDA-core prefill; prefill plus two decode steps against the oracle."""
+    _set_path(sata, "auto")
+    B, H, steps = 1, 1, 2
+    q, k, v = wl.random_inputs(B, H, N + steps, d_K, d_V, seed=1300 + d_K + d_V)
+    st = sata.State(B, H, d_K, d_V, 4)
+    y = sata.prefill(q[:, :, :N].contiguous().cuda(), k[:, :, :N].contiguous().cuda(),
+                     v[:, :, :N].contiguous().cuda(), P=4, state=st)
+    ys = [sata.decode_step(st, q[:, :, N + i].contiguous().cuda(), k[:, :, N + i].contiguous().cuda(),
+                           v[:, :, N + i].contiguous().cuda()) for i in range(steps)]
+    torch.cuda.synchronize()
+    assert sata.sata_sync_status() == 0
+    yall = torch.cat([y, torch.stack(ys, dim=2)], dim=2)
+    _check_heads(yall, _oracle_heads(oracle_mod, q, k, v, 4, [(0, 0)]), what=f"d_K={d_K} d_V={d_V}")
+
+
 @pytest.mark.parametrize("name", ["tiny_d8", "prefill_d16"])
 def test_prefill_workload_all_heads(sata, oracle_mod, name):
     _set_path(sata, "auto")
