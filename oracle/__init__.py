@@ -63,6 +63,9 @@ def _load():
             lib.oracle_direct.restype = ctypes.c_int
             lib.oracle_direct.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_double,
                                           ctypes.c_longlong, _dp, _dp, _dp, _dp, _dp, _dp]
+            lib.oracle_direct_grad.restype = ctypes.c_int
+            lib.oracle_direct_grad.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_double,
+                                               ctypes.c_longlong, _dp, _dp, _dp, _dp, _dp, _dp, _dp]
             lib.oracle_softmax.restype = ctypes.c_int
             lib.oracle_softmax.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_double,
                                            ctypes.c_longlong, _dp, _dp, _dp, _dp]
@@ -161,6 +164,42 @@ def direct(q, k, v, P: int, c: float | None = None):
     _check(_load().oracle_direct(dK, dV, P, c, T, _ptr(q), _ptr(k), _ptr(v), _ptr(y), _ptr(den),
                                  _ptr(kappa)), "direct")
     return y, den, kappa
+
+
+def direct_grad(q, k, v, dy, P: int, c: float | None = None):
+    """Gradient of sum(dy * y) for the direct form of one head: (dq, dk, dv).
+
+    q, k: [T, d_K]; v, dy: [T, d_V].  The exact chain rule through y = num/den
+    (the pages define no backward pass; see ``oracle_direct_grad``)."""
+    q, k, v, dy = _f64(q), _f64(k), _f64(v), _f64(dy)
+    T, dK = q.shape
+    dV = v.shape[1]
+    c = default_c(dK) if c is None else float(c)
+    dq = np.zeros((T, dK))
+    dk = np.zeros((T, dK))
+    dv = np.zeros((T, dV))
+    _check(_load().oracle_direct_grad(dK, dV, P, c, T, _ptr(q), _ptr(k), _ptr(v), _ptr(dy),
+                                      _ptr(dq), _ptr(dk), _ptr(dv)), "direct_grad")
+    return dq, dk, dv
+
+
+def grad_heads(q, k, v, dy, P: int, heads=None, T: int | None = None, threads: int | None = None,
+               c: float | None = None):
+    """``direct_grad`` for several heads of [B, H, N, d] inputs in parallel threads.
+
+    Returns {(b, h): (dq, dk, dv)} over the first T tokens of each head."""
+    q, k, v, dy = _f64(q), _f64(k), _f64(v), _f64(dy)
+    B, H, N, _ = q.shape
+    T = N if T is None else int(T)
+    heads = [(b, h) for b in range(B) for h in range(H)] if heads is None else list(heads)
+    threads = threads or len(os.sched_getaffinity(0))
+
+    def one(bh):
+        b, h = bh
+        return bh, direct_grad(q[b, h, :T], k[b, h, :T], v[b, h, :T], dy[b, h, :T], P, c)
+
+    with ThreadPoolExecutor(max_workers=threads) as ex:
+        return dict(ex.map(one, heads))
 
 
 def softmax(q, k, v, c: float | None = None) -> np.ndarray:

@@ -243,6 +243,81 @@ int oracle_direct(int dK, int dV, int P, double c, long long T,
 }
 
 /*
+ * Gradient of the loss L = sum_t dy_t . y_t with respect to q, k and v, for the
+ * masked direct form above.  The pages define no backward pass; they expect the
+ * attention to be trained inside ordinary Transformer pipelines ([CC-TAYLOR]
+ * "Comparison with other methods"; end-to-end training is listed under "Future
+ * directions").  The reading taken: the exact chain-rule gradient of
+ *   y_t = num_t / den_t,  num_t = sum_{s<=t} w_ts v_s,  den_t = sum_{s<=t} w_ts,
+ *   w_ts = T_P(x_ts) = sum_{p<P} x_ts^p / p!,  x_ts = q_t . k_s / c,
+ * with the inputs taken as real numbers.  Written out:
+ *   g_t = dy_t / den_t,  e_t = -(dy_t . y_t) / den_t    (through num and den)
+ *   dw_ts = g_t . v_s + e_t
+ *   dv_s += w_ts g_t
+ *   dx_ts = dw_ts * T_{P-1}(x_ts)      (d/dx T_P = T_{P-1}; T_0 = 0)
+ *   dq_t += dx_ts k_s / c,  dk_s += dx_ts q_t / c
+ * over every pair s <= t.  Outputs are overwritten.  dq, dk are [T][d_K], dv is
+ * [T][d_V].
+ */
+int oracle_direct_grad(int dK, int dV, int P, double c, long long T,
+                       const double *q, const double *k, const double *v, const double *dy,
+                       double *dq, double *dk, double *dv) {
+    if (dK < 1 || dV < 1 || P < 1 || T < 0) return -1;
+    if (T > 0 && (!q || !k || !v || !dy || !dq || !dk || !dv)) return -1;
+    double *y = (double *)malloc(sizeof(double) * (T > 0 ? T * dV : 1));
+    double *den = (double *)malloc(sizeof(double) * (T > 0 ? T : 1));
+    double *g = (double *)malloc(sizeof(double) * dV);
+    if (!y || !den || !g) {
+        free(y);
+        free(den);
+        free(g);
+        return -2;
+    }
+    int rc = oracle_direct(dK, dV, P, c, T, q, k, v, y, den, NULL);
+    if (rc != 0) {
+        free(y);
+        free(den);
+        free(g);
+        return rc;
+    }
+    for (long long i = 0; i < T * dK; ++i) dq[i] = dk[i] = 0.0;
+    for (long long i = 0; i < T * dV; ++i) dv[i] = 0.0;
+    for (long long t = 0; t < T; ++t) {
+        double e = 0.0;
+        for (int j = 0; j < dV; ++j) {
+            g[j] = dy[t * dV + j] / den[t];
+            e -= g[j] * y[t * dV + j];
+        }
+        for (long long s = 0; s <= t; ++s) {
+            double x = 0.0;
+            for (int i = 0; i < dK; ++i) x += q[t * dK + i] * k[s * dK + i];
+            x /= c;
+            /* w = T_P(x) and its derivative T_{P-1}(x), summed term by term */
+            double w = 0.0, dwdx = 0.0, term = 1.0;
+            for (int p = 0; p < P; ++p) {
+                w += term;
+                if (p < P - 1) dwdx += term;
+                term = term * x / (double)(p + 1);
+            }
+            double dw = e;
+            for (int j = 0; j < dV; ++j) {
+                dw += g[j] * v[s * dV + j];
+                dv[s * dV + j] += w * g[j];
+            }
+            const double dx = dw * dwdx / c;
+            for (int i = 0; i < dK; ++i) {
+                dq[t * dK + i] += dx * k[s * dK + i];
+                dk[s * dK + i] += dx * q[t * dK + i];
+            }
+        }
+    }
+    free(y);
+    free(den);
+    free(g);
+    return 0;
+}
+
+/*
  * Exact causal softmax attention, the limit P -> infinity of the above
  * ([CC-TAYLOR] "The Taylor approximation": the series of exp(q.k/c)).
  * Uses the running maximum for the exponent, as any careful softmax does.

@@ -352,3 +352,77 @@ def test_fourth_term_coefficient(golden):
     c = math.sqrt(g["d_K"])
     alpha = Fraction(1, math.factorial(g["p"])) / Fraction(int(c)) ** g["p"]
     assert alpha == Fraction(1, g["value_inverse"])
+
+
+# ------------------------------------------------------------- gradient ----
+# The gradient of L = sum(dy * y) (the pages define no backward pass; the
+# oracle states the exact chain rule).  Pinned against central differences of
+# the forward oracle (itself pinned above), the P = 1 closed form, and two
+# identities that hold for any P.
+
+def _loss(oracle_mod, q, k, v, dy, P):
+    y, _, _ = oracle_mod.direct(q, k, v, P)
+    return float((y * dy).sum())
+
+
+@pytest.mark.parametrize("dK,dV,P,T", [(3, 2, 4, 6), (2, 3, 2, 5), (4, 1, 5, 5), (1, 2, 3, 7)])
+def test_grad_matches_central_differences(oracle_mod, dK, dV, P, T):
+    rng = np.random.default_rng(40 + P)
+    q, k, v = _inputs(rng, T, dK, dV)
+    dy = rng.standard_normal((T, dV))
+    dq, dk, dv = oracle_mod.direct_grad(q, k, v, dy, P)
+    h = 1e-6
+    for name, x, g in (("q", q, dq), ("k", k, dk), ("v", v, dv)):
+        fd = np.zeros_like(x)
+        for idx in np.ndindex(x.shape):
+            xp, xm = x.copy(), x.copy()
+            xp[idx] += h
+            xm[idx] -= h
+            args = {"q": q, "k": k, "v": v}
+            lp = _loss(oracle_mod, **{**args, name: xp}, dy=dy, P=P)
+            lm = _loss(oracle_mod, **{**args, name: xm}, dy=dy, P=P)
+            fd[idx] = (lp - lm) / (2 * h)
+        np.testing.assert_allclose(g, fd, rtol=1e-6, atol=1e-7 * max(1.0, np.abs(fd).max()),
+                                   err_msg=f"d{name}")
+
+
+def test_grad_P1_is_running_mean_gradient(oracle_mod):
+    """P = 1: y_t is the mean of v_0..v_t, so dv_s = sum_{t>=s} dy_t / (t+1) and
+    q, k receive no gradient."""
+    rng = np.random.default_rng(41)
+    T = 25
+    q, k, v = _inputs(rng, T, 3, 4)
+    dy = rng.standard_normal((T, 4))
+    dq, dk, dv = oracle_mod.direct_grad(q, k, v, dy, P=1)
+    scaled = dy / np.arange(1, T + 1)[:, None]
+    want = np.cumsum(scaled[::-1], axis=0)[::-1]
+    np.testing.assert_allclose(dv, want, rtol=1e-12)
+    assert np.all(dq == 0) and np.all(dk == 0)
+
+
+@pytest.mark.parametrize("P", [2, 3, 4, 6])
+def test_grad_identities(oracle_mod, P):
+    """(1) Shifting every v by b shifts every y by b, so sum_s dv_s = sum_t dy_t.
+    (2) y depends on q and k only through q_t . k_s, so
+        sum_t q_t . dq_t = sum_s k_s . dk_s (both are sum x_ts dL/dx_ts)."""
+    rng = np.random.default_rng(42 + P)
+    T, dK, dV = 40, 5, 3
+    q, k, v = _inputs(rng, T, dK, dV, scale=0.7)
+    dy = rng.standard_normal((T, dV))
+    dq, dk, dv = oracle_mod.direct_grad(q, k, v, dy, P)
+    np.testing.assert_allclose(dv.sum(0), dy.sum(0), rtol=1e-10, atol=1e-10)
+    a, b = float((q * dq).sum()), float((k * dk).sum())
+    assert a == pytest.approx(b, rel=1e-10, abs=1e-10)
+    assert abs(a) > 1e-3   # not trivially zero
+
+
+def test_grad_is_causal(oracle_mod):
+    """dy on tokens before s gives token s's keys and values no gradient."""
+    rng = np.random.default_rng(43)
+    T = 20
+    q, k, v = _inputs(rng, T, 3, 3)
+    dy = np.zeros((T, 3))
+    dy[:8] = rng.standard_normal((8, 3))
+    dq, dk, dv = oracle_mod.direct_grad(q, k, v, dy, P=4)
+    assert np.all(dk[8:] == 0) and np.all(dv[8:] == 0) and np.all(dq[8:] == 0)
+    assert np.abs(dk[:8]).max() > 0 and np.abs(dv[:8]).max() > 0
