@@ -185,6 +185,32 @@ SATA_API int sata_prefill_host(const void *q, const void *k, const void *v, floa
                     sata_state *st, void *stream);
 
 /*
+ * Backward pass of a fresh-state prefill: the gradients of a loss L with
+ * respect to q, k and v, given dy = dL/dy for every output of sata_prefill on
+ * the same inputs.  The method's pages define no backward pass (they expect the
+ * attention to be trained in ordinary Transformer pipelines: [CC-TAYLOR]
+ * "Comparison with other methods", "Future directions"); this is the exact
+ * gradient of the forward as defined in [CC-TAYLOR] "Feature maps and linear
+ * attention", y_t = num_t / den_t, computed in the same chunked feature form
+ * (fixed cost per token): the forward is recomputed, then one pass forward
+ * over the sequence with S gives dq and one pass backward with
+ * G = sum_t phi(q_t) [dy_t / den_t | -(dy_t . y_t) / den_t]^T gives dk and dv.
+ * Runs on CUDA cores in fp32 for every supported shape.
+ *   q, k: bf16 [B][H][N][d_K];  v: bf16 [B][H][N][d_V]  (the forward's inputs)
+ *   dy:   fp32 [B][H][N][d_V]
+ *   dq, dk: fp32 [B][H][N][d_K];  dv: fp32 [B][H][N][d_V]  (overwritten)
+ *   workspace: NULL (library-owned) or a device buffer of ws_bytes >=
+ *              sata_backward_workspace_bytes(...).
+ *   stream: cudaStream_t (NULL: legacy stream).
+ * The result is deterministic (partial sums are added in a fixed order).
+ * N = 0 is a no-op.  Errors as sata_prefill_ex.
+ */
+SATA_API int sata_backward_workspace_bytes(int B, int H, int64_t N, int d_K, int d_V, int P, size_t *bytes);
+SATA_API int sata_prefill_backward(const void *q, const void *k, const void *v, const float *dy,
+                    float *dq, float *dk, float *dv, int B, int H, int64_t N, int d_K, int d_V, int P,
+                    void *workspace, size_t ws_bytes, void *stream);
+
+/*
  * One decode step for every head of `st`, on st->stream: the state absorbs
  * (k, v) and the output is read with q ([CC-TAYLOR] "Feature maps and linear
  * attention": Z_T = Z_{T-1} + phi(k_T), S_T = S_{T-1} + phi(k_T) v_T^T, then

@@ -36,6 +36,7 @@ EXPORTED = (
     "sata_state_bytes", "sata_state_init", "sata_workspace_bytes", "sata_prefill",
     "sata_prefill_ex", "sata_decode_step", "sata_set_option", "sata_get_option",
     "sata_kernel_stats", "sata_reset_kernel_stats", "sata_decode_step_static", "sata_prefill_host",
+    "sata_backward_workspace_bytes", "sata_prefill_backward",
 )
 
 
@@ -96,6 +97,9 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "sata_reset_kernel_stats": (i32, []),
         "sata_decode_step_static": (i32, [st_p, vp, vp, vp, vp]),
         "sata_prefill_host": (i32, [vp, vp, vp, vp, i32, i32, i64, i32, i32, i32, st_p, vp]),
+        "sata_backward_workspace_bytes": (i32, [i32, i32, i64, i32, i32, i32, P_sz]),
+        "sata_prefill_backward": (i32, [vp, vp, vp, vp, vp, vp, vp, i32, i32, i64, i32, i32, i32,
+                                        vp, sz, vp]),
     }
     for name, (res, args) in sigs.items():
         fn = getattr(lib, name)
@@ -204,6 +208,13 @@ def sata_workspace_bytes(B, H, N, d_K, d_V, P) -> int:
     return b.value
 
 
+def sata_backward_workspace_bytes(B, H, N, d_K, d_V, P) -> int:
+    b = ctypes.c_size_t(0)
+    _check(load().sata_backward_workspace_bytes(B, H, N, d_K, d_V, P, ctypes.byref(b)),
+           "sata_backward_workspace_bytes")
+    return b.value
+
+
 # ---------------------------------------------------------- device calls ----
 
 def sata_prefill(q, k, v, out, B, H, N, d_K, d_V, P):
@@ -228,6 +239,13 @@ def sata_prefill_host(q, k, v, out, B, H, N, d_K, d_V, P, st=None, stream=None):
     _check(load().sata_prefill_host(_ptr(q), _ptr(k), _ptr(v), _ptr(out), B, H, N, d_K, d_V, P,
                                     None if st is None else ctypes.byref(st), _stream(stream)),
            "sata_prefill_host")
+
+
+def sata_prefill_backward(q, k, v, dy, dq, dk, dv, B, H, N, d_K, d_V, P, workspace=None, stream=None):
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(load().sata_prefill_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(dy), _ptr(dq), _ptr(dk),
+                                        _ptr(dv), B, H, N, d_K, d_V, P, _ptr(workspace), ws_bytes,
+                                        _stream(stream)), "sata_prefill_backward")
 
 
 def sata_state_init(st, B, H, d_K, d_V, P, S, Z, stream=None):
@@ -280,6 +298,42 @@ def prefill(q, k, v, P: int = 4, state: State | None = None, out=None, workspace
     sata_prefill_ex(q, k, v, out, B, H, N, d_K, d_V, P, None if state is None else state.st,
                     workspace, stream)
     return out
+
+
+def prefill_backward(q, k, v, dy, P: int = 4, workspace=None, stream=None):
+    """Gradients (dq, dk, dv), fp32, of sum(dy * y) for y = prefill(q, k, v, P) from a
+    fresh state; dy is fp32 [B, H, N, d_V]."""
+    B, H, N, d_K = q.shape
+    d_V = v.shape[-1]
+    _need(q, torch.bfloat16, (B, H, N, d_K), "q")
+    _need(k, torch.bfloat16, (B, H, N, d_K), "k")
+    _need(v, torch.bfloat16, (B, H, N, d_V), "v")
+    _need(dy, torch.float32, (B, H, N, d_V), "dy")
+    dq = torch.empty((B, H, N, d_K), dtype=torch.float32, device=q.device)
+    dk = torch.empty_like(dq)
+    dv = torch.empty((B, H, N, d_V), dtype=torch.float32, device=q.device)
+    sata_prefill_backward(q, k, v, dy, dq, dk, dv, B, H, N, d_K, d_V, P, workspace, stream)
+    return dq, dk, dv
+
+
+class _Attention(torch.autograd.Function):
+    @staticmethod
+    def forward(ctx, q, k, v, P):
+        ctx.P = P
+        ctx.save_for_backward(q, k, v)
+        return prefill(q, k, v, P)
+
+    @staticmethod
+    def backward(ctx, dy):
+        q, k, v = ctx.saved_tensors
+        dq, dk, dv = prefill_backward(q, k, v, dy.float().contiguous(), ctx.P)
+        return dq, dk, dv, None
+
+
+def attention(q, k, v, P: int = 4):
+    """prefill() as a differentiable op: y (fp32) = attention(q, k, v, P), and
+    y.backward(...) runs sata_prefill_backward (gradients cast to the inputs' bf16)."""
+    return _Attention.apply(q, k, v, P)
 
 
 def decode_step(state: State, q, k, v, out=None):

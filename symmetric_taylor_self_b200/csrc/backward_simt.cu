@@ -1,0 +1,582 @@
+// Backward pass of the causal prefill on CUDA cores (fp32): the gradients of a
+// loss L with respect to q, k and v, given dL/dy for every output.
+//
+// The method's pages define no backward pass; they expect the attention to be
+// trained inside ordinary Transformer pipelines ([CC-TAYLOR] "Comparison with
+// other methods"; end-to-end training is listed under "Future directions").
+// This is the exact gradient of the forward as defined ([CC-TAYLOR] "Feature
+// maps and linear attention"), written in the same feature form so that it
+// costs a fixed amount per token:
+//   y_t = num_t / den_t,  [num_t | den_t] = sum_{s<=t} w_ts u_s,  u_s = [v_s | 1],
+//   w_ts = sum_f a_f phi_f(q_t) phi_f(k_s),  a_f = alpha_p C_p  (coef[] below).
+// With g_t = dy_t / den_t and r_t = [g_t | -(g_t . y_t)], the gradient of w_ts
+// is dw_ts = r_t . u_s, and
+//   dq_t = J_phi(q_t)^T (a (.) S_t r_t),          S_t = sum_{s<=t} phi(k_s) u_s^T
+//   dk_s = J_phi(k_s)^T (a (.) G_s u_s),          G_s = sum_{t>=s} phi(q_t) r_t^T
+//   dv_s = (a (.) phi(k_s))^T G_s[:, :d_V],
+// where J_phi is the Jacobian of the monomial features: d phi_f / d x_i =
+// mult_i(f) * (the product of f's other indices).  Chunked like the forward
+// (chunks of kL tokens): the state before / after a chunk gives the inter-chunk
+// part; pairs inside a chunk are summed directly, with
+//   dx_ts = dw_ts * T_{P-1}(x_ts)   (T_P' = T_{P-1}),  x_ts = q_t . k_s / c,
+//   dq_t += dx_ts k_s / c,  dk_s += dx_ts q_t / c,  dv_s += w_ts g_t.
+//
+// Kernels, in stream order:
+//   forward (prefill_simt.cu) -> y and den;  bwd_r -> r;
+//   bwd_q_scan: per feature tile, forward over the chunks with S: dq partials;
+//   bwd_finish<dq>: sum the tiles' partials, add the intra-chunk part;
+//   bwd_kv_scan: per feature tile, backward over the chunks with G: dk, dv partials;
+//   bwd_finish<dk, dv>.
+// Partials are summed in a fixed order: the result is deterministic.
+#include <cuda_bf16.h>
+
+#include <cstring>
+#include <map>
+#include <mutex>
+#include <vector>
+
+#include "sata_internal.h"
+
+namespace sata {
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kTF = 128;   // features per CTA
+constexpr int kL = 32;     // chunk length
+constexpr int kMaxComp = kMaxP - 2;   // indices left of a top-degree feature after removing one
+constexpr size_t kPartialBudget = size_t(2) << 30;  // bytes of partials per segment
+
+// Jacobian table of one (d_K, P): for every feature tile and every input index
+// i, the features of the tile that contain i.  Entry (uint64):
+//   bits 0..7 the feature's position in its tile, 8..15 the multiplicity of i,
+//   16..63 the feature's other indices (one copy of i removed), 8 bits each,
+//   padded with d_K (the constant 1).
+// Layout: uint32 offsets[ntiles][d_K + 1] (into the entry array), then the
+// entries, 8-byte aligned.
+struct JacTable {
+    std::vector<uint8_t> image;
+    size_t off_entries = 0;
+};
+
+bool build_jac_table(int d_K, int P, JacTable &jt) {
+    HostBasis hb;
+    if (!build_basis_host(d_K, P, hb)) return false;
+    const int64_t F = hb.offsets[P];
+    const int64_t ntiles = (F + kTF - 1) / kTF;
+    std::vector<std::vector<uint64_t>> lists((size_t)ntiles * d_K);
+    for (int64_t f = 0; f < F; ++f) {
+        const auto &t = hb.tuples[f];
+        const int p = (int)t.size();
+        size_t s = 0;
+        while (s < t.size()) {   // runs of equal indices: one entry per distinct index
+            size_t e = s;
+            while (e < t.size() && t[e] == t[s]) ++e;
+            uint64_t ent = (uint64_t)(f % kTF) | ((uint64_t)(e - s) << 8);
+            int m = 0;
+            for (int x = 0; x < p; ++x) {
+                if (x == (int)s) continue;   // drop one copy of the index
+                ent |= (uint64_t)t[x] << (16 + 8 * m);
+                ++m;
+            }
+            for (; m < kMaxComp; ++m) ent |= (uint64_t)d_K << (16 + 8 * m);
+            lists[(size_t)(f / kTF) * d_K + t[s]].push_back(ent);
+            s = e;
+        }
+    }
+    const size_t noff = (size_t)ntiles * (d_K + 1);
+    size_t total = 0;
+    for (auto &l : lists) total += l.size();
+    jt.off_entries = (noff * sizeof(uint32_t) + 7) / 8 * 8;
+    jt.image.assign(jt.off_entries + (total ? total : 1) * sizeof(uint64_t), 0);
+    uint32_t *off = (uint32_t *)jt.image.data();
+    uint64_t *ent = (uint64_t *)(jt.image.data() + jt.off_entries);
+    size_t pos = 0;
+    for (int64_t tile = 0; tile < ntiles; ++tile) {
+        for (int i = 0; i < d_K; ++i) {
+            off[tile * (d_K + 1) + i] = (uint32_t)pos;
+            for (uint64_t e : lists[(size_t)tile * d_K + i]) ent[pos++] = e;
+        }
+        off[tile * (d_K + 1) + d_K] = (uint32_t)pos;
+    }
+    return true;
+}
+
+// Device copy of the table, cached per (device, d_K, P).
+const uint8_t *jac_table(int d_K, int P, size_t *off_entries, cudaError_t *err) {
+    static std::mutex mu;
+    static std::map<std::pair<int, int>, JacTable> cache;
+    const JacTable *jt = nullptr;
+    {
+        std::lock_guard<std::mutex> lk(mu);
+        auto key = std::make_pair(d_K, P);
+        auto it = cache.find(key);
+        if (it == cache.end()) {
+            JacTable t;
+            if (!build_jac_table(d_K, P, t)) {
+                *err = cudaErrorInvalidValue;
+                return nullptr;
+            }
+            it = cache.emplace(key, std::move(t)).first;
+        }
+        jt = &it->second;
+    }
+    *off_entries = jt->off_entries;
+    const uint64_t key = (uint64_t(0xB0) << 56) | ((uint64_t)d_K << 16) | (uint64_t)P;
+    return (const uint8_t *)device_table(
+        key, jt->image.size(), [jt](uint8_t *h) { std::memcpy(h, jt->image.data(), jt->image.size()); },
+        err);
+}
+
+// phi_f(x~) for the packed feature word(s): x~ is a row of d_K + 1 values whose
+// last one is the constant 1.
+__device__ __forceinline__ float feature(const float *x, uint32_t w, const uint32_t *packed_hi,
+                                         int64_t fg) {
+    float v = x[w & 255] * x[(w >> 8) & 255] * x[(w >> 16) & 255];
+    if (packed_hi) {   // degrees above 3: the leading indices
+        const uint32_t wh = packed_hi[fg];
+#pragma unroll
+        for (int m = 0; m < 4; ++m) v *= x[(wh >> (8 * m)) & 255];
+    }
+    return v;
+}
+
+// J_phi(x~)^T applied to one tile's feature values `val` (one token):
+// sum over the tile's features f containing index i of val[f] * d phi_f / d x_i.
+__device__ __forceinline__ float jac_t(const uint32_t *__restrict__ off, const uint64_t *__restrict__ ent,
+                                       int i, const float *x, const float *val, int ncomp) {
+    const uint32_t b = off[i], e = off[i + 1];
+    float acc = 0.f;
+    for (uint32_t n = b; n < e; ++n) {
+        const uint64_t u = ent[n];
+        float d = (float)((u >> 8) & 255);
+        for (int m = 0; m < ncomp; ++m) d *= x[(u >> (16 + 8 * m)) & 255];
+        acc = fmaf(val[u & 255], d, acc);
+    }
+    return acc;
+}
+
+// Loads one chunk: x~q, x~k [kL][d_K+1] (last column 1), u = [v | 1] and r
+// [kL][d_V+1]; rows past the end are zero.
+__device__ __forceinline__ void load_chunk(const __nv_bfloat16 *q, const __nv_bfloat16 *k,
+                                           const __nv_bfloat16 *v, const float *r, int64_t row0,
+                                           int nt, int d_K, int d_V, float *xq, float *xk, float *xu,
+                                           float *xr) {
+    const int DK1 = d_K + 1, DV1 = d_V + 1;
+    for (int e = threadIdx.x; e < kL * DK1; e += kThreads) {
+        const int t = e / DK1, i = e % DK1;
+        float a = 0.f, b = 0.f;
+        if (t < nt) {
+            a = i < d_K ? __bfloat162float(q[(row0 + t) * d_K + i]) : 1.f;
+            b = i < d_K ? __bfloat162float(k[(row0 + t) * d_K + i]) : 1.f;
+        }
+        xq[e] = a;
+        xk[e] = b;
+    }
+    for (int e = threadIdx.x; e < kL * DV1; e += kThreads) {
+        const int t = e / DV1, j = e % DV1;
+        float a = 0.f, b = 0.f;
+        if (t < nt) {
+            a = j < d_V ? __bfloat162float(v[(row0 + t) * d_V + j]) : 1.f;
+            b = r[(row0 + t) * DV1 + j];
+        }
+        xu[e] = a;
+        xr[e] = b;
+    }
+}
+
+// r_t = [dy_t / den_t | -(dy_t . y_t) / den_t], one warp per token.
+__global__ void __launch_bounds__(kThreads)
+bwd_r_kernel(const float *__restrict__ dy, const float *__restrict__ y, const float *__restrict__ den,
+             float *__restrict__ r, int d_V, int64_t rows) {
+    const int64_t row = (int64_t)blockIdx.x * (kThreads / 32) + threadIdx.x / 32;
+    const int lane = threadIdx.x & 31;
+    if (row >= rows) return;
+    const float inv = 1.0f / den[row];
+    float s = 0.f;
+    for (int j = lane; j < d_V; j += 32) {
+        const float g = dy[row * d_V + j] * inv;
+        r[row * (d_V + 1) + j] = g;
+        s = fmaf(g, y[row * d_V + j], s);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+    if (lane == 0) r[row * (d_V + 1) + d_V] = -s;
+}
+
+// dq partials of one feature tile of one head over the tokens [t0, t0 + T):
+// forward over the chunks with the tile's rows of S = sum phi(k) u^T.
+__global__ void __launch_bounds__(kThreads)
+bwd_q_scan_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k,
+                  const __nv_bfloat16 *__restrict__ v, const float *__restrict__ r,
+                  float *__restrict__ state, const uint32_t *__restrict__ packed,
+                  const uint32_t *__restrict__ packed_hi, const float *__restrict__ coef,
+                  const uint32_t *__restrict__ jac_off, const uint64_t *__restrict__ jac_ent, int d_K,
+                  int d_V, int ncomp, int64_t F, int64_t N, int64_t t0, int T, int Tseg, int load_state,
+                  float *__restrict__ partials) {
+    extern __shared__ float smem[];
+    const int DK1 = d_K + 1, DV1 = d_V + 1;
+    float *Sx = smem;                  // [kTF][DV1]
+    float *xq = Sx + kTF * DV1;        // [kL][DK1]
+    float *xk = xq + kL * DK1;
+    float *xu = xk + kL * DK1;         // [kL][DV1]
+    float *xr = xu + kL * DV1;
+    float *phik = xr + kL * DV1;       // [kL][kTF]
+    float *val = phik + kL * kTF;      // [kL][kTF]
+
+    const int64_t bh = blockIdx.x;
+    const int BH = gridDim.x;
+    const int tile = blockIdx.y;
+    const int64_t f0 = (int64_t)tile * kTF;
+    const int nf = (int)(F - f0 < (int64_t)kTF ? F - f0 : (int64_t)kTF);
+    const int tid = threadIdx.x;
+    const uint32_t *toff = jac_off + (size_t)tile * (d_K + 1);
+
+    for (int e = tid; e < kTF * DV1; e += kThreads) {
+        const int f = e / DV1;
+        Sx[e] = (load_state && f < nf) ? state[(bh * F + f0) * DV1 + e] : 0.f;
+    }
+    for (int c0 = 0; c0 < T; c0 += kL) {
+        const int nt = min(kL, T - c0);
+        __syncthreads();
+        load_chunk(q, k, v, r, bh * N + t0 + c0, nt, d_K, d_V, xq, xk, xu, xr);
+        __syncthreads();
+        for (int e = tid; e < kL * kTF; e += kThreads) {
+            const int t = e / kTF, f = e % kTF;
+            float pk = 0.f, vl = 0.f;
+            if (t < nt && f < nf) {
+                pk = feature(xk + t * DK1, packed[f0 + f], packed_hi, f0 + f);
+                float acc = 0.f;
+                for (int j = 0; j < DV1; ++j) acc = fmaf(Sx[f * DV1 + j], xr[t * DV1 + j], acc);
+                vl = coef[f0 + f] * acc;
+            }
+            phik[e] = pk;
+            val[e] = vl;
+        }
+        __syncthreads();
+        for (int e = tid; e < nt * d_K; e += kThreads) {
+            const int t = e / d_K, i = e % d_K;
+            partials[(((int64_t)tile * BH + bh) * Tseg + c0 + t) * d_K + i] =
+                jac_t(toff, jac_ent, i, xq + t * DK1, val + t * kTF, ncomp);
+        }
+        for (int e = tid; e < nf * DV1; e += kThreads) {
+            const int f = e / DV1, j = e % DV1;
+            float acc = Sx[e];
+            for (int t = 0; t < nt; ++t) acc = fmaf(phik[t * kTF + f], xu[t * DV1 + j], acc);
+            Sx[e] = acc;
+        }
+    }
+    __syncthreads();
+    for (int e = tid; e < nf * DV1; e += kThreads) state[(bh * F + f0) * DV1 + e] = Sx[e];
+}
+
+// dk and dv partials of one feature tile of one head over the tokens
+// [t0, t0 + T): backward over the chunks with the tile's rows of
+// G = sum phi(q) r^T over the tokens after the chunk.
+__global__ void __launch_bounds__(kThreads)
+bwd_kv_scan_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k,
+                   const __nv_bfloat16 *__restrict__ v, const float *__restrict__ r,
+                   float *__restrict__ state, const uint32_t *__restrict__ packed,
+                   const uint32_t *__restrict__ packed_hi, const float *__restrict__ coef,
+                   const uint32_t *__restrict__ jac_off, const uint64_t *__restrict__ jac_ent, int d_K,
+                   int d_V, int ncomp, int64_t F, int64_t N, int64_t t0, int T, int Tseg,
+                   int load_state, float *__restrict__ partials) {
+    extern __shared__ float smem[];
+    const int DK1 = d_K + 1, DV1 = d_V + 1, DKV = d_K + d_V;
+    float *Gx = smem;                  // [kTF][DV1]
+    float *xq = Gx + kTF * DV1;        // [kL][DK1]
+    float *xk = xq + kL * DK1;
+    float *xu = xk + kL * DK1;         // [kL][DV1]
+    float *xr = xu + kL * DV1;
+    float *phiq = xr + kL * DV1;       // [kL][kTF]
+    float *pka = phiq + kL * kTF;      // [kL][kTF]  a (.) phi(k)
+    float *val = pka + kL * kTF;       // [kL][kTF]  a (.) G u
+
+    const int64_t bh = blockIdx.x;
+    const int BH = gridDim.x;
+    const int tile = blockIdx.y;
+    const int64_t f0 = (int64_t)tile * kTF;
+    const int nf = (int)(F - f0 < (int64_t)kTF ? F - f0 : (int64_t)kTF);
+    const int tid = threadIdx.x;
+    const uint32_t *toff = jac_off + (size_t)tile * (d_K + 1);
+
+    for (int e = tid; e < kTF * DV1; e += kThreads) {
+        const int f = e / DV1;
+        Gx[e] = (load_state && f < nf) ? state[(bh * F + f0) * DV1 + e] : 0.f;
+    }
+    const int nchunks = (T + kL - 1) / kL;
+    for (int ci = nchunks - 1; ci >= 0; --ci) {
+        const int c0 = ci * kL;
+        const int nt = min(kL, T - c0);
+        __syncthreads();
+        load_chunk(q, k, v, r, bh * N + t0 + c0, nt, d_K, d_V, xq, xk, xu, xr);
+        __syncthreads();
+        for (int e = tid; e < kL * kTF; e += kThreads) {
+            const int t = e / kTF, f = e % kTF;
+            float pq = 0.f, pk = 0.f, vl = 0.f;
+            if (t < nt && f < nf) {
+                const uint32_t w = packed[f0 + f];
+                const float a = coef[f0 + f];
+                pq = feature(xq + t * DK1, w, packed_hi, f0 + f);
+                pk = a * feature(xk + t * DK1, w, packed_hi, f0 + f);
+                float acc = 0.f;
+                for (int j = 0; j < DV1; ++j) acc = fmaf(Gx[f * DV1 + j], xu[t * DV1 + j], acc);
+                vl = a * acc;
+            }
+            phiq[e] = pq;
+            pka[e] = pk;
+            val[e] = vl;
+        }
+        __syncthreads();
+        for (int e = tid; e < nt * d_K; e += kThreads) {
+            const int t = e / d_K, i = e % d_K;
+            partials[(((int64_t)tile * BH + bh) * Tseg + c0 + t) * DKV + i] =
+                jac_t(toff, jac_ent, i, xk + t * DK1, val + t * kTF, ncomp);
+        }
+        for (int e = tid; e < nt * d_V; e += kThreads) {
+            const int t = e / d_V, j = e % d_V;
+            float acc = 0.f;
+            for (int f = 0; f < nf; ++f) acc = fmaf(pka[t * kTF + f], Gx[f * DV1 + j], acc);
+            partials[(((int64_t)tile * BH + bh) * Tseg + c0 + t) * DKV + d_K + j] = acc;
+        }
+        __syncthreads();
+        for (int e = tid; e < nf * DV1; e += kThreads) {
+            const int f = e / DV1, j = e % DV1;
+            float acc = Gx[e];
+            for (int t = 0; t < nt; ++t) acc = fmaf(phiq[t * kTF + f], xr[t * DV1 + j], acc);
+            Gx[e] = acc;
+        }
+    }
+    __syncthreads();
+    for (int e = tid; e < nf * DV1; e += kThreads) state[(bh * F + f0) * DV1 + e] = Gx[e];
+}
+
+// Per chunk: sum the tiles' partials in tile order and add the pairs inside the
+// chunk.  KV = false: dq (partials [tile][BH][Tseg][d_K]); KV = true: dk and dv
+// (partials [tile][BH][Tseg][d_K + d_V]).
+template <bool KV>
+__global__ void __launch_bounds__(kThreads)
+bwd_finish_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k,
+                  const __nv_bfloat16 *__restrict__ v, const float *__restrict__ r,
+                  const float *__restrict__ partials, int ntiles, int d_K, int d_V, int P, float inv_c,
+                  int64_t N, int64_t t0, int T, int Tseg, float *__restrict__ dqk,
+                  float *__restrict__ dv) {
+    extern __shared__ float smem[];
+    const int DV1 = d_V + 1;
+    const int PW = KV ? d_K + d_V : d_K;   // partial row width
+    float *xq = smem;                  // [kL][d_K]
+    float *xk = xq + kL * d_K;
+    float *xu = xk + kL * d_K;         // [kL][DV1]
+    float *xr = xu + kL * DV1;
+    float *Wd = xr + kL * DV1;         // [kL][kL]  dx_ts / c
+    float *Ww = Wd + kL * kL;          // [kL][kL]  w_ts
+
+    const int64_t bh = blockIdx.x;
+    const int BH = gridDim.x;
+    const int c0 = blockIdx.y * kL;
+    const int nt = min(kL, T - c0);
+    const int64_t row0 = bh * N + t0 + c0;
+    const int tid = threadIdx.x;
+    for (int e = tid; e < kL * d_K; e += kThreads) {
+        const int t = e / d_K, i = e % d_K;
+        float a = 0.f, b = 0.f;
+        if (t < nt) {
+            a = __bfloat162float(q[(row0 + t) * d_K + i]);
+            b = __bfloat162float(k[(row0 + t) * d_K + i]);
+        }
+        xq[e] = a;
+        xk[e] = b;
+    }
+    for (int e = tid; e < kL * DV1; e += kThreads) {
+        const int t = e / DV1, j = e % DV1;
+        float a = 0.f, b = 0.f;
+        if (t < nt) {
+            a = j < d_V ? __bfloat162float(v[(row0 + t) * d_V + j]) : 1.f;
+            b = r[(row0 + t) * DV1 + j];
+        }
+        xu[e] = a;
+        xr[e] = b;
+    }
+    __syncthreads();
+    for (int e = tid; e < kL * kL; e += kThreads) {
+        const int t = e / kL, s = e % kL;
+        float wd = 0.f, w = 0.f;
+        if (t < nt && s <= t) {
+            float x = 0.f;
+            for (int i = 0; i < d_K; ++i) x = fmaf(xq[t * d_K + i], xk[s * d_K + i], x);
+            x *= inv_c;
+            // Horner forms of T_P(x) = sum_{p<P} x^p / p! and of T_{P-1}(x)
+            float h = 1.f;
+            for (int p = P - 1; p >= 1; --p) h = fmaf(h, x / (float)p, 1.f);
+            float hd = 0.f;
+            if (P > 1) {
+                hd = 1.f;
+                for (int p = P - 2; p >= 1; --p) hd = fmaf(hd, x / (float)p, 1.f);
+            }
+            float dw = 0.f;
+            for (int j = 0; j < DV1; ++j) dw = fmaf(xr[t * DV1 + j], xu[s * DV1 + j], dw);
+            wd = dw * hd * inv_c;
+            w = h;
+        }
+        Wd[e] = wd;
+        Ww[e] = w;
+    }
+    __syncthreads();
+    for (int e = tid; e < nt * d_K; e += kThreads) {
+        const int t = e / d_K, i = e % d_K;
+        float a = 0.f;
+        for (int tile = 0; tile < ntiles; ++tile)
+            a += partials[(((int64_t)tile * BH + bh) * Tseg + c0 + t) * PW + i];
+        float b = 0.f;
+        if (!KV) {
+            for (int s = 0; s <= t; ++s) b = fmaf(Wd[t * kL + s], xk[s * d_K + i], b);
+        } else {   // row t is the key token s here
+            for (int u = t; u < nt; ++u) b = fmaf(Wd[u * kL + t], xq[u * d_K + i], b);
+        }
+        dqk[(row0 + t) * d_K + i] = a + b;
+    }
+    if (KV) {
+        for (int e = tid; e < nt * d_V; e += kThreads) {
+            const int s = e / d_V, j = e % d_V;
+            float a = 0.f;
+            for (int tile = 0; tile < ntiles; ++tile)
+                a += partials[(((int64_t)tile * BH + bh) * Tseg + c0 + s) * PW + d_K + j];
+            float b = 0.f;
+            for (int u = s; u < nt; ++u) b = fmaf(Ww[u * kL + s], xr[u * DV1 + j], b);
+            dv[(row0 + s) * d_V + j] = a + b;
+        }
+    }
+}
+
+int64_t segment_tokens(int BH, int64_t N, int64_t F, int d_K, int d_V) {
+    const int64_t ntiles = (F + kTF - 1) / kTF;
+    const int64_t per_token = ntiles * BH * (d_K + d_V) * (int64_t)sizeof(float);
+    int64_t T = (int64_t)(kPartialBudget / (size_t)per_token) / kL * kL;
+    if (T < kL) T = kL;
+    if (T > (int64_t)65535 * kL) T = (int64_t)65535 * kL;   // finish kernels' grid.y
+    const int64_t Nr = (N + kL - 1) / kL * kL;
+    return T < Nr ? T : Nr;
+}
+
+size_t round256(size_t b) { return (b + 255) / 256 * 256; }
+
+struct BwdLayout {
+    int64_t Tseg = 0;
+    size_t fwd = 0, part = 0, off_state = 0, off_y = 0, off_den = 0, off_r = 0, total = 0;
+};
+
+BwdLayout bwd_layout(int BH, int64_t N, int64_t F, int d_K, int d_V) {
+    BwdLayout L;
+    const int64_t ntiles = (F + kTF - 1) / kTF;
+    L.Tseg = segment_tokens(BH, N, F, d_K, d_V);
+    L.fwd = prefill_simt_workspace_bytes(BH, N, F, d_V, true);
+    L.part = round256((size_t)ntiles * BH * L.Tseg * (d_K + d_V) * sizeof(float));
+    const size_t front = L.fwd > L.part ? L.fwd : L.part;   // the forward's workspace, then the partials
+    L.off_state = round256(front);
+    L.off_y = L.off_state + round256((size_t)BH * F * (d_V + 1) * sizeof(float));
+    L.off_den = L.off_y + round256((size_t)BH * N * d_V * sizeof(float));
+    L.off_r = L.off_den + round256((size_t)BH * N * sizeof(float));
+    L.total = L.off_r + round256((size_t)BH * N * (d_V + 1) * sizeof(float));
+    return L;
+}
+
+size_t scan_smem(int d_K, int d_V, int nphi) {
+    return sizeof(float) * ((size_t)kTF * (d_V + 1) + 2 * kL * (d_K + 1) + 2 * kL * (d_V + 1) +
+                            (size_t)nphi * kL * kTF);
+}
+
+}  // namespace
+
+size_t prefill_backward_workspace_bytes(int BH, int64_t N, int64_t F, int d_K, int d_V) {
+    return bwd_layout(BH, N, F, d_K, d_V).total;
+}
+
+cudaError_t launch_prefill_backward(const DeviceBasis &basis, int BH, int64_t N, int d_V,
+                                    const void *q, const void *k, const void *v, const float *dy,
+                                    float *dq, float *dk, float *dv, void *ws, size_t ws_bytes,
+                                    cudaStream_t stream) {
+    const int d_K = basis.d_K, P = basis.P;
+    const int64_t F = basis.F;
+    const BwdLayout L = bwd_layout(BH, N, F, d_K, d_V);
+    if (ws_bytes < L.total) return cudaErrorInvalidValue;
+    const int ntiles = (int)((F + kTF - 1) / kTF);
+    const int ncomp = P > 2 ? P - 2 : 0;
+    cudaError_t e = cudaSuccess;
+    size_t off_ent = 0;
+    const uint8_t *jt = jac_table(d_K, P, &off_ent, &e);
+    if (!jt) return e != cudaSuccess ? e : cudaErrorMemoryAllocation;
+    const uint32_t *jac_off = (const uint32_t *)jt;
+    const uint64_t *jac_ent = (const uint64_t *)(jt + off_ent);
+
+    uint8_t *w = (uint8_t *)ws;
+    float *partials = (float *)w;
+    float *state = (float *)(w + L.off_state);
+    float *y = (float *)(w + L.off_y);
+    float *den = (float *)(w + L.off_den);
+    float *r = (float *)(w + L.off_r);
+    const __nv_bfloat16 *qb = (const __nv_bfloat16 *)q, *kb = (const __nv_bfloat16 *)k,
+                        *vb = (const __nv_bfloat16 *)v;
+
+    // forward: y and den (fresh state, carried in the front region)
+    e = launch_prefill_simt(basis, BH, N, d_V, q, k, v, y, nullptr, nullptr, false, ws, L.fwd, stream, den);
+    if (e != cudaSuccess) return e;
+    const int64_t rows = (int64_t)BH * N;
+    launch_begin(kBwdR, stream);
+    bwd_r_kernel<<<(unsigned)((rows + kThreads / 32 - 1) / (kThreads / 32)), kThreads, 0, stream>>>(
+        dy, y, den, r, d_V, rows);
+    launch_end(kBwdR, stream);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+
+    const size_t smemQ = scan_smem(d_K, d_V, 2), smemKV = scan_smem(d_K, d_V, 3);
+    const size_t smemF = sizeof(float) * ((size_t)2 * kL * d_K + 2 * kL * (d_V + 1) + 2 * kL * kL);
+    if ((e = cudaFuncSetAttribute(bwd_q_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)smemQ)) != cudaSuccess)
+        return e;
+    if ((e = cudaFuncSetAttribute(bwd_kv_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)smemKV)) != cudaSuccess)
+        return e;
+    if ((e = cudaFuncSetAttribute(bwd_finish_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)smemF)) != cudaSuccess)
+        return e;
+    if ((e = cudaFuncSetAttribute(bwd_finish_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)smemF)) != cudaSuccess)
+        return e;
+    const float inv_c = 1.0f / sqrtf((float)d_K);
+    const int64_t Tseg = L.Tseg;
+    const int nseg = (int)((N + Tseg - 1) / Tseg);
+
+    // dq: segments in order, S carried forward
+    for (int sg = 0; sg < nseg; ++sg) {
+        const int64_t t0 = (int64_t)sg * Tseg;
+        const int T = (int)(N - t0 < Tseg ? N - t0 : Tseg);
+        launch_begin(kBwdQScan, stream);
+        bwd_q_scan_kernel<<<dim3(BH, ntiles), kThreads, smemQ, stream>>>(
+            qb, kb, vb, r, state, basis.packed, basis.packed_hi, basis.coef, jac_off, jac_ent, d_K, d_V,
+            ncomp, F, N, t0, T, (int)Tseg, sg > 0 ? 1 : 0, partials);
+        launch_end(kBwdQScan, stream);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        launch_begin(kBwdFinish, stream);
+        bwd_finish_kernel<false><<<dim3(BH, (T + kL - 1) / kL), kThreads, smemF, stream>>>(
+            qb, kb, vb, r, partials, ntiles, d_K, d_V, P, inv_c, N, t0, T, (int)Tseg, dq, nullptr);
+        launch_end(kBwdFinish, stream);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+    // dk, dv: segments in reverse, G carried backward
+    for (int sg = nseg - 1; sg >= 0; --sg) {
+        const int64_t t0 = (int64_t)sg * Tseg;
+        const int T = (int)(N - t0 < Tseg ? N - t0 : Tseg);
+        launch_begin(kBwdKVScan, stream);
+        bwd_kv_scan_kernel<<<dim3(BH, ntiles), kThreads, smemKV, stream>>>(
+            qb, kb, vb, r, state, basis.packed, basis.packed_hi, basis.coef, jac_off, jac_ent, d_K, d_V,
+            ncomp, F, N, t0, T, (int)Tseg, sg < nseg - 1 ? 1 : 0, partials);
+        launch_end(kBwdKVScan, stream);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        launch_begin(kBwdFinish, stream);
+        bwd_finish_kernel<true><<<dim3(BH, (T + kL - 1) / kL), kThreads, smemF, stream>>>(
+            qb, kb, vb, r, partials, ntiles, d_K, d_V, P, inv_c, N, t0, T, (int)Tseg, dk, dv);
+        launch_end(kBwdFinish, stream);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+    return cudaSuccess;
+}
+
+}  // namespace sata

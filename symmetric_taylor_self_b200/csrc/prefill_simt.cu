@@ -146,7 +146,7 @@ __global__ void __launch_bounds__(kThreads)
 simt_finish_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k,
                    const __nv_bfloat16 *__restrict__ v, const float *__restrict__ partials,
                    int ntiles, int d_K, int d_V, int P, float inv_c, int64_t N, int64_t t0,
-                   int T, int Tseg, float *__restrict__ out) {
+                   int T, int Tseg, float *__restrict__ out, float *__restrict__ den_out) {
     extern __shared__ float smem[];
     const int DV1 = d_V + 1;
     float *xq = smem;                  // [kL][d_K]
@@ -207,6 +207,8 @@ simt_finish_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
         const int t = e / d_V, j = e % d_V;
         out[(bh * N + t0 + c0 + t) * d_V + j] = acc[t * DV1 + j] / acc[t * DV1 + d_V];
     }
+    if (den_out)   // the denominators, for the backward pass
+        for (int t = tid; t < nt; t += kThreads) den_out[bh * N + t0 + c0 + t] = acc[t * DV1 + d_V];
 }
 
 int64_t segment_tokens(int BH, int64_t N, int64_t F, int d_V) {
@@ -233,7 +235,7 @@ size_t prefill_simt_workspace_bytes(int BH, int64_t N, int64_t F, int d_V, bool 
 cudaError_t launch_prefill_simt(const DeviceBasis &basis, int BH, int64_t N, int d_V,
                                 const void *q, const void *k, const void *v, float *out,
                                 float *S, float *Z, bool state_in, void *ws, size_t ws_bytes,
-                                cudaStream_t stream) {
+                                cudaStream_t stream, float *den_out) {
     const int d_K = basis.d_K;
     const int64_t F = basis.F;
     const int ntiles = (int)((F + kTF - 1) / kTF);
@@ -272,7 +274,7 @@ cudaError_t launch_prefill_simt(const DeviceBasis &basis, int BH, int64_t N, int
         launch_begin(kSimtFinish, stream);
         simt_finish_kernel<<<dim3(BH, nchunks), kThreads, smemB, stream>>>(
             (const __nv_bfloat16 *)q, (const __nv_bfloat16 *)k, (const __nv_bfloat16 *)v,
-            partials, ntiles, d_K, d_V, basis.P, inv_c, N, t0, T, (int)Tseg, out);
+            partials, ntiles, d_K, d_V, basis.P, inv_c, N, t0, T, (int)Tseg, out, den_out);
         launch_end(kSimtFinish, stream);
         e = cudaGetLastError();
         if (e != cudaSuccess) return e;

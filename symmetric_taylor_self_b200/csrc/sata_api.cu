@@ -396,6 +396,52 @@ int sata_workspace_bytes(int B, int H, int64_t N, int d_K, int d_V, int P, size_
     return SATA_OK;
 }
 
+int sata_backward_workspace_bytes(int B, int H, int64_t N, int d_K, int d_V, int P, size_t *bytes) {
+    if (!bytes || N < 0) return SATA_EINVAL;
+    int BH = 0;
+    int rc = check_heads(B, H, &BH);
+    if (rc) return rc;
+    rc = check_shape(d_K, d_V, P);
+    if (rc) return rc;
+    *bytes = prefill_backward_workspace_bytes(BH, N, num_features(d_K, P), d_K, d_V);
+    return SATA_OK;
+}
+
+int sata_prefill_backward(const void *q, const void *k, const void *v, const float *dy, float *dq,
+                          float *dk, float *dv, int B, int H, int64_t N, int d_K, int d_V, int P,
+                          void *workspace, size_t ws_bytes, void *stream) {
+    int BH = 0;
+    int rc = check_heads(B, H, &BH);
+    if (rc) return rc;
+    if (N < 0) return SATA_EINVAL;
+    rc = check_shape(d_K, d_V, P);
+    if (rc) return rc;
+    if (N == 0 || BH == 0) return SATA_OK;
+    if (!q || !k || !v || !dy || !dq || !dk || !dv) return SATA_EINVAL;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(dy) || !aligned16(dq) ||
+        !aligned16(dk) || !aligned16(dv))
+        return SATA_EALIGN;
+    if (workspace && !aligned16(workspace)) return SATA_EALIGN;
+    cudaError_t e = cudaSuccess;
+    const DeviceBasis *basis = device_basis(d_K, P, &e);
+    if (!basis) return cuda_fail(e);
+    const size_t need = prefill_backward_workspace_bytes(BH, N, basis->F, d_K, d_V);
+    if (workspace) {
+        if (ws_bytes < need) return SATA_ENOMEM;
+    } else {
+        workspace = device_workspace(3, need, &e);
+        if (!workspace) {
+            g_last_cuda = (int)e;
+            return SATA_ENOMEM;
+        }
+        ws_bytes = need;
+    }
+    e = launch_prefill_backward(*basis, BH, N, d_V, q, k, v, dy, dq, dk, dv, workspace, ws_bytes,
+                                (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e);
+    return SATA_OK;
+}
+
 int sata_prefill_ex(const void *q, const void *k, const void *v, float *out, int B, int H,
                     int64_t N, int d_K, int d_V, int P, sata_state *st, void *workspace,
                     size_t ws_bytes, void *stream) {

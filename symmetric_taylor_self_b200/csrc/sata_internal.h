@@ -67,7 +67,7 @@ const void *device_table(uint64_t key, size_t bytes, const std::function<void(ui
 // Kernel identities for launch statistics.
 enum KernelId {
     kDecodeStream = 0, kDecodeFinish, kSimtScan, kSimtFinish, kTcPrep, kTcScan, kTcFinish, kTcReduce,
-    kNumKernels
+    kBwdR, kBwdQScan, kBwdKVScan, kBwdFinish, kNumKernels
 };
 const char *kernel_name(int id);
 // Call around every kernel launch: begin() records a start event when timing is
@@ -92,7 +92,14 @@ size_t prefill_simt_workspace_bytes(int BH, int64_t N, int64_t F, int d_V, bool 
 cudaError_t launch_prefill_simt(const DeviceBasis &basis, int BH, int64_t N, int d_V,
                                 const void *q, const void *k, const void *v, float *out,
                                 float *S, float *Z, bool state_in, void *ws, size_t ws_bytes,
-                                cudaStream_t stream);
+                                cudaStream_t stream, float *den_out = nullptr);
+
+// ---- backward of the prefill, CUDA-core path (backward_simt.cu) ----
+size_t prefill_backward_workspace_bytes(int BH, int64_t N, int64_t F, int d_K, int d_V);
+cudaError_t launch_prefill_backward(const DeviceBasis &basis, int BH, int64_t N, int d_V,
+                                    const void *q, const void *k, const void *v, const float *dy,
+                                    float *dq, float *dk, float *dv, void *ws, size_t ws_bytes,
+                                    cudaStream_t stream);
 
 // ---- prefill, tensor-core path (prefill_tc.cu) ----
 // Host-buffer prefill: the kernels read and write the device copies passed as q, k, v, out;

@@ -93,6 +93,13 @@ def make_inputs(w: Workload, dtype=torch.bfloat16):
     return pre, dec
 
 
+def random_cotangent(B, H, N, d_V, seed):
+    """Seeded N(0, 1) fp32 [B, H, N, d_V]: an upstream gradient dL/dy for the
+    backward pass (any values will do; a loss's gradient has no special form)."""
+    g = torch.Generator("cpu").manual_seed(seed)
+    return torch.randn(B, H, N, d_V, generator=g)
+
+
 def random_inputs(B, H, N, d_K, d_V, seed, dtype=torch.bfloat16, scale=1.0):
     """Free-form seeded N(0, scale^2) inputs [B, H, N, d] for edge-case tests."""
     g = torch.Generator("cpu").manual_seed(seed)

@@ -32,3 +32,17 @@ def token_rel_err(y, y_ref, kappa=None):
     if not np.all(np.isfinite(y)):
         worst = float("inf")
     return worst, int((~keep).sum()), tensor
+
+
+def tensor_rel_err(g, g_ref):
+    """max |g - g_ref| / max |g_ref| over a whole tensor (the gradients' metric:
+    per-token norms of a gradient can be arbitrarily small, so the error is taken
+    relative to the tensor's largest entry)."""
+    g = np.asarray(g, dtype=np.float64)
+    r = np.asarray(g_ref, dtype=np.float64)
+    if not np.all(np.isfinite(g)):
+        return float("inf")
+    scale = np.abs(r).max()
+    if scale == 0.0:   # an exactly zero reference (e.g. dq, dk at P = 1): absolute error
+        return float(np.abs(g).max())
+    return float(np.abs(g - r).max() / scale)

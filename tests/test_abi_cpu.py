@@ -98,6 +98,10 @@ def test_size_queries(lib):
     assert S == 8 * 47905 * 64 * 4 and Z == 8 * 47905 * 4
     assert (S + Z) // 8 // 4 == 3113825           # (d_V + 1) binom(67, 3) per head
     assert sata_workspace_bytes(1, 8, 65536, 64, 64, 4) > 0
+    from symmetric_taylor_self_b200 import sata_backward_workspace_bytes as bwb
+    small, big = bwb(1, 1, 1000, 16, 16, 4), bwb(1, 1, 100000, 16, 16, 4)
+    # y, den and r are kept for every token: at least (2 d_V + 2) fp32 values per token
+    assert big - small >= (100000 - 1000) * (2 * 16 + 2) * 4
 
 
 def test_argument_validation_needs_no_gpu(lib):
@@ -125,6 +129,14 @@ def test_argument_validation_needs_no_gpu(lib):
     assert lib.sata_prefill_host(fake, fake, fake, fake, 1, 1, 8, 8, 12, 4, None, None) == bd.SATA_EUNSUPPORTED
     assert lib.sata_prefill_host(None, fake, fake, fake, 1, 1, 8, 8, 8, 4, None, None) == bd.SATA_EINVAL
     assert lib.sata_prefill_host(None, None, None, None, 1, 1, 0, 8, 8, 4, None, None) == bd.SATA_OK
+    # backward
+    bw = lambda *a: lib.sata_prefill_backward(*a, None, 0, None)
+    assert bw(fake, fake, fake, fake, fake, fake, fake, 1, 1, 8, 8, 12, 4) == bd.SATA_EUNSUPPORTED
+    assert bw(fake, fake, fake, fake, fake, fake, fake, 1, 1, 8, 8, 8, 9) == bd.SATA_EUNSUPPORTED
+    assert bw(fake, fake, fake, None, fake, fake, fake, 1, 1, 8, 8, 8, 4) == bd.SATA_EINVAL
+    assert bw(fake, fake, fake, fake, fake, fake, fake, 1, -1, 8, 8, 8, 4) == bd.SATA_EINVAL
+    assert bw(fake, fake, fake, fake, fake, vp(0x10004), fake, 1, 1, 8, 8, 8, 4) == bd.SATA_EALIGN
+    assert bw(None, None, None, None, None, None, None, 1, 1, 0, 8, 8, 4) == bd.SATA_OK
     # decode
     assert lib.sata_decode_step(None, fake, fake, fake, fake) == bd.SATA_EINVAL
     st = bd.sata_state(B=1, H=1, d_K=8, d_V=8, P=4, F=999, S=0x10000, Z=0x10000, stream=None, tokens=0)

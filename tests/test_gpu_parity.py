@@ -13,7 +13,7 @@ import pytest
 import torch
 
 from symmetric_taylor_self_b200 import workloads as wl
-from tests.parity import TOL, token_rel_err
+from tests.parity import TOL, tensor_rel_err, token_rel_err
 
 pytestmark = pytest.mark.gpu
 
@@ -339,3 +339,74 @@ def test_out_of_range_inputs_are_reported(sata):
     sata.prefill(q.cuda(), k.cuda(), v.cuda(), P=4)
     assert sata.sata_sync_status() == 0
     sata.sata_set_option(sata.SATA_OPT_PREFILL_PATH, 0)
+
+
+# ------------------------------------------------------------ backward ----
+# sata_prefill_backward against the oracle's chain-rule gradient of the direct
+# form, on every token of the checked heads.  Gate: tensor-wise max error over
+# max |reference| <= TOL for each of dq, dk, dv.
+
+def _check_grads(sata, oracle_mod, B, H, N, d_K, d_V, P, seed, heads=None):
+    q, k, v = wl.random_inputs(B, H, N, d_K, d_V, seed=seed)
+    dy = wl.random_cotangent(B, H, N, d_V, seed=seed + 1)
+    dq, dk, dv = sata.prefill_backward(q.cuda(), k.cuda(), v.cuda(), dy.cuda(), P)
+    torch.cuda.synchronize()
+    heads = heads or [(b, h) for b in range(B) for h in range(H)]
+    ref = oracle_mod.grad_heads(q, k, v, dy, P, heads=heads)
+    for (b, h), (rq, rk, rv) in ref.items():
+        for name, g, r in (("dq", dq, rq), ("dk", dk, rk), ("dv", dv, rv)):
+            err = tensor_rel_err(g[b, h].double().cpu().numpy(), r)
+            assert err <= TOL, f"{name} head {(b, h)} d_K={d_K} d_V={d_V} P={P} N={N}: {err:.3e}"
+    return dq, dk, dv
+
+
+@pytest.mark.parametrize("d_K,d_V,P,N", [(16, 16, 4, 100), (8, 8, 4, 77), (32, 32, 4, 70),
+                                         (64, 64, 4, 130), (16, 32, 3, 65), (12, 8, 2, 50),
+                                         (8, 8, 5, 40), (4, 4, 1, 33), (128, 128, 2, 37)])
+def test_backward_matches_oracle(sata, oracle_mod, d_K, d_V, P, N):
+    _check_grads(sata, oracle_mod, 1, 2, N, d_K, d_V, P, seed=5000 + d_K + P * 3 + N)
+
+
+def test_backward_single_token(sata):
+    """N = 1: y_0 = v_0 whatever q and k are, so dv = dy and dq = dk = 0 (up to
+    rounding: dw = g.v - g.y cancels)."""
+    q, k, v = (x.cuda() for x in wl.random_inputs(1, 2, 1, 8, 16, seed=5050))
+    dy = wl.random_cotangent(1, 2, 1, 16, seed=5051).cuda()
+    dq, dk, dv = sata.prefill_backward(q, k, v, dy, 4)
+    torch.cuda.synchronize()
+    assert torch.allclose(dv, dy, rtol=1e-6, atol=1e-6)
+    assert dq.abs().max().item() <= 1e-5 and dk.abs().max().item() <= 1e-5
+
+
+def test_backward_several_segments(sata, oracle_mod):
+    """d = 64, P = 4 with 8 heads: the partial buffer holds about 1400 tokens,
+    so 3000 tokens run as three segments (S carried forward, G backward)."""
+    _check_grads(sata, oracle_mod, 2, 4, 3000, 64, 64, 4, seed=5100, heads=[(0, 0), (1, 3)])
+
+
+def test_backward_is_deterministic_and_linear_in_dy(sata):
+    q, k, v = (x.cuda() for x in wl.random_inputs(1, 2, 200, 16, 16, seed=5200))
+    dy1 = wl.random_cotangent(1, 2, 200, 16, seed=5201).cuda()
+    dy2 = wl.random_cotangent(1, 2, 200, 16, seed=5202).cuda()
+    a = sata.prefill_backward(q, k, v, dy1, 4)
+    b = sata.prefill_backward(q, k, v, dy1, 4)
+    for x, y in zip(a, b):
+        assert torch.equal(x, y)
+    c = sata.prefill_backward(q, k, v, dy2, 4)
+    s = sata.prefill_backward(q, k, v, dy1 + 2.0 * dy2, 4)
+    for x, y, z in zip(a, c, s):
+        assert torch.allclose(z, x + 2.0 * y, rtol=1e-4, atol=1e-4 * z.abs().max().item())
+
+
+def test_attention_autograd(sata, oracle_mod):
+    """attention() as a torch autograd op: y matches prefill, and .backward()
+    gives the oracle's gradients (cast to the inputs' bf16)."""
+    q, k, v = wl.random_inputs(1, 1, 90, 16, 16, seed=5300)
+    dy = wl.random_cotangent(1, 1, 90, 16, seed=5301)
+    qc, kc, vc = (x.cuda().requires_grad_() for x in (q, k, v))
+    y = sata.attention(qc, kc, vc, 4)
+    y.backward(dy.cuda())
+    rq, rk, rv = oracle_mod.direct_grad(q[0, 0], k[0, 0], v[0, 0], dy[0, 0], 4)
+    for g, r in ((qc.grad, rq), (kc.grad, rk), (vc.grad, rv)):
+        assert g.dtype == torch.bfloat16
+        assert tensor_rel_err(g[0, 0].double().cpu().numpy(), r) <= 1e-2   # bf16 rounding of the gradient
