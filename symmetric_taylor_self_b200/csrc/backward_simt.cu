@@ -36,26 +36,38 @@
 #include <vector>
 
 #include "sata_internal.h"
+#include "simt_tiles.cuh"
 
 namespace sata {
 namespace {
 
-constexpr int kThreads = 256;
-constexpr int kTF = 128;   // features per CTA
-constexpr int kL = 32;     // chunk length
+using simt::kThreads;
+using simt::kTF;
+using simt::kL;
+using simt::contract_rows;
+using simt::readout_cols;
+using simt::update_rows;
 constexpr int kMaxComp = kMaxP - 2;   // indices left of a top-degree feature after removing one
 constexpr size_t kPartialBudget = size_t(2) << 30;  // bytes of partials per segment
 
-// Jacobian table of one (d_K, P): for every feature tile and every input index
-// i, the features of the tile that contain i.  Entry (uint64):
-//   bits 0..7 the feature's position in its tile, 8..15 the multiplicity of i,
-//   16..63 the feature's other indices (one copy of i removed), 8 bits each,
+// Features are dealt to the kTF-feature tiles round-robin: tile tau holds the
+// features f = tau + m * ntiles, m = 0, 1, ...  The set of monomials of a
+// degree is symmetric under relabelling the indices, so a strided sample of it
+// contains every index about equally often: the Jacobian lists below have
+// nearly equal lengths (a lexicographic block of 128 features would put one
+// leading index in every feature and leave the other lists nearly empty).
+//
+// Jacobian table of one (d_K, P): for every tile and every input index i, the
+// tile's features that contain i.  Entry (uint64):
+//   bits 0..7 the feature's position m in its tile, 8..15 the multiplicity of
+//   i, 16..63 the feature's other indices (one copy of i removed), 8 bits each,
 //   padded with d_K (the constant 1).
 // Layout: uint32 offsets[ntiles][d_K + 1] (into the entry array), then the
 // entries, 8-byte aligned.
 struct JacTable {
     std::vector<uint8_t> image;
     size_t off_entries = 0;
+    int max_entries = 0;   // longest per-tile entry list
 };
 
 bool build_jac_table(int d_K, int P, JacTable &jt) {
@@ -67,19 +79,20 @@ bool build_jac_table(int d_K, int P, JacTable &jt) {
     for (int64_t f = 0; f < F; ++f) {
         const auto &t = hb.tuples[f];
         const int p = (int)t.size();
+        const int64_t tile = f % ntiles, m = f / ntiles;
         size_t s = 0;
         while (s < t.size()) {   // runs of equal indices: one entry per distinct index
             size_t e = s;
             while (e < t.size() && t[e] == t[s]) ++e;
-            uint64_t ent = (uint64_t)(f % kTF) | ((uint64_t)(e - s) << 8);
-            int m = 0;
+            uint64_t ent = (uint64_t)m | ((uint64_t)(e - s) << 8);
+            int c = 0;
             for (int x = 0; x < p; ++x) {
                 if (x == (int)s) continue;   // drop one copy of the index
-                ent |= (uint64_t)t[x] << (16 + 8 * m);
-                ++m;
+                ent |= (uint64_t)t[x] << (16 + 8 * c);
+                ++c;
             }
-            for (; m < kMaxComp; ++m) ent |= (uint64_t)d_K << (16 + 8 * m);
-            lists[(size_t)(f / kTF) * d_K + t[s]].push_back(ent);
+            for (; c < kMaxComp; ++c) ent |= (uint64_t)d_K << (16 + 8 * c);
+            lists[(size_t)tile * d_K + t[s]].push_back(ent);
             s = e;
         }
     }
@@ -91,18 +104,21 @@ bool build_jac_table(int d_K, int P, JacTable &jt) {
     uint32_t *off = (uint32_t *)jt.image.data();
     uint64_t *ent = (uint64_t *)(jt.image.data() + jt.off_entries);
     size_t pos = 0;
+    jt.max_entries = 0;
     for (int64_t tile = 0; tile < ntiles; ++tile) {
+        const size_t start = pos;
         for (int i = 0; i < d_K; ++i) {
             off[tile * (d_K + 1) + i] = (uint32_t)pos;
             for (uint64_t e : lists[(size_t)tile * d_K + i]) ent[pos++] = e;
         }
         off[tile * (d_K + 1) + d_K] = (uint32_t)pos;
+        if ((int)(pos - start) > jt.max_entries) jt.max_entries = (int)(pos - start);
     }
     return true;
 }
 
 // Device copy of the table, cached per (device, d_K, P).
-const uint8_t *jac_table(int d_K, int P, size_t *off_entries, cudaError_t *err) {
+const uint8_t *jac_table(int d_K, int P, size_t *off_entries, int *max_entries, cudaError_t *err) {
     static std::mutex mu;
     static std::map<std::pair<int, int>, JacTable> cache;
     const JacTable *jt = nullptr;
@@ -121,29 +137,27 @@ const uint8_t *jac_table(int d_K, int P, size_t *off_entries, cudaError_t *err) 
         jt = &it->second;
     }
     *off_entries = jt->off_entries;
-    const uint64_t key = (uint64_t(0xB0) << 56) | ((uint64_t)d_K << 16) | (uint64_t)P;
+    *max_entries = jt->max_entries;
+    const uint64_t key = (uint64_t(0xB1) << 56) | ((uint64_t)d_K << 16) | (uint64_t)P;
     return (const uint8_t *)device_table(
         key, jt->image.size(), [jt](uint8_t *h) { std::memcpy(h, jt->image.data(), jt->image.size()); },
         err);
 }
 
-// phi_f(x~) for the packed feature word(s): x~ is a row of d_K + 1 values whose
-// last one is the constant 1.
-__device__ __forceinline__ float feature(const float *x, uint32_t w, const uint32_t *packed_hi,
-                                         int64_t fg) {
+// phi_f(x~) for a feature's packed words: x~ is a row of d_K + 1 values whose
+// last one is the constant 1; hi = the leading indices (degrees above 3), or
+// all d_K when there are none.
+__device__ __forceinline__ float feature(const float *x, uint32_t w, uint32_t hi) {
     float v = x[w & 255] * x[(w >> 8) & 255] * x[(w >> 16) & 255];
-    if (packed_hi) {   // degrees above 3: the leading indices
-        const uint32_t wh = packed_hi[fg];
 #pragma unroll
-        for (int m = 0; m < 4; ++m) v *= x[(wh >> (8 * m)) & 255];
-    }
+    for (int m = 0; m < 4; ++m) v *= x[(hi >> (8 * m)) & 255];
     return v;
 }
 
-// J_phi(x~)^T applied to one tile's feature values `val` (one token):
-// sum over the tile's features f containing index i of val[f] * d phi_f / d x_i.
-__device__ __forceinline__ float jac_t(const uint32_t *__restrict__ off, const uint64_t *__restrict__ ent,
-                                       int i, const float *x, const float *val, int ncomp) {
+// J_phi(x~)^T applied to one token's tile values `val`: the sum over the
+// tile's features f containing index i of val[f] * d phi_f / d x_i.
+__device__ __forceinline__ float jac_t(const uint32_t *off, const uint64_t *ent, int i, const float *x,
+                                       const float *val, int ncomp) {
     const uint32_t b = off[i], e = off[i + 1];
     float acc = 0.f;
     for (uint32_t n = b; n < e; ++n) {
@@ -184,6 +198,35 @@ __device__ __forceinline__ void load_chunk(const __nv_bfloat16 *q, const __nv_bf
     }
 }
 
+// Shared-memory image of one tile: its features' packed words and weights, its
+// Jacobian lists (offsets rebased to 0), and its state rows.
+struct TileSmem {
+    uint64_t *ent;     // [max_entries]
+    uint32_t *off;     // [d_K + 1]
+    uint32_t *pk;      // [kTF] packed word (padding rows: the constant feature)
+    uint32_t *hi;      // [kTF] leading indices (all d_K when P <= 4)
+    float *coef;       // [kTF] a_f (0 on padding rows)
+};
+
+__device__ __forceinline__ void load_tile(TileSmem ts, const uint32_t *packed, const uint32_t *packed_hi,
+                                          const float *coef, const uint32_t *jac_off, const uint64_t *jac_ent,
+                                          int tile, int ntiles, int nf, int d_K) {
+    const uint32_t pad = (uint32_t)d_K | ((uint32_t)d_K << 8) | ((uint32_t)d_K << 16);
+    const uint32_t pad_hi = pad | ((uint32_t)d_K << 24);
+    for (int m = threadIdx.x; m < kTF; m += kThreads) {
+        const int64_t fg = (int64_t)tile + (int64_t)m * ntiles;
+        const bool ok = m < nf;
+        ts.pk[m] = ok ? packed[fg] : pad;
+        ts.hi[m] = (ok && packed_hi) ? packed_hi[fg] : pad_hi;
+        ts.coef[m] = ok ? coef[fg] : 0.f;
+    }
+    const uint32_t *toff = jac_off + (size_t)tile * (d_K + 1);
+    const uint32_t base = toff[0];
+    for (int i = threadIdx.x; i <= d_K; i += kThreads) ts.off[i] = toff[i] - base;
+    const uint32_t n = toff[d_K] - base;
+    for (uint32_t e = threadIdx.x; e < n; e += kThreads) ts.ent[e] = jac_ent[base + e];
+}
+
 // r_t = [dy_t / den_t | -(dy_t . y_t) / den_t], one warp per token.
 __global__ void __launch_bounds__(kThreads)
 bwd_r_kernel(const float *__restrict__ dy, const float *__restrict__ y, const float *__restrict__ den,
@@ -203,19 +246,54 @@ bwd_r_kernel(const float *__restrict__ dy, const float *__restrict__ y, const fl
     if (lane == 0) r[row * (d_V + 1) + d_V] = -s;
 }
 
+// Shared-memory layout of the two scan kernels (floats after the tables).
+struct ScanSmem {
+    static size_t tables(int d_K, int max_entries) {
+        size_t b = (size_t)(max_entries > 0 ? max_entries : 1) * sizeof(uint64_t);
+        b += ((size_t)(d_K + 1) + 2 * kTF) * sizeof(uint32_t) + kTF * sizeof(float);
+        return (b + 15) / 16 * 16;
+    }
+    static size_t bytes(int d_K, int d_V, int nphi, int max_entries) {
+        return tables(d_K, max_entries) +
+               sizeof(float) * ((size_t)kTF * (d_V + 1) + 2 * kL * (d_K + 1) + 2 * kL * (d_V + 1) +
+                                (size_t)nphi * kL * kTF);
+    }
+};
+
+__device__ __forceinline__ TileSmem carve_tables(uint8_t *base, int d_K, int max_entries, float **rest) {
+    TileSmem ts;
+    ts.ent = (uint64_t *)base;
+    uint8_t *p = base + (size_t)(max_entries > 0 ? max_entries : 1) * sizeof(uint64_t);
+    ts.off = (uint32_t *)p;
+    p += (d_K + 1) * sizeof(uint32_t);
+    ts.pk = (uint32_t *)p;
+    p += kTF * sizeof(uint32_t);
+    ts.hi = (uint32_t *)p;
+    p += kTF * sizeof(uint32_t);
+    ts.coef = (float *)p;
+    p += kTF * sizeof(float);
+    const size_t used = (size_t)(p - base);
+    *rest = (float *)(base + (used + 15) / 16 * 16);
+    return ts;
+}
+
 // dq partials of one feature tile of one head over the tokens [t0, t0 + T):
 // forward over the chunks with the tile's rows of S = sum phi(k) u^T.
+template <int DV>
 __global__ void __launch_bounds__(kThreads)
 bwd_q_scan_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k,
                   const __nv_bfloat16 *__restrict__ v, const float *__restrict__ r,
                   float *__restrict__ state, const uint32_t *__restrict__ packed,
                   const uint32_t *__restrict__ packed_hi, const float *__restrict__ coef,
                   const uint32_t *__restrict__ jac_off, const uint64_t *__restrict__ jac_ent, int d_K,
-                  int d_V, int ncomp, int64_t F, int64_t N, int64_t t0, int T, int Tseg, int load_state,
-                  float *__restrict__ partials) {
-    extern __shared__ float smem[];
-    const int DK1 = d_K + 1, DV1 = d_V + 1;
-    float *Sx = smem;                  // [kTF][DV1]
+                  int max_entries, int ncomp, int64_t F, int64_t N, int64_t t0, int T, int Tseg,
+                  int load_state, float *__restrict__ partials) {
+    constexpr int DV1 = DV + 1;
+    extern __shared__ __align__(16) uint8_t smem_raw[];
+    const int DK1 = d_K + 1;
+    float *fs;
+    const TileSmem ts = carve_tables(smem_raw, d_K, max_entries, &fs);
+    float *Sx = fs;                    // [kTF][DV1]
     float *xq = Sx + kTF * DV1;        // [kL][DK1]
     float *xk = xq + kL * DK1;
     float *xu = xk + kL * DK1;         // [kL][DV1]
@@ -225,129 +303,120 @@ bwd_q_scan_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__re
 
     const int64_t bh = blockIdx.x;
     const int BH = gridDim.x;
-    const int tile = blockIdx.y;
-    const int64_t f0 = (int64_t)tile * kTF;
-    const int nf = (int)(F - f0 < (int64_t)kTF ? F - f0 : (int64_t)kTF);
+    const int tile = blockIdx.y, ntiles = gridDim.y;
+    const int nf = (int)((F - tile + ntiles - 1) / ntiles);
     const int tid = threadIdx.x;
-    const uint32_t *toff = jac_off + (size_t)tile * (d_K + 1);
-
+    load_tile(ts, packed, packed_hi, coef, jac_off, jac_ent, tile, ntiles, nf, d_K);
     for (int e = tid; e < kTF * DV1; e += kThreads) {
-        const int f = e / DV1;
-        Sx[e] = (load_state && f < nf) ? state[(bh * F + f0) * DV1 + e] : 0.f;
+        const int m = e / DV1, j = e % DV1;
+        Sx[e] = (load_state && m < nf) ? state[(bh * F + tile + (int64_t)m * ntiles) * DV1 + j] : 0.f;
     }
     for (int c0 = 0; c0 < T; c0 += kL) {
         const int nt = min(kL, T - c0);
         __syncthreads();
-        load_chunk(q, k, v, r, bh * N + t0 + c0, nt, d_K, d_V, xq, xk, xu, xr);
+        load_chunk(q, k, v, r, bh * N + t0 + c0, nt, d_K, DV, xq, xk, xu, xr);
         __syncthreads();
         for (int e = tid; e < kL * kTF; e += kThreads) {
-            const int t = e / kTF, f = e % kTF;
-            float pk = 0.f, vl = 0.f;
-            if (t < nt && f < nf) {
-                pk = feature(xk + t * DK1, packed[f0 + f], packed_hi, f0 + f);
-                float acc = 0.f;
-                for (int j = 0; j < DV1; ++j) acc = fmaf(Sx[f * DV1 + j], xr[t * DV1 + j], acc);
-                vl = coef[f0 + f] * acc;
-            }
-            phik[e] = pk;
-            val[e] = vl;
+            const int t = e / kTF, m = e % kTF;
+            phik[e] = (t < nt && m < nf) ? feature(xk + t * DK1, ts.pk[m], ts.hi[m]) : 0.f;
         }
+        contract_rows<DV1>(Sx, xr, ts.coef, val);   // a (.) S r_t (zero rows past nt)
         __syncthreads();
         for (int e = tid; e < nt * d_K; e += kThreads) {
             const int t = e / d_K, i = e % d_K;
             partials[(((int64_t)tile * BH + bh) * Tseg + c0 + t) * d_K + i] =
-                jac_t(toff, jac_ent, i, xq + t * DK1, val + t * kTF, ncomp);
+                jac_t(ts.off, ts.ent, i, xq + t * DK1, val + t * kTF, ncomp);
         }
-        for (int e = tid; e < nf * DV1; e += kThreads) {
-            const int f = e / DV1, j = e % DV1;
-            float acc = Sx[e];
-            for (int t = 0; t < nt; ++t) acc = fmaf(phik[t * kTF + f], xu[t * DV1 + j], acc);
-            Sx[e] = acc;
-        }
+        update_rows<DV1>(Sx, phik, xu, nt);          // S += phi(K)^T U
     }
     __syncthreads();
-    for (int e = tid; e < nf * DV1; e += kThreads) state[(bh * F + f0) * DV1 + e] = Sx[e];
+    for (int e = tid; e < nf * DV1; e += kThreads) {
+        const int m = e / DV1, j = e % DV1;
+        state[(bh * F + tile + (int64_t)m * ntiles) * DV1 + j] = Sx[e];
+    }
 }
 
 // dk and dv partials of one feature tile of one head over the tokens
 // [t0, t0 + T): backward over the chunks with the tile's rows of
 // G = sum phi(q) r^T over the tokens after the chunk.
+template <int DV>
 __global__ void __launch_bounds__(kThreads)
 bwd_kv_scan_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k,
                    const __nv_bfloat16 *__restrict__ v, const float *__restrict__ r,
                    float *__restrict__ state, const uint32_t *__restrict__ packed,
                    const uint32_t *__restrict__ packed_hi, const float *__restrict__ coef,
                    const uint32_t *__restrict__ jac_off, const uint64_t *__restrict__ jac_ent, int d_K,
-                   int d_V, int ncomp, int64_t F, int64_t N, int64_t t0, int T, int Tseg,
+                   int max_entries, int ncomp, int64_t F, int64_t N, int64_t t0, int T, int Tseg,
                    int load_state, float *__restrict__ partials) {
-    extern __shared__ float smem[];
-    const int DK1 = d_K + 1, DV1 = d_V + 1, DKV = d_K + d_V;
-    float *Gx = smem;                  // [kTF][DV1]
+    constexpr int DV1 = DV + 1;
+    extern __shared__ __align__(16) uint8_t smem_raw[];
+    const int DK1 = d_K + 1, DKV = d_K + DV;
+    float *fs;
+    const TileSmem ts = carve_tables(smem_raw, d_K, max_entries, &fs);
+    float *Gx = fs;                    // [kTF][DV1]
     float *xq = Gx + kTF * DV1;        // [kL][DK1]
     float *xk = xq + kL * DK1;
     float *xu = xk + kL * DK1;         // [kL][DV1]
     float *xr = xu + kL * DV1;
-    float *phiq = xr + kL * DV1;       // [kL][kTF]
-    float *pka = phiq + kL * kTF;      // [kL][kTF]  a (.) phi(k)
-    float *val = pka + kL * kTF;       // [kL][kTF]  a (.) G u
+    float *pka = xr + kL * DV1;        // [kL][kTF]  a (.) phi(k)
+    float *val = pka + kL * kTF;       // [kL][kTF]  a (.) G u, then phi(q)
 
     const int64_t bh = blockIdx.x;
     const int BH = gridDim.x;
-    const int tile = blockIdx.y;
-    const int64_t f0 = (int64_t)tile * kTF;
-    const int nf = (int)(F - f0 < (int64_t)kTF ? F - f0 : (int64_t)kTF);
-    const int tid = threadIdx.x;
-    const uint32_t *toff = jac_off + (size_t)tile * (d_K + 1);
-
+    const int tile = blockIdx.y, ntiles = gridDim.y;
+    const int nf = (int)((F - tile + ntiles - 1) / ntiles);
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    load_tile(ts, packed, packed_hi, coef, jac_off, jac_ent, tile, ntiles, nf, d_K);
     for (int e = tid; e < kTF * DV1; e += kThreads) {
-        const int f = e / DV1;
-        Gx[e] = (load_state && f < nf) ? state[(bh * F + f0) * DV1 + e] : 0.f;
+        const int m = e / DV1, j = e % DV1;
+        Gx[e] = (load_state && m < nf) ? state[(bh * F + tile + (int64_t)m * ntiles) * DV1 + j] : 0.f;
     }
     const int nchunks = (T + kL - 1) / kL;
     for (int ci = nchunks - 1; ci >= 0; --ci) {
         const int c0 = ci * kL;
         const int nt = min(kL, T - c0);
         __syncthreads();
-        load_chunk(q, k, v, r, bh * N + t0 + c0, nt, d_K, d_V, xq, xk, xu, xr);
+        load_chunk(q, k, v, r, bh * N + t0 + c0, nt, d_K, DV, xq, xk, xu, xr);
         __syncthreads();
         for (int e = tid; e < kL * kTF; e += kThreads) {
-            const int t = e / kTF, f = e % kTF;
-            float pq = 0.f, pk = 0.f, vl = 0.f;
-            if (t < nt && f < nf) {
-                const uint32_t w = packed[f0 + f];
-                const float a = coef[f0 + f];
-                pq = feature(xq + t * DK1, w, packed_hi, f0 + f);
-                pk = a * feature(xk + t * DK1, w, packed_hi, f0 + f);
-                float acc = 0.f;
-                for (int j = 0; j < DV1; ++j) acc = fmaf(Gx[f * DV1 + j], xu[t * DV1 + j], acc);
-                vl = a * acc;
-            }
-            phiq[e] = pq;
-            pka[e] = pk;
-            val[e] = vl;
+            const int t = e / kTF, m = e % kTF;
+            pka[e] = (t < nt && m < nf) ? ts.coef[m] * feature(xk + t * DK1, ts.pk[m], ts.hi[m]) : 0.f;
         }
+        contract_rows<DV1>(Gx, xu, ts.coef, val);   // a (.) G u_s
         __syncthreads();
         for (int e = tid; e < nt * d_K; e += kThreads) {
             const int t = e / d_K, i = e % d_K;
             partials[(((int64_t)tile * BH + bh) * Tseg + c0 + t) * DKV + i] =
-                jac_t(toff, jac_ent, i, xk + t * DK1, val + t * kTF, ncomp);
+                jac_t(ts.off, ts.ent, i, xk + t * DK1, val + t * kTF, ncomp);
         }
-        for (int e = tid; e < nt * d_V; e += kThreads) {
-            const int t = e / d_V, j = e % d_V;
-            float acc = 0.f;
-            for (int f = 0; f < nf; ++f) acc = fmaf(pka[t * kTF + f], Gx[f * DV1 + j], acc);
-            partials[(((int64_t)tile * BH + bh) * Tseg + c0 + t) * DKV + d_K + j] = acc;
+        {   // dv partial: (a (.) phi(k_s))^T G[:, :d_V]
+            constexpr int JV = (DV + 31) / 32;
+            float acc[4][JV];
+            readout_cols<JV, DV1>(pka, Gx, DV, acc);
+#pragma unroll
+            for (int b = 0; b < 4; ++b) {
+                const int t = warp + 8 * b;
+#pragma unroll
+                for (int n = 0; n < JV; ++n) {
+                    const int j = lane + 32 * n;
+                    if (t < nt && j < DV)
+                        partials[(((int64_t)tile * BH + bh) * Tseg + c0 + t) * DKV + d_K + j] = acc[b][n];
+                }
+            }
         }
         __syncthreads();
-        for (int e = tid; e < nf * DV1; e += kThreads) {
-            const int f = e / DV1, j = e % DV1;
-            float acc = Gx[e];
-            for (int t = 0; t < nt; ++t) acc = fmaf(phiq[t * kTF + f], xr[t * DV1 + j], acc);
-            Gx[e] = acc;
+        for (int e = tid; e < kL * kTF; e += kThreads) {   // phi(q) over the consumed values
+            const int t = e / kTF, m = e % kTF;
+            val[e] = (t < nt && m < nf) ? feature(xq + t * DK1, ts.pk[m], ts.hi[m]) : 0.f;
         }
+        __syncthreads();
+        update_rows<DV1>(Gx, val, xr, nt);          // G += phi(Q)^T R
     }
     __syncthreads();
-    for (int e = tid; e < nf * DV1; e += kThreads) state[(bh * F + f0) * DV1 + e] = Gx[e];
+    for (int e = tid; e < nf * DV1; e += kThreads) {
+        const int m = e / DV1, j = e % DV1;
+        state[(bh * F + tile + (int64_t)m * ntiles) * DV1 + j] = Gx[e];
+    }
 }
 
 // Per chunk: sum the tiles' partials in tile order and add the pairs inside the
@@ -479,9 +548,21 @@ BwdLayout bwd_layout(int BH, int64_t N, int64_t F, int d_K, int d_V) {
     return L;
 }
 
-size_t scan_smem(int d_K, int d_V, int nphi) {
-    return sizeof(float) * ((size_t)kTF * (d_V + 1) + 2 * kL * (d_K + 1) + 2 * kL * (d_V + 1) +
-                            (size_t)nphi * kL * kTF);
+using ScanFn = void (*)(const __nv_bfloat16 *, const __nv_bfloat16 *, const __nv_bfloat16 *, const float *,
+                       float *, const uint32_t *, const uint32_t *, const float *, const uint32_t *,
+                       const uint64_t *, int, int, int, int64_t, int64_t, int64_t, int, int, int, float *);
+
+// The scan kernels are compiled per d_V (register tiles sized at compile time).
+bool scan_kernels(int d_V, ScanFn *fq, ScanFn *fkv) {
+    switch (d_V) {
+        case 4: *fq = bwd_q_scan_kernel<4>; *fkv = bwd_kv_scan_kernel<4>; return true;
+        case 8: *fq = bwd_q_scan_kernel<8>; *fkv = bwd_kv_scan_kernel<8>; return true;
+        case 16: *fq = bwd_q_scan_kernel<16>; *fkv = bwd_kv_scan_kernel<16>; return true;
+        case 32: *fq = bwd_q_scan_kernel<32>; *fkv = bwd_kv_scan_kernel<32>; return true;
+        case 64: *fq = bwd_q_scan_kernel<64>; *fkv = bwd_kv_scan_kernel<64>; return true;
+        case 128: *fq = bwd_q_scan_kernel<128>; *fkv = bwd_kv_scan_kernel<128>; return true;
+        default: return false;
+    }
 }
 
 }  // namespace
@@ -501,8 +582,11 @@ cudaError_t launch_prefill_backward(const DeviceBasis &basis, int BH, int64_t N,
     const int ntiles = (int)((F + kTF - 1) / kTF);
     const int ncomp = P > 2 ? P - 2 : 0;
     cudaError_t e = cudaSuccess;
+    ScanFn q_scan = nullptr, kv_scan = nullptr;
+    if (!scan_kernels(d_V, &q_scan, &kv_scan)) return cudaErrorInvalidValue;
     size_t off_ent = 0;
-    const uint8_t *jt = jac_table(d_K, P, &off_ent, &e);
+    int max_ent = 0;
+    const uint8_t *jt = jac_table(d_K, P, &off_ent, &max_ent, &e);
     if (!jt) return e != cudaSuccess ? e : cudaErrorMemoryAllocation;
     const uint32_t *jac_off = (const uint32_t *)jt;
     const uint64_t *jac_ent = (const uint64_t *)(jt + off_ent);
@@ -526,12 +610,13 @@ cudaError_t launch_prefill_backward(const DeviceBasis &basis, int BH, int64_t N,
     launch_end(kBwdR, stream);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
 
-    const size_t smemQ = scan_smem(d_K, d_V, 2), smemKV = scan_smem(d_K, d_V, 3);
+    const size_t smemQ = ScanSmem::bytes(d_K, d_V, 2, max_ent);
+    const size_t smemKV = ScanSmem::bytes(d_K, d_V, 2, max_ent);
     const size_t smemF = sizeof(float) * ((size_t)2 * kL * d_K + 2 * kL * (d_V + 1) + 2 * kL * kL);
-    if ((e = cudaFuncSetAttribute(bwd_q_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if ((e = cudaFuncSetAttribute(q_scan, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   (int)smemQ)) != cudaSuccess)
         return e;
-    if ((e = cudaFuncSetAttribute(bwd_kv_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if ((e = cudaFuncSetAttribute(kv_scan, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   (int)smemKV)) != cudaSuccess)
         return e;
     if ((e = cudaFuncSetAttribute(bwd_finish_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -549,8 +634,8 @@ cudaError_t launch_prefill_backward(const DeviceBasis &basis, int BH, int64_t N,
         const int64_t t0 = (int64_t)sg * Tseg;
         const int T = (int)(N - t0 < Tseg ? N - t0 : Tseg);
         launch_begin(kBwdQScan, stream);
-        bwd_q_scan_kernel<<<dim3(BH, ntiles), kThreads, smemQ, stream>>>(
-            qb, kb, vb, r, state, basis.packed, basis.packed_hi, basis.coef, jac_off, jac_ent, d_K, d_V,
+        q_scan<<<dim3(BH, ntiles), kThreads, smemQ, stream>>>(
+            qb, kb, vb, r, state, basis.packed, basis.packed_hi, basis.coef, jac_off, jac_ent, d_K, max_ent,
             ncomp, F, N, t0, T, (int)Tseg, sg > 0 ? 1 : 0, partials);
         launch_end(kBwdQScan, stream);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
@@ -565,8 +650,8 @@ cudaError_t launch_prefill_backward(const DeviceBasis &basis, int BH, int64_t N,
         const int64_t t0 = (int64_t)sg * Tseg;
         const int T = (int)(N - t0 < Tseg ? N - t0 : Tseg);
         launch_begin(kBwdKVScan, stream);
-        bwd_kv_scan_kernel<<<dim3(BH, ntiles), kThreads, smemKV, stream>>>(
-            qb, kb, vb, r, state, basis.packed, basis.packed_hi, basis.coef, jac_off, jac_ent, d_K, d_V,
+        kv_scan<<<dim3(BH, ntiles), kThreads, smemKV, stream>>>(
+            qb, kb, vb, r, state, basis.packed, basis.packed_hi, basis.coef, jac_off, jac_ent, d_K, max_ent,
             ncomp, F, N, t0, T, (int)Tseg, sg < nseg - 1 ? 1 : 0, partials);
         launch_end(kBwdKVScan, stream);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;

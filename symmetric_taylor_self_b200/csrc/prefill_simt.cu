@@ -22,13 +22,14 @@
 #include <cuda_bf16.h>
 
 #include "sata_internal.h"
+#include "simt_tiles.cuh"
 
 namespace sata {
 namespace {
 
-constexpr int kThreads = 256;
-constexpr int kTF = 128;   // features per CTA
-constexpr int kL = 32;     // chunk length
+using simt::kThreads;
+using simt::kTF;
+using simt::kL;
 constexpr size_t kPartialBudget = size_t(2) << 30;  // bytes of partials per segment
 
 struct SimtSmem {
@@ -39,16 +40,19 @@ struct SimtSmem {
 };
 
 // Kernel A: inter-chunk readout partials and state update for one feature tile
-// of one head over the tokens [t0, t0 + T) of a segment.
+// of one head over the tokens [t0, t0 + T) of a segment (compiled per d_V: the
+// two contractions are register-tiled, simt_tiles.cuh).
+template <int DV>
 __global__ void __launch_bounds__(kThreads)
 simt_scan_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k,
                  const __nv_bfloat16 *__restrict__ v, float *__restrict__ S,
                  float *__restrict__ Z, const uint32_t *__restrict__ packed,
-                 const uint32_t *__restrict__ packed_hi, const float *__restrict__ coef, int d_K, int d_V,
+                 const uint32_t *__restrict__ packed_hi, const float *__restrict__ coef, int d_K,
                  int64_t F, int64_t N,
                  int64_t t0, int T, int Tseg, int load_state, float *__restrict__ partials) {
+    constexpr int d_V = DV, DV1 = DV + 1;
     extern __shared__ float smem[];
-    const int DK1 = d_K + 1, DV1 = d_V + 1;
+    const int DK1 = d_K + 1;
     float *Sx = smem;                       // [kTF][DV1]
     float *xq = Sx + kTF * DV1;             // [kL][DK1]
     float *xk = xq + kL * DK1;              // [kL][DK1]
@@ -115,21 +119,24 @@ simt_scan_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__res
             aq[e] = pq;
         }
         __syncthreads();
-        // readout against the state before this chunk
-        for (int e = tid; e < nt * DV1; e += kThreads) {
-            const int t = e / DV1, j = e % DV1;
-            float acc = 0.f;
-            for (int f = 0; f < nf; ++f) acc = fmaf(aq[t * kTF + f], Sx[f * DV1 + j], acc);
-            partials[(((int64_t)tile * gridDim.x + bh) * Tseg + c0 + t) * DV1 + j] = acc;
+        {   // readout against the state before this chunk (rows past nf are zero)
+            constexpr int JV = (DV1 + 31) / 32;
+            float acc[4][JV];
+            simt::readout_cols<JV, DV1>(aq, Sx, DV1, acc);
+            const int lane = tid & 31, warp = tid >> 5;
+#pragma unroll
+            for (int b = 0; b < 4; ++b) {
+                const int t = warp + 8 * b;
+#pragma unroll
+                for (int n = 0; n < JV; ++n) {
+                    const int j = lane + 32 * n;
+                    if (t < nt && j < DV1)
+                        partials[(((int64_t)tile * gridDim.x + bh) * Tseg + c0 + t) * DV1 + j] = acc[b][n];
+                }
+            }
         }
         __syncthreads();
-        // update with this chunk
-        for (int e = tid; e < nf * DV1; e += kThreads) {
-            const int f = e / DV1, j = e % DV1;
-            float acc = Sx[e];
-            for (int t = 0; t < nt; ++t) acc = fmaf(phik[t * kTF + f], xv[t * DV1 + j], acc);
-            Sx[e] = acc;
-        }
+        simt::update_rows<DV1>(Sx, phik, xv, nt);   // update with this chunk
     }
     __syncthreads();
     for (int e = tid; e < nf * DV1; e += kThreads) {
@@ -250,10 +257,23 @@ cudaError_t launch_prefill_simt(const DeviceBasis &basis, int BH, int64_t N, int
         Z = S + (size_t)BH * F * d_V;
         state_in = false;
     }
+    using ScanFn = void (*)(const __nv_bfloat16 *, const __nv_bfloat16 *, const __nv_bfloat16 *, float *,
+                            float *, const uint32_t *, const uint32_t *, const float *, int, int64_t,
+                            int64_t, int64_t, int, int, int, float *);
+    ScanFn scan = nullptr;
+    switch (d_V) {
+        case 4: scan = simt_scan_kernel<4>; break;
+        case 8: scan = simt_scan_kernel<8>; break;
+        case 16: scan = simt_scan_kernel<16>; break;
+        case 32: scan = simt_scan_kernel<32>; break;
+        case 64: scan = simt_scan_kernel<64>; break;
+        case 128: scan = simt_scan_kernel<128>; break;
+        default: return cudaErrorInvalidValue;
+    }
     const size_t smemA = SimtSmem::bytes(d_K, d_V);
     const size_t smemB = sizeof(float) * ((size_t)2 * kL * d_K + kL * (d_V + 1) + kL * kL +
                                           kL * (d_V + 1));
-    cudaError_t e = cudaFuncSetAttribute(simt_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(scan, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smemA);
     if (e != cudaSuccess) return e;
     e = cudaFuncSetAttribute(simt_finish_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -264,9 +284,9 @@ cudaError_t launch_prefill_simt(const DeviceBasis &basis, int BH, int64_t N, int
         const int T = (int)(N - t0 < Tseg ? N - t0 : Tseg);
         const int load = (t0 > 0 || state_in) ? 1 : 0;
         launch_begin(kSimtScan, stream);
-        simt_scan_kernel<<<dim3(BH, ntiles), kThreads, smemA, stream>>>(
+        scan<<<dim3(BH, ntiles), kThreads, smemA, stream>>>(
             (const __nv_bfloat16 *)q, (const __nv_bfloat16 *)k, (const __nv_bfloat16 *)v, S, Z,
-            basis.packed, basis.packed_hi, basis.coef, d_K, d_V, F, N, t0, T, (int)Tseg, load, partials);
+            basis.packed, basis.packed_hi, basis.coef, d_K, F, N, t0, T, (int)Tseg, load, partials);
         launch_end(kSimtScan, stream);
         e = cudaGetLastError();
         if (e != cudaSuccess) return e;
