@@ -7,7 +7,8 @@ One "step" is one causal SATA prefill of the d_K = d_V = 64, P = 4 workload
 (B=1, H=8, N=65536: 47905 features per head) through the C ABI, inputs resident
 in HBM.  Decode is measured beside it on the decode workload (B=64, H=32,
 d_K = d_V = 32, a state built by an 8192-token prefill, then decode steps) and
-reported under "decode".  For N > 1 (torchrun) every rank runs its own copy of
+reported under "decode", and the backward pass of the prefill (gradients of q,
+k, v on the d = 64, P = 4 head shape over 4096 tokens) under "backward".  For N > 1 (torchrun) every rank runs its own copy of
 the workload on its own GPU (weak scaling, no collective on the data path);
 times are max over ranks.
 
@@ -48,7 +49,9 @@ def parse():
     ap.add_argument("--decode-workload", default="decode_d32")
     ap.add_argument("--decode-steps", type=int, default=256)
     ap.add_argument("--no-decode", action="store_true")
-    ap.add_argument("--only", choices=["all", "prefill", "decode"], default="all",
+    ap.add_argument("--backward-workload", default="backward_d64")
+    ap.add_argument("--no-backward", action="store_true")
+    ap.add_argument("--only", choices=["all", "prefill", "decode", "backward"], default="all",
                     help="run one part only (reduced workloads for profiler captures)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
@@ -400,6 +403,11 @@ def main():
     if not args.no_decode:
         dec = bench_decode(torch, sata, wl, args, world, dev, stream, peaks, peaks_src)
 
+    # ---------------- backward of the prefill ----------------
+    bwd = None
+    if not args.no_backward:
+        bwd = bench_backward(torch, sata, wl, args, world, dev, stream, clocks)
+
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True,
@@ -411,6 +419,7 @@ def main():
                    "l2": f"inputs {in_bytes / 1e6:.0f} MB + output {out_bytes / 1e6:.0f} MB per step > 126 MB L2",
                    "path": args.path},
         "roofline": roof, "gpu_launches": launches, "clocks": clocks, "e2e": e2e, "decode": dec,
+        "backward": bwd,
         "kernel_ms": {k_: {"launches": n, "ms": t} for k_, (n, t) in stats.items()},
         "peaks_source": peaks_src,
     }
@@ -428,7 +437,14 @@ def run_part(torch, sata, wl, args, world):
     """One part alone, no JSON line: the command profiler captures run."""
     dev = torch.device("cuda", torch.cuda.current_device())
     stream = torch.cuda.Stream()
-    if args.only == "prefill":
+    if args.only == "backward":
+        w = wl.WORKLOADS[args.backward_workload]
+        (q, k, v), _ = wl.make_inputs(w)
+        qd, kd, vd, dy = q.to(dev), k.to(dev), v.to(dev), wl.cotangent(w).to(dev)
+        g = [torch.empty(x.shape, dtype=torch.float32, device=dev) for x in (q, k, v)]
+        for _ in range(args.warmup + args.steps):
+            sata.sata_prefill_backward(qd, kd, vd, dy, *g, w.B, w.H, w.N, w.d_K, w.d_V, w.P, None, stream)
+    elif args.only == "prefill":
         w = wl.WORKLOADS[args.workload]
         (q, k, v), _ = wl.make_inputs(w)
         qd, kd, vd = q.to(dev), k.to(dev), v.to(dev)
@@ -448,6 +464,64 @@ def run_part(torch, sata, wl, args, world):
     status = sata.sata_sync_status(stream)
     print(json.dumps({"part": args.only, "status": status}), flush=True)
     return 0 if status == 0 else 1
+
+
+def backward_flops(d_K, d_V, P):
+    """Algorithmic FLOPs per token and head of the backward's two scans (the
+    feature-form contractions; the Jacobian products and features not counted):
+    dq scan: S r_t and the S update, 2 x 2F(d_V+1);
+    dk/dv scan: G u_s, the dv readout 2F d_V, the G update: 4F(d_V+1) + 2F d_V."""
+    F = math.comb(d_K + P - 1, P - 1)
+    return {"bwd_q_scan": 4 * F * (d_V + 1), "bwd_kv_scan": 4 * F * (d_V + 1) + 2 * F * d_V}
+
+
+def bench_backward(torch, sata, wl, args, world, dev, stream, clocks):
+    w = wl.WORKLOADS[args.backward_workload]
+    (q, k, v), _ = wl.make_inputs(w)
+    qd, kd, vd, dy = q.to(dev), k.to(dev), v.to(dev), wl.cotangent(w).to(dev)
+    dq = torch.empty((w.B, w.H, w.N, w.d_K), dtype=torch.float32, device=dev)
+    dk = torch.empty_like(dq)
+    dv = torch.empty((w.B, w.H, w.N, w.d_V), dtype=torch.float32, device=dev)
+
+    def step():
+        sata.sata_prefill_backward(qd, kd, vd, dy, dq, dk, dv, w.B, w.H, w.N, w.d_K, w.d_V, w.P, None,
+                                   stream)
+
+    with torch.cuda.stream(stream):
+        step()                                   # allocates the library workspace
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    sata.sata_reset_kernel_stats()
+    sata.sata_set_option(sata.SATA_OPT_TIME_KERNELS, 1)
+    ms = timed(torch, world, step, args.steps, 0, stream)
+    stats = sata.sata_kernel_stats()
+    sata.sata_set_option(sata.SATA_OPT_TIME_KERNELS, 0)
+    if sata.sata_sync_status(stream) != 0:
+        raise RuntimeError("device status after the backward")
+    value = job_throughput(w.B * w.N, args.steps, world, ms)
+    per_tok = backward_flops(w.d_K, w.d_V, w.P)
+    sm_ghz = (clocks.get("sm_max_mhz") or 1965.0) / 1000.0
+    alu_peak = NUM_SMS * FP32_LANES_PER_SM * 2 * sm_ghz / 1000.0
+    roof = None
+    scans = {k_: stats[k_] for k_ in per_tok if k_ in stats}
+    if scans:
+        dom = max(scans, key=lambda n: scans[n][1])
+        n_l, ms_l = scans[dom]
+        flops_per_launch = per_tok[dom] * w.B * w.H * w.N * args.steps / n_l
+        achieved = flops_per_launch / (ms_l / n_l / 1000.0) / 1e12
+        roof = {"bound": "alu", "achieved": achieved, "peak": alu_peak, "unit": "TFLOP/s",
+                "frac": achieved / alu_peak, "kernel": dom, "launches_per_step": n_l / args.steps,
+                "ms_per_launch": ms_l / n_l, "algorithmic_flops_per_launch": flops_per_launch,
+                "peak_kind": "fp32 FMA: 148 SMs x 128 lanes x 2 FLOP x max SM clock",
+                "traffic": ncu_traffic(dom)}
+    return {"metric": "SATA prefill backward tokens/s (dq, dk, dv)", "value": value, "unit": "tokens/s",
+            "steps": args.steps, "ms_per_step": ms / args.steps,
+            "workload": f"{w.name}: B={w.B} H={w.H} N={w.N} d_K={w.d_K} d_V={w.d_V} P={w.P} F={w.F}; "
+                        f"dy N(0,1) fp32; the step recomputes the forward (CUDA-core, fp32)",
+            "l2": "each step writes more than 1 GB of partial sums, far above the 126 MB L2",
+            "roofline": roof, "gpu_launches": sum(n for n, _ in stats.values()),
+            "kernel_ms": {k_: {"launches": n, "ms": t} for k_, (n, t) in stats.items()}}
 
 
 def bench_decode(torch, sata, wl, args, world, dev, stream, peaks, peaks_src):

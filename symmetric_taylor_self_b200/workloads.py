@@ -54,10 +54,17 @@ WORKLOADS = {
                             oracle_heads=((0, 0),), oracle_tokens=2048),
     "decode_d32": Workload("decode_d32", B=64, H=32, N=8192, d_K=32, d_V=32, P=4, seed=4,
                            steps=1024, oracle_heads=((0, 0), (63, 31), (17, 5), (40, 22))),
-    # reduced sizes of the two benchmark workloads, for ncu captures
+    # backward pass of the prefill (gradients of q, k, v): the prefill_d64 head
+    # shape over 4096 tokens; the upstream gradient dy is N(0, 1) (cotangent())
+    "backward_d64": Workload("backward_d64", B=1, H=8, N=4096, d_K=64, d_V=64, P=4, seed=5,
+                             oracle_heads=((0, 0),)),
+    "backward_d16": Workload("backward_d16", B=1, H=8, N=4096, d_K=16, d_V=16, P=4, seed=6,
+                             oracle_heads=((0, 3),)),
+    # reduced sizes of the benchmark workloads, for ncu captures
     "prefill_d64_small": Workload("prefill_d64_small", B=1, H=8, N=8192, d_K=64, d_V=64, P=4, seed=3),
     "decode_d32_small": Workload("decode_d32_small", B=8, H=32, N=256, d_K=32, d_V=32, P=4, seed=4,
                                  steps=16),
+    "backward_d64_small": Workload("backward_d64_small", B=1, H=4, N=1024, d_K=64, d_V=64, P=4, seed=5),
 }
 
 
@@ -98,6 +105,11 @@ def random_cotangent(B, H, N, d_V, seed):
     backward pass (any values will do; a loss's gradient has no special form)."""
     g = torch.Generator("cpu").manual_seed(seed)
     return torch.randn(B, H, N, d_V, generator=g)
+
+
+def cotangent(w: Workload):
+    """The upstream gradient dy [B, H, N, d_V] (fp32, N(0, 1)) of a backward workload."""
+    return random_cotangent(w.B, w.H, w.N, w.d_V, seed=w.seed * 2 ** 20 + 2 ** 19)
 
 
 def random_inputs(B, H, N, d_K, d_V, seed, dtype=torch.bfloat16, scale=1.0):

@@ -410,3 +410,20 @@ def test_attention_autograd(sata, oracle_mod):
     for g, r in ((qc.grad, rq), (kc.grad, rk), (vc.grad, rv)):
         assert g.dtype == torch.bfloat16
         assert tensor_rel_err(g[0, 0].double().cpu().numpy(), r) <= 1e-2   # bf16 rounding of the gradient
+
+
+@pytest.mark.parametrize("name", ["backward_d64", "backward_d16"])
+def test_backward_workload_full_size(sata, oracle_mod, name):
+    """The benchmark's backward workloads at full size, in the benchmark's
+    launch configuration (all heads, library workspace); the oracle checks
+    every token of the listed heads."""
+    w = wl.WORKLOADS[name]
+    (q, k, v), _ = wl.make_inputs(w)
+    dy = wl.cotangent(w)
+    dq, dk, dv = sata.prefill_backward(q.cuda(), k.cuda(), v.cuda(), dy.cuda(), w.P)
+    torch.cuda.synchronize()
+    ref = oracle_mod.grad_heads(q, k, v, dy, w.P, heads=list(w.oracle_heads))
+    for (b, h), (rq, rk, rv) in ref.items():
+        for nm, g, r in (("dq", dq, rq), ("dk", dk, rk), ("dv", dv, rv)):
+            err = tensor_rel_err(g[b, h].double().cpu().numpy(), r)
+            assert err <= TOL, f"{name} {nm} head {(b, h)}: {err:.3e}"
