@@ -250,8 +250,16 @@ enum sata_option {
     SATA_OPT_TEST_STALL = 3,     /* 1: the next tensor-core prefill launch withholds
                                     one producer signal, so its bounded wait expires
                                     (tests the SATA_ETIMEOUT path); auto-resets */
-    SATA_OPT_TIME_KERNELS = 4    /* 1: bracket every kernel launch with CUDA events on
+    SATA_OPT_TIME_KERNELS = 4,   /* 1: bracket every kernel launch with CUDA events on
                                     its own stream (read with sata_kernel_stats) */
+    SATA_OPT_DETERMINISTIC = 5   /* tensor-core prefill: 0 (default) adds each feature
+                                    group's inter-chunk partial sums into one fp32 buffer
+                                    with atomic adds (resolved in L2; the order of the
+                                    additions, and so the last bits of the output, can
+                                    differ between runs); 1 writes every group's partial
+                                    and sums them in a fixed order (bitwise reproducible,
+                                    one more pass over the partials through HBM).  The
+                                    CUDA-core paths and the decode are always reproducible. */
 };
 SATA_API int sata_set_option(int key, int64_t value);
 SATA_API int sata_get_option(int key, int64_t *value);

@@ -29,6 +29,7 @@ SATA_OPT_PREFILL_PATH = 1
 SATA_OPT_WAIT_LIMIT = 2
 SATA_OPT_TEST_STALL = 3
 SATA_OPT_TIME_KERNELS = 4
+SATA_OPT_DETERMINISTIC = 5
 
 EXPORTED = (
     "sata_status_string", "sata_last_cuda_error", "sata_version", "sata_num_features",

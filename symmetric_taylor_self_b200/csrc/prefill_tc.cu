@@ -115,7 +115,8 @@ struct ScanParams {
     const float *unit_coef;     // [G][MT_MAX][128] C/p! of feature (pair, l), 0 if none
     const int32_t *unit_fidx;   // [G][MT_MAX][128] basis index of feature (pair, l), -1 if none
     float *S, *Z;               // state in/out
-    float *part;                // [BH][G][nc][DV+1][128]
+    float *part;                // [BH][G][nc][DV+1][128], or with red_atomic the sums [BH][nc][DV+1][128]
+    int red_atomic;             // 1: add R into the sums in L2 (fp32 atomics); 0: one partial per unit
     int *flags;
     int64_t F, N;
     int BH, G, c0, nc, nchunks, P;
@@ -672,7 +673,8 @@ __global__ void __launch_bounds__(kScanThreads, 1) tc_scan_kernel(const ScanPara
         const int quarter = warp & 3;
         const int t = quarter * 32 + lane;               // token row of the chunk = TMEM lane
         const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
-        const int64_t part_base = ((int64_t)bh * p.G + u) * p.nc;
+        // one partial row block per (unit, chunk), or the head's shared sums (added in L2)
+        const int64_t part_base = p.red_atomic ? (int64_t)bh * p.nc : ((int64_t)bh * p.G + u) * p.nc;
         int qa = 0;
         bool ok = true;
         // R of chunk cl -> partial (x 2^sigma_cl); the caller has seen the completion of the
@@ -686,9 +688,15 @@ __global__ void __launch_bounds__(kScanThreads, 1) tc_scan_kernel(const ScanPara
                 uint32_t rr[16];
                 tc_ld16(tmem + lane_off + C::COL_R + c16 * 16, rr);
                 tc_wait_ld();
+                if (p.red_atomic) {
 #pragma unroll
-                for (int i = 0; i < 16; ++i)
-                    if (c16 * 16 + i <= D) dst[(c16 * 16 + i) * kL] = __uint_as_float(rr[i]) * up;
+                    for (int i = 0; i < 16; ++i)
+                        if (c16 * 16 + i <= D) atomicAdd(dst + (c16 * 16 + i) * kL, __uint_as_float(rr[i]) * up);
+                } else {
+#pragma unroll
+                    for (int i = 0; i < 16; ++i)
+                        if (c16 * 16 + i <= D) dst[(c16 * 16 + i) * kL] = __uint_as_float(rr[i]) * up;
+                }
             }
             tc_before();
             __syncwarp();
@@ -1315,7 +1323,14 @@ cudaError_t run(const DeviceBasis &basis, int BH, int64_t N, const void *q, cons
         sp.unit_fidx = (const int32_t *)(tab + up.off_fidx);
         sp.S = S;
         sp.Z = Z;
-        sp.part = part;
+        float *red = (float *)(w + pl.off_red);
+        const int nc_here = (pl.nchunks - s * pl.nc_seg < pl.nc_seg) ? pl.nchunks - s * pl.nc_seg : pl.nc_seg;
+        const bool atomic = g_opt_deterministic == 0;
+        if (atomic && (e = cudaMemsetAsync(red, 0, (size_t)BH * nc_here * (DV + 1) * kL * sizeof(float), stream)) !=
+                          cudaSuccess)
+            return e;
+        sp.part = atomic ? red : part;
+        sp.red_atomic = atomic ? 1 : 0;
         sp.flags = flags;
         sp.F = F;
         sp.N = N;
@@ -1334,13 +1349,14 @@ cudaError_t run(const DeviceBasis &basis, int BH, int64_t N, const void *q, cons
         tc_scan_kernel<DK, DV><<<BH * pl.G, kScanThreads, C::SMEM, stream>>>(sp);
         launch_end(kTcScan, stream);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
-        float *red = (float *)(w + pl.off_red);
-        const int64_t rwork = (int64_t)BH * sp.nc * (DV + 1) * (kL / 4);
-        launch_begin(kTcReduce, stream);
-        tc_reduce_kernel<DV><<<(int)((rwork + 255) / 256 < 148 * 32 ? (rwork + 255) / 256 : 148 * 32), 256, 0, stream>>>(
-            (const float4 *)part, (float4 *)red, BH, pl.G, sp.nc);
-        launch_end(kTcReduce, stream);
-        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        if (!atomic) {   // the units' partials summed in a fixed order
+            const int64_t rwork = (int64_t)BH * sp.nc * (DV + 1) * (kL / 4);
+            launch_begin(kTcReduce, stream);
+            tc_reduce_kernel<DV><<<(int)((rwork + 255) / 256 < 148 * 32 ? (rwork + 255) / 256 : 148 * 32), 256, 0,
+                                   stream>>>((const float4 *)part, (float4 *)red, BH, pl.G, sp.nc);
+            launch_end(kTcReduce, stream);
+            if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        }
         launch_begin(kTcFinish, stream);
         tc_finish_kernel<DK, DV><<<(int)((int64_t)BH * sp.nc), 128, FinCfg<DK, DV>::SMEM, stream>>>(
             qb, kb, vb, red, out, sp.c0, sp.nc, N, basis.P, inv_c, flags, wait_ns);

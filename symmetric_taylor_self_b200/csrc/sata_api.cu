@@ -18,6 +18,7 @@ namespace sata {
 int64_t g_opt_prefill_path = 0;
 int64_t g_opt_wait_limit = 0;
 int64_t g_opt_test_stall = 0;
+int64_t g_opt_deterministic = 0;
 
 namespace {
 
@@ -585,6 +586,9 @@ int sata_set_option(int key, int64_t value) {
         case SATA_OPT_TIME_KERNELS:
             g_opt_time_kernels = value ? 1 : 0;
             return SATA_OK;
+        case SATA_OPT_DETERMINISTIC:
+            g_opt_deterministic = value ? 1 : 0;
+            return SATA_OK;
         default: return SATA_EINVAL;
     }
 }
@@ -596,6 +600,7 @@ int sata_get_option(int key, int64_t *value) {
         case SATA_OPT_WAIT_LIMIT: *value = g_opt_wait_limit; return SATA_OK;
         case SATA_OPT_TEST_STALL: *value = g_opt_test_stall; return SATA_OK;
         case SATA_OPT_TIME_KERNELS: *value = g_opt_time_kernels; return SATA_OK;
+        case SATA_OPT_DETERMINISTIC: *value = g_opt_deterministic; return SATA_OK;
         default: return SATA_EINVAL;
     }
 }

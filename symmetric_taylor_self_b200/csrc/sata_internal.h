@@ -80,6 +80,7 @@ extern int64_t g_opt_prefill_path;
 extern int64_t g_opt_wait_limit;
 extern int64_t g_opt_test_stall;
 extern int64_t g_opt_time_kernels;
+extern int64_t g_opt_deterministic;
 
 // ---- decode (decode.cu) ----
 size_t decode_workspace_bytes(int BH, int64_t F, int d_V);

@@ -205,12 +205,36 @@ def test_state_output_and_continuation(sata, oracle_mod, path):
 
 @pytest.mark.parametrize("path", list(PATHS))
 def test_deterministic(sata, path):
+    """With SATA_OPT_DETERMINISTIC = 1 every path is bitwise reproducible."""
     _set_path(sata, path)
-    q, k, v = wl.random_inputs(1, 4, 333, 32, 32, seed=5)
-    qc, kc, vc = q.cuda(), k.cuda(), v.cuda()
-    a = sata.prefill(qc, kc, vc, P=4)
-    b = sata.prefill(qc, kc, vc, P=4)
-    assert torch.equal(a, b)
+    sata.sata_set_option(sata.SATA_OPT_DETERMINISTIC, 1)
+    try:
+        q, k, v = wl.random_inputs(1, 4, 333, 32, 32, seed=5)
+        qc, kc, vc = q.cuda(), k.cuda(), v.cuda()
+        a = sata.prefill(qc, kc, vc, P=4)
+        b = sata.prefill(qc, kc, vc, P=4)
+        assert torch.equal(a, b)
+    finally:
+        sata.sata_set_option(sata.SATA_OPT_DETERMINISTIC, 0)
+
+
+@pytest.mark.parametrize("d", [16, 32, 64])
+def test_atomic_partials_match_fixed_order(sata, d):
+    """The default tensor-core prefill (partial sums added in L2) agrees with
+    the fixed-order reduction to fp32 rounding, and runs no tc_reduce."""
+    _set_path(sata, "auto")
+    q, k, v = (x.cuda() for x in wl.random_inputs(1, 3, 700, d, d, seed=77 + d))
+    sata.sata_set_option(sata.SATA_OPT_DETERMINISTIC, 1)
+    try:
+        ref = sata.prefill(q, k, v, P=4)
+    finally:
+        sata.sata_set_option(sata.SATA_OPT_DETERMINISTIC, 0)
+    sata.sata_reset_kernel_stats()
+    y = sata.prefill(q, k, v, P=4)
+    torch.cuda.synchronize()
+    stats = sata.sata_kernel_stats()
+    assert "tc_scan" in stats and "tc_reduce" not in stats
+    assert (y - ref).abs().max().item() <= 1e-5 * ref.abs().max().item()
 
 
 def test_empty_inputs_are_noops(sata):
@@ -326,7 +350,8 @@ def test_bounded_wait_reports_timeout(sata):
     a = sata.prefill(qc, kc, vc, P=4)
     assert sata.sata_sync_status() == 0
     b = sata.prefill(qc, kc, vc, P=4)
-    assert torch.equal(a, b)
+    # equal up to the order of the L2 partial-sum additions (SATA_OPT_DETERMINISTIC = 0)
+    assert (a - b).abs().max().item() <= 1e-6 * a.abs().max().item()
     sata.sata_set_option(sata.SATA_OPT_PREFILL_PATH, 0)
 
 
