@@ -56,6 +56,10 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--path", choices=["auto", "cuda_core", "tensor_core"], default="auto")
+    ap.add_argument("--seq-split", action="store_true",
+                    help="split each sequence across the ranks (segment states, all-gather, prefix, "
+                         "prefill from the prefix): strong scaling of one prefill; the default shards "
+                         "heads (weak scaling, no collective)")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     return ap.parse_args()
 
@@ -312,6 +316,8 @@ def main():
     rank, world, local = dist_setup(torch)
     if args.only != "all":
         return run_part(torch, sata, wl, args, world)
+    if args.seq_split:
+        return run_seq_split(torch, sata, wl, args, rank, world)
     dev = torch.device("cuda", torch.cuda.current_device())
     sata.load()
     sata.sata_set_option(sata.SATA_OPT_PREFILL_PATH, {"auto": 0, "cuda_core": 1, "tensor_core": 2}[args.path])
@@ -425,6 +431,50 @@ def main():
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_oracle_rate(w, args.cpu_seconds)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
+def run_seq_split(torch, sata, wl, args, rank, world):
+    """One prefill of the workload's sequences split by token ranges across the
+    ranks (seqsplit.py): strong scaling, one JSON line from rank 0."""
+    from symmetric_taylor_self_b200 import seqsplit
+    dev = torch.device("cuda", torch.cuda.current_device())
+    sata.load()
+    w = wl.WORKLOADS[args.workload]
+    n = -(-w.N // world)
+    a, b = min(rank * n, w.N), min((rank + 1) * n, w.N)
+    (q, k, v), _ = wl.make_inputs(w)
+    qd, kd, vd = (x[:, :, a:b].contiguous().to(dev) for x in (q, k, v))
+    stream = torch.cuda.Stream()
+
+    def step():
+        with torch.cuda.stream(stream):
+            seqsplit.prefill_sequence_split(qd, kd, vd, w.P)
+
+    step()
+    torch.cuda.synchronize()
+    sampler = ClockSampler(gpu_uuid(torch, dev))
+    sampler.start()
+    ms = timed(torch, world, step, args.steps, args.warmup, stream)
+    clocks = sampler.stop()
+    if sata.sata_sync_status(stream) != 0:
+        raise RuntimeError("device status after the split prefill")
+    value = w.B * w.N * args.steps / (ms / 1000.0)
+    line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True,
+            "scaling": "strong", "vs_baseline": None, "dtype": "f16", "accumulate": "f32",
+            "data": "synthetic (seeded N(0,1) bf16 inputs; no dataset involved)",
+            "config": {"workload": f"{w.name}: B={w.B} H={w.H} N={w.N} d_K={w.d_K} d_V={w.d_V} P={w.P}",
+                       "parallelism": f"sequence split over {world} ranks: {n} tokens per rank, segment "
+                                      f"states all-gathered, exclusive prefix, prefill from the prefix",
+                       "l2": "inputs and state exchange larger than L2 at this size"},
+            "roofline": None, "e2e": None, "clocks": clocks,
+            "note": "two prefills of each rank's segment plus the state all-gather; see DESIGN"}
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:

@@ -133,6 +133,21 @@ SATA_API int sata_state_bytes(int B, int H, int d_K, int d_V, int P, size_t *S_b
 SATA_API int sata_state_init(sata_state *st, int B, int H, int d_K, int d_V, int P,
                     float *S, float *Z, void *stream);
 
+/*
+ * Absorb another token segment's state into st: st->S += S, st->Z += Z
+ * (elementwise), st->tokens += tokens, on st->stream.  S and Z are device
+ * buffers of st's shape ([B][H][F][d_V] and [B][H][F] fp32), e.g. the state a
+ * prefill of the segment left in a fresh sata_state.  The states are sums over
+ * tokens, so the state after a concatenation of segments is the sum of the
+ * segments' states ([CC-TAYLOR] "Feature maps and linear attention": the
+ * recurrence may be evaluated as a parallel prefix scan).  This is the
+ * combining step of a prefill split by sequence across GPUs: after an
+ * all-gather of the segment states, each rank adds those of the segments
+ * before its own, then prefills its segment from the sum.
+ * Errors: SATA_EINVAL (null, negative tokens, st inconsistent), SATA_EALIGN.
+ */
+SATA_API int sata_state_accumulate(sata_state *st, const float *S, const float *Z, int64_t tokens);
+
 /* Workspace bytes sata_prefill_ex needs for this shape. */
 SATA_API int sata_workspace_bytes(int B, int H, int64_t N, int d_K, int d_V, int P, size_t *bytes);
 

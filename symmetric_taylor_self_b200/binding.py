@@ -37,7 +37,7 @@ EXPORTED = (
     "sata_state_bytes", "sata_state_init", "sata_workspace_bytes", "sata_prefill",
     "sata_prefill_ex", "sata_decode_step", "sata_set_option", "sata_get_option",
     "sata_kernel_stats", "sata_reset_kernel_stats", "sata_decode_step_static", "sata_prefill_host",
-    "sata_backward_workspace_bytes", "sata_prefill_backward",
+    "sata_backward_workspace_bytes", "sata_prefill_backward", "sata_state_accumulate",
 )
 
 
@@ -99,6 +99,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "sata_decode_step_static": (i32, [st_p, vp, vp, vp, vp]),
         "sata_prefill_host": (i32, [vp, vp, vp, vp, i32, i32, i64, i32, i32, i32, st_p, vp]),
         "sata_backward_workspace_bytes": (i32, [i32, i32, i64, i32, i32, i32, P_sz]),
+        "sata_state_accumulate": (i32, [st_p, vp, vp, i64]),
         "sata_prefill_backward": (i32, [vp, vp, vp, vp, vp, vp, vp, i32, i32, i64, i32, i32, i32,
                                         vp, sz, vp]),
     }
@@ -252,6 +253,10 @@ def sata_prefill_backward(q, k, v, dy, dq, dk, dv, B, H, N, d_K, d_V, P, workspa
 def sata_state_init(st, B, H, d_K, d_V, P, S, Z, stream=None):
     _check(load().sata_state_init(ctypes.byref(st), B, H, d_K, d_V, P, _ptr(S), _ptr(Z),
                                   _stream(stream)), "sata_state_init")
+
+
+def sata_state_accumulate(st, S, Z, tokens):
+    _check(load().sata_state_accumulate(ctypes.byref(st), _ptr(S), _ptr(Z), tokens), "sata_state_accumulate")
 
 
 def sata_decode_step(st, q, k, v, out):

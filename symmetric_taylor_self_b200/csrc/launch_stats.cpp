@@ -27,7 +27,7 @@ thread_local cudaEvent_t t_start[kNumKernels] = {};
 const char *const kNames[kNumKernels] = {
     "decode_stream", "decode_finish", "simt_scan", "simt_finish",
     "tc_prep", "tc_scan", "tc_finish", "tc_reduce",
-    "bwd_r", "bwd_q_scan", "bwd_kv_scan", "bwd_finish",
+    "bwd_r", "bwd_q_scan", "bwd_kv_scan", "bwd_finish", "state_add",
 };
 
 void drain_locked() {

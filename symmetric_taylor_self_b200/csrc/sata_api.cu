@@ -384,6 +384,25 @@ int sata_state_init(sata_state *st, int B, int H, int d_K, int d_V, int P, float
     return e == cudaSuccess ? SATA_OK : cuda_fail(e);
 }
 
+int sata_state_accumulate(sata_state *st, const float *S, const float *Z, int64_t tokens) {
+    if (!st || tokens < 0) return SATA_EINVAL;
+    size_t sb = 0, zb = 0;
+    int rc = sata_state_bytes(st->B, st->H, st->d_K, st->d_V, st->P, &sb, &zb);
+    if (rc) return rc;
+    if (st->F != num_features(st->d_K, st->P)) return SATA_EINVAL;
+    if (sb + zb == 0) {
+        st->tokens += tokens;
+        return SATA_OK;
+    }
+    if (!st->S || !st->Z || !S || !Z) return SATA_EINVAL;
+    if (!aligned16(st->S) || !aligned16(st->Z) || !aligned16(S) || !aligned16(Z)) return SATA_EALIGN;
+    const cudaError_t e = launch_state_add(st->S, st->Z, S, Z, (int64_t)(sb / sizeof(float)),
+                                           (int64_t)(zb / sizeof(float)), (cudaStream_t)st->stream);
+    if (e != cudaSuccess) return cuda_fail(e);
+    st->tokens += tokens;
+    return SATA_OK;
+}
+
 int sata_workspace_bytes(int B, int H, int64_t N, int d_K, int d_V, int P, size_t *bytes) {
     if (!bytes || N < 0) return SATA_EINVAL;
     int BH = 0;

@@ -67,7 +67,7 @@ const void *device_table(uint64_t key, size_t bytes, const std::function<void(ui
 // Kernel identities for launch statistics.
 enum KernelId {
     kDecodeStream = 0, kDecodeFinish, kSimtScan, kSimtFinish, kTcPrep, kTcScan, kTcFinish, kTcReduce,
-    kBwdR, kBwdQScan, kBwdKVScan, kBwdFinish, kNumKernels
+    kBwdR, kBwdQScan, kBwdKVScan, kBwdFinish, kStateAdd, kNumKernels
 };
 const char *kernel_name(int id);
 // Call around every kernel launch: begin() records a start event when timing is
@@ -94,6 +94,11 @@ cudaError_t launch_prefill_simt(const DeviceBasis &basis, int BH, int64_t N, int
                                 const void *q, const void *k, const void *v, float *out,
                                 float *S, float *Z, bool state_in, void *ws, size_t ws_bytes,
                                 cudaStream_t stream, float *den_out = nullptr);
+
+// ---- state operations (state_ops.cu) ----
+// S += dS (nS floats), Z += dZ (nZ floats), on `stream`.
+cudaError_t launch_state_add(float *S, float *Z, const float *dS, const float *dZ, int64_t nS, int64_t nZ,
+                             cudaStream_t stream);
 
 // ---- backward of the prefill, CUDA-core path (backward_simt.cu) ----
 size_t prefill_backward_workspace_bytes(int BH, int64_t N, int64_t F, int d_K, int d_V);

@@ -137,6 +137,14 @@ def test_argument_validation_needs_no_gpu(lib):
     assert bw(fake, fake, fake, fake, fake, fake, fake, 1, -1, 8, 8, 8, 4) == bd.SATA_EINVAL
     assert bw(fake, fake, fake, fake, fake, vp(0x10004), fake, 1, 1, 8, 8, 8, 4) == bd.SATA_EALIGN
     assert bw(None, None, None, None, None, None, None, 1, 1, 0, 8, 8, 4) == bd.SATA_OK
+    # state accumulation
+    st = bd.sata_state(B=1, H=1, d_K=8, d_V=8, P=4, F=165, S=0x10000, Z=0x10000, stream=None, tokens=0)
+    assert lib.sata_state_accumulate(None, fake, fake, 1) == bd.SATA_EINVAL
+    assert lib.sata_state_accumulate(ctypes.byref(st), None, fake, 1) == bd.SATA_EINVAL
+    assert lib.sata_state_accumulate(ctypes.byref(st), fake, fake, -1) == bd.SATA_EINVAL
+    assert lib.sata_state_accumulate(ctypes.byref(st), vp(0x10008), fake, 1) == bd.SATA_EALIGN
+    st.F = 999
+    assert lib.sata_state_accumulate(ctypes.byref(st), fake, fake, 1) == bd.SATA_EINVAL
     # decode
     assert lib.sata_decode_step(None, fake, fake, fake, fake) == bd.SATA_EINVAL
     st = bd.sata_state(B=1, H=1, d_K=8, d_V=8, P=4, F=999, S=0x10000, Z=0x10000, stream=None, tokens=0)

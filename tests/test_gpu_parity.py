@@ -452,3 +452,42 @@ def test_backward_workload_full_size(sata, oracle_mod, name):
         for nm, g, r in (("dq", dq, rq), ("dk", dk, rk), ("dv", dv, rv)):
             err = tensor_rel_err(g[b, h].double().cpu().numpy(), r)
             assert err <= TOL, f"{name} {nm} head {(b, h)}: {err:.3e}"
+
+
+# ------------------------------------------------ sequence split (row f4) ----
+
+@pytest.mark.parametrize("d,lens", [(32, (300, 212)), (64, (128, 257, 100)), (16, (64, 64, 64, 65))])
+def test_sequence_split_emulated_ranks(sata, oracle_mod, d, lens):
+    """The product steps of the sequence split on one GPU, its ranks run one
+    after another in this process (no kernel waits on another rank): segment
+    states, the exclusive prefix in rank order (sata_state_accumulate), then
+    each segment's prefill from its prefix.  The concatenated outputs match the
+    oracle over the whole sequence and one prefill on one GPU; the last rank's
+    state matches the whole sequence's state."""
+    from symmetric_taylor_self_b200 import seqsplit
+    _set_path(sata, "auto")
+    N = sum(lens)
+    q, k, v = wl.random_inputs(1, 2, N, d, d, seed=900 + d)
+    qc, kc, vc = q.cuda(), k.cuda(), v.cuda()
+    bounds = np.cumsum((0,) + lens)
+    segs = [(qc[:, :, a:b].contiguous(), kc[:, :, a:b].contiguous(), vc[:, :, a:b].contiguous())
+            for a, b in zip(bounds[:-1], bounds[1:])]
+    impl = seqsplit.LibraryImpl()
+    gathered = [impl.tensors(impl.segment_state(*sg, 4)) for sg in segs]
+    ys, st = [], None
+    for r, sg in enumerate(segs):
+        st = seqsplit.exclusive_prefix(impl, (1, 2, d, d, 4), gathered, r, list(lens), qc.device)
+        assert st.tokens == bounds[r]
+        ys.append(impl.prefill(*sg, 4, st))
+    y = torch.cat(ys, dim=2)
+    torch.cuda.synchronize()
+    assert sata.sata_sync_status() == 0
+    ref = _oracle_heads(oracle_mod, q, k, v, 4, [(0, 0), (0, 1)])
+    _check_heads(y, ref, what=f"split d={d} {lens}")
+    whole = sata.State(1, 2, d, d, 4)
+    y1 = sata.prefill(qc, kc, vc, P=4, state=whole)
+    torch.cuda.synchronize()
+    assert (y - y1).abs().max().item() <= 1e-3 * y1.abs().max().item()
+    assert st.tokens == N
+    for got, want in ((st.S, whole.S), (st.Z, whole.Z)):
+        assert (got - want).abs().max().item() <= 1e-4 * want.abs().max().item()

@@ -1,8 +1,9 @@
-"""The multi-rank host logic of bench.py on CPU: two gloo ranks on 127.0.0.1.
+"""Multi-rank host logic on CPU: gloo ranks on 127.0.0.1.
 
-On GPUs every rank runs its own copy of the workload (heads are independent,
-no collective on the data path); the only cross-rank steps are the barrier and
-the max-over-ranks time, which these tests exercise without a GPU.
+bench.py: on GPUs every rank runs its own copy of the workload (heads are
+independent, no collective on the data path); the only cross-rank steps are
+the barrier and the max-over-ranks time.  The sequence split (seqsplit.py)
+has one real exchange, the all-gather of segment states and their prefix sum.
 """
 import os
 import socket
@@ -77,3 +78,107 @@ def test_job_throughput_single_rank():
     import bench
 
     assert bench.job_throughput(1000, 4, 1, 2000.0) == pytest.approx(2000.0)
+
+
+# ------------------------------------------------ sequence split (row f4) ----
+# The exchange logic of symmetric_taylor_self_b200.seqsplit on gloo CPU ranks:
+# the per-rank steps run on the float64 oracle (a reference implementation of
+# the same four methods), the all-gather and the prefix order are the product
+# code's.
+
+class _OracleImpl:
+    """Per-rank steps on the oracle: states are float64 CPU tensors."""
+
+    def zero_state(self, B, H, d_K, d_V, P, device):
+        import math
+        F = math.comb(d_K + P - 1, P - 1)
+        return {"S": torch.zeros(B, H, F, d_V, dtype=torch.float64),
+                "Z": torch.zeros(B, H, F, dtype=torch.float64), "tokens": 0}
+
+    def _run(self, q, k, v, P, st):
+        import oracle
+        B, H, n, _ = q.shape
+        y = torch.zeros(B, H, n, v.shape[-1], dtype=torch.float64)
+        for b in range(B):
+            for h in range(H):
+                yy, _, S, Z = oracle.scan(q[b, h], k[b, h], v[b, h], P, S=st["S"][b, h].numpy(),
+                                          Z=st["Z"][b, h].numpy())
+                y[b, h] = torch.from_numpy(yy)
+                st["S"][b, h] = torch.from_numpy(S)
+                st["Z"][b, h] = torch.from_numpy(Z)
+        st["tokens"] += n
+        return y
+
+    def segment_state(self, q, k, v, P):
+        st = self.zero_state(q.shape[0], q.shape[1], q.shape[-1], v.shape[-1], P, None)
+        self._run(q, k, v, P, st)
+        return st
+
+    def accumulate(self, st, S, Z, tokens):
+        st["S"] += S
+        st["Z"] += Z
+        st["tokens"] += tokens
+
+    def prefill(self, q, k, v, P, st):
+        return self._run(q, k, v, P, st)
+
+    @staticmethod
+    def tensors(st):
+        return st["S"], st["Z"]
+
+
+def _split_worker(rank, world, port, lens, q):
+    sys.path.insert(0, ROOT)
+    import datetime
+
+    import torch.distributed as dist
+
+    from symmetric_taylor_self_b200 import seqsplit
+    from symmetric_taylor_self_b200 import workloads as wl
+
+    dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    try:
+        qa, ka, va = wl.random_inputs(1, 2, sum(lens), 4, 3, seed=77)
+        t0 = sum(lens[:rank])
+        sl = slice(t0, t0 + lens[rank])
+        y, st = seqsplit.prefill_sequence_split(qa[:, :, sl], ka[:, :, sl], va[:, :, sl], P=3,
+                                                impl=_OracleImpl())
+        q.put((rank, y.numpy(), st["S"].numpy(), st["Z"].numpy(), st["tokens"]))
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("lens", [(40, 40), (23, 50, 31)])
+def test_sequence_split_exchange_gloo(lens):
+    """G ranks, each with one segment (lengths may differ): the concatenated
+    outputs and the last rank's state equal one prefill of the whole sequence."""
+    import numpy as np
+
+    sys.path.insert(0, ROOT)
+    import oracle
+    from symmetric_taylor_self_b200 import workloads as wl
+
+    world = len(lens)
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_split_worker, args=(r, world, port, lens, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    got = {}
+    for _ in range(world):
+        r, y, S, Z, tokens = q.get(timeout=120)
+        got[r] = (y, S, Z, tokens)
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    qa, ka, va = wl.random_inputs(1, 2, sum(lens), 4, 3, seed=77)
+    y_all = np.concatenate([got[r][0] for r in range(world)], axis=2)
+    for h in range(2):
+        yr, _, Sr, Zr = oracle.scan(qa[0, h], ka[0, h], va[0, h], 3)
+        np.testing.assert_allclose(y_all[0, h], yr, rtol=1e-10, atol=1e-12)
+        _, S_last, Z_last, tokens = got[world - 1]
+        np.testing.assert_allclose(S_last[0, h], Sr, rtol=1e-10, atol=1e-12)
+        np.testing.assert_allclose(Z_last[0, h], Zr, rtol=1e-10, atol=1e-12)
+        assert tokens == sum(lens)
