@@ -568,7 +568,7 @@ def bench_backward(torch, sata, wl, args, world, dev, stream, clocks):
     return {"metric": "SATA prefill backward tokens/s (dq, dk, dv)", "value": value, "unit": "tokens/s",
             "steps": args.steps, "ms_per_step": ms / args.steps,
             "workload": f"{w.name}: B={w.B} H={w.H} N={w.N} d_K={w.d_K} d_V={w.d_V} P={w.P} F={w.F}; "
-                        f"dy N(0,1) fp32; the step recomputes the forward (CUDA-core, fp32)",
+                        f"dy N(0,1) fp32; the step recomputes the forward on the prefill's path",
             "l2": "each step writes more than 1 GB of partial sums, far above the 126 MB L2",
             "roofline": roof, "gpu_launches": sum(n for n, _ in stats.values()),
             "kernel_ms": {k_: {"launches": n, "ms": t} for k_, (n, t) in stats.items()}}

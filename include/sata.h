@@ -210,14 +210,18 @@ SATA_API int sata_prefill_host(const void *q, const void *k, const void *v, floa
  * (fixed cost per token): the forward is recomputed, then one pass forward
  * over the sequence with S gives dq and one pass backward with
  * G = sum_t phi(q_t) [dy_t / den_t | -(dy_t . y_t) / den_t]^T gives dk and dv.
- * Runs on CUDA cores in fp32 for every supported shape.
+ * The recomputed forward takes the prefill's path (tensor cores where
+ * sata_prefill_ex would use them, keeping den); the two gradient scans run on
+ * CUDA cores in fp32 for every supported shape.
  *   q, k: bf16 [B][H][N][d_K];  v: bf16 [B][H][N][d_V]  (the forward's inputs)
  *   dy:   fp32 [B][H][N][d_V]
  *   dq, dk: fp32 [B][H][N][d_K];  dv: fp32 [B][H][N][d_V]  (overwritten)
  *   workspace: NULL (library-owned) or a device buffer of ws_bytes >=
  *              sata_backward_workspace_bytes(...).
  *   stream: cudaStream_t (NULL: legacy stream).
- * The result is deterministic (partial sums are added in a fixed order).
+ * The gradient scans add their partial sums in a fixed order; the result is
+ * bitwise reproducible when the forward is (SATA_OPT_DETERMINISTIC = 1, or the
+ * CUDA-core path).
  * N = 0 is a no-op.  Errors as sata_prefill_ex.
  */
 SATA_API int sata_backward_workspace_bytes(int B, int H, int64_t N, int d_K, int d_V, int P, size_t *bytes);

@@ -533,11 +533,12 @@ struct BwdLayout {
     size_t fwd = 0, part = 0, off_state = 0, off_y = 0, off_den = 0, off_r = 0, total = 0;
 };
 
-BwdLayout bwd_layout(int BH, int64_t N, int64_t F, int d_K, int d_V) {
+BwdLayout bwd_layout(int BH, int64_t N, int64_t F, int d_K, int d_V, int P, bool use_tc) {
     BwdLayout L;
     const int64_t ntiles = (F + kTF - 1) / kTF;
     L.Tseg = segment_tokens(BH, N, F, d_K, d_V);
-    L.fwd = prefill_simt_workspace_bytes(BH, N, F, d_V, true);
+    L.fwd = use_tc ? prefill_tc_workspace_bytes(BH, N, F, d_K, d_V, P, true, false)
+                   : prefill_simt_workspace_bytes(BH, N, F, d_V, true);
     L.part = round256((size_t)ntiles * BH * L.Tseg * (d_K + d_V) * sizeof(float));
     const size_t front = L.fwd > L.part ? L.fwd : L.part;   // the forward's workspace, then the partials
     L.off_state = round256(front);
@@ -567,17 +568,17 @@ bool scan_kernels(int d_V, ScanFn *fq, ScanFn *fkv) {
 
 }  // namespace
 
-size_t prefill_backward_workspace_bytes(int BH, int64_t N, int64_t F, int d_K, int d_V) {
-    return bwd_layout(BH, N, F, d_K, d_V).total;
+size_t prefill_backward_workspace_bytes(int BH, int64_t N, int64_t F, int d_K, int d_V, int P, bool use_tc) {
+    return bwd_layout(BH, N, F, d_K, d_V, P, use_tc).total;
 }
 
 cudaError_t launch_prefill_backward(const DeviceBasis &basis, int BH, int64_t N, int d_V,
                                     const void *q, const void *k, const void *v, const float *dy,
                                     float *dq, float *dk, float *dv, void *ws, size_t ws_bytes,
-                                    cudaStream_t stream) {
+                                    bool use_tc, int *flags, cudaStream_t stream) {
     const int d_K = basis.d_K, P = basis.P;
     const int64_t F = basis.F;
-    const BwdLayout L = bwd_layout(BH, N, F, d_K, d_V);
+    const BwdLayout L = bwd_layout(BH, N, F, d_K, d_V, P, use_tc);
     if (ws_bytes < L.total) return cudaErrorInvalidValue;
     const int ntiles = (int)((F + kTF - 1) / kTF);
     const int ncomp = P > 2 ? P - 2 : 0;
@@ -600,8 +601,12 @@ cudaError_t launch_prefill_backward(const DeviceBasis &basis, int BH, int64_t N,
     const __nv_bfloat16 *qb = (const __nv_bfloat16 *)q, *kb = (const __nv_bfloat16 *)k,
                         *vb = (const __nv_bfloat16 *)v;
 
-    // forward: y and den (fresh state, carried in the front region)
-    e = launch_prefill_simt(basis, BH, N, d_V, q, k, v, y, nullptr, nullptr, false, ws, L.fwd, stream, den);
+    // forward: y and den (fresh state, carried in the front region), on tensor cores where the
+    // prefill runs there
+    e = use_tc ? launch_prefill_tc(basis, BH, N, d_V, q, k, v, y, nullptr, nullptr, false, ws, L.fwd, flags,
+                                   stream, nullptr, den)
+               : launch_prefill_simt(basis, BH, N, d_V, q, k, v, y, nullptr, nullptr, false, ws, L.fwd, stream,
+                                     den);
     if (e != cudaSuccess) return e;
     const int64_t rows = (int64_t)BH * N;
     launch_begin(kBwdR, stream);

@@ -867,7 +867,8 @@ template <int DK, int DV>
 __global__ void __launch_bounds__(128)
 tc_finish_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k,
                  const __nv_bfloat16 *__restrict__ v, const float *__restrict__ red, float *__restrict__ out,
-                 int c0, int nc, int64_t N, int P, float inv_c, int *flags, int64_t wait_ns) {
+                 float *__restrict__ den_out, int c0, int nc, int64_t N, int P, float inv_c, int *flags,
+                 int64_t wait_ns) {
     using F = FinCfg<DK, DV>;
     constexpr int NV = F::NV;
     extern __shared__ uint8_t fraw[];
@@ -1025,7 +1026,9 @@ tc_finish_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__res
             uint32_t rr[16];
             tc_ld16(tmem + 128 + lane_off + DV, rr);
             tc_wait_ld();
-            inv = 1.f / fmaf(__uint_as_float(rr[0]), up, rp[DV * kL]);
+            const float den = fmaf(__uint_as_float(rr[0]), up, rp[DV * kL]);
+            inv = 1.f / den;
+            if (den_out && t < nt) den_out[bh * N + t0 + t] = den;   // kept for the backward pass
         }
 #pragma unroll
         for (int c16 = 0; c16 < DV / 16; ++c16) {
@@ -1224,7 +1227,7 @@ cudaError_t copy_rows(void *dst, const void *src, int BH, int64_t N, int64_t t0,
 template <int DK, int DV>
 cudaError_t run(const DeviceBasis &basis, int BH, int64_t N, const void *q, const void *k, const void *v,
                 float *out, float *S, float *Z, bool state_in, void *ws, size_t ws_bytes, int *flags,
-                cudaStream_t stream, const HostIO *io) {
+                cudaStream_t stream, const HostIO *io, float *den_out) {
     using C = Cfg<DK, DV>;
     const int64_t F = basis.F;
     const bool own_state = (S == nullptr);
@@ -1359,7 +1362,7 @@ cudaError_t run(const DeviceBasis &basis, int BH, int64_t N, const void *q, cons
         }
         launch_begin(kTcFinish, stream);
         tc_finish_kernel<DK, DV><<<(int)((int64_t)BH * sp.nc), 128, FinCfg<DK, DV>::SMEM, stream>>>(
-            qb, kb, vb, red, out, sp.c0, sp.nc, N, basis.P, inv_c, flags, wait_ns);
+            qb, kb, vb, red, out, den_out, sp.c0, sp.nc, N, basis.P, inv_c, flags, wait_ns);
         launch_end(kTcFinish, stream);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
         if (io) {   // this segment's output: device -> host on the second copy stream
@@ -1399,11 +1402,15 @@ size_t prefill_tc_workspace_bytes(int BH, int64_t N, int64_t F, int d_K, int d_V
 
 cudaError_t launch_prefill_tc(const DeviceBasis &basis, int BH, int64_t N, int d_V, const void *q,
                               const void *k, const void *v, float *out, float *S, float *Z, bool state_in,
-                              void *ws, size_t ws_bytes, int *flags, cudaStream_t stream, const HostIO *io) {
+                              void *ws, size_t ws_bytes, int *flags, cudaStream_t stream, const HostIO *io,
+                              float *den_out) {
     switch (basis.d_K * 1000 + d_V) {
-        case 16016: return run<16, 16>(basis, BH, N, q, k, v, out, S, Z, state_in, ws, ws_bytes, flags, stream, io);
-        case 32032: return run<32, 32>(basis, BH, N, q, k, v, out, S, Z, state_in, ws, ws_bytes, flags, stream, io);
-        case 64064: return run<64, 64>(basis, BH, N, q, k, v, out, S, Z, state_in, ws, ws_bytes, flags, stream, io);
+        case 16016:
+            return run<16, 16>(basis, BH, N, q, k, v, out, S, Z, state_in, ws, ws_bytes, flags, stream, io, den_out);
+        case 32032:
+            return run<32, 32>(basis, BH, N, q, k, v, out, S, Z, state_in, ws, ws_bytes, flags, stream, io, den_out);
+        case 64064:
+            return run<64, 64>(basis, BH, N, q, k, v, out, S, Z, state_in, ws, ws_bytes, flags, stream, io, den_out);
         default: return cudaErrorNotSupported;
     }
 }

@@ -423,7 +423,9 @@ int sata_backward_workspace_bytes(int B, int H, int64_t N, int d_K, int d_V, int
     if (rc) return rc;
     rc = check_shape(d_K, d_V, P);
     if (rc) return rc;
-    *bytes = prefill_backward_workspace_bytes(BH, N, num_features(d_K, P), d_K, d_V);
+    bool use_tc = false;
+    prefill_ws_bytes(BH, N, d_K, d_V, P, true, &use_tc);
+    *bytes = prefill_backward_workspace_bytes(BH, N, num_features(d_K, P), d_K, d_V, P, use_tc);
     return SATA_OK;
 }
 
@@ -445,7 +447,12 @@ int sata_prefill_backward(const void *q, const void *k, const void *v, const flo
     cudaError_t e = cudaSuccess;
     const DeviceBasis *basis = device_basis(d_K, P, &e);
     if (!basis) return cuda_fail(e);
-    const size_t need = prefill_backward_workspace_bytes(BH, N, basis->F, d_K, d_V);
+    int *flags = device_flags(&e);
+    if (!flags) return cuda_fail(e);
+    bool use_tc = false;   // the forward it recomputes takes the prefill's path
+    prefill_ws_bytes(BH, N, d_K, d_V, P, true, &use_tc);
+    if (g_opt_prefill_path == 2 && !use_tc) return SATA_EUNSUPPORTED;
+    const size_t need = prefill_backward_workspace_bytes(BH, N, basis->F, d_K, d_V, P, use_tc);
     if (workspace) {
         if (ws_bytes < need) return SATA_ENOMEM;
     } else {
@@ -456,8 +463,8 @@ int sata_prefill_backward(const void *q, const void *k, const void *v, const flo
         }
         ws_bytes = need;
     }
-    e = launch_prefill_backward(*basis, BH, N, d_V, q, k, v, dy, dq, dk, dv, workspace, ws_bytes,
-                                (cudaStream_t)stream);
+    e = launch_prefill_backward(*basis, BH, N, d_V, q, k, v, dy, dq, dk, dv, workspace, ws_bytes, use_tc,
+                                flags, (cudaStream_t)stream);
     if (e != cudaSuccess) return cuda_fail(e);
     return SATA_OK;
 }

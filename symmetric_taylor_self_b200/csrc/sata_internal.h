@@ -101,11 +101,12 @@ cudaError_t launch_state_add(float *S, float *Z, const float *dS, const float *d
                              cudaStream_t stream);
 
 // ---- backward of the prefill, CUDA-core path (backward_simt.cu) ----
-size_t prefill_backward_workspace_bytes(int BH, int64_t N, int64_t F, int d_K, int d_V);
+size_t prefill_backward_workspace_bytes(int BH, int64_t N, int64_t F, int d_K, int d_V, int P, bool use_tc);
+// The forward it recomputes runs on tensor cores when use_tc (flags: the device status words).
 cudaError_t launch_prefill_backward(const DeviceBasis &basis, int BH, int64_t N, int d_V,
                                     const void *q, const void *k, const void *v, const float *dy,
                                     float *dq, float *dk, float *dv, void *ws, size_t ws_bytes,
-                                    cudaStream_t stream);
+                                    bool use_tc, int *flags, cudaStream_t stream);
 
 // ---- prefill, tensor-core path (prefill_tc.cu) ----
 // Host-buffer prefill: the kernels read and write the device copies passed as q, k, v, out;
@@ -123,7 +124,7 @@ size_t prefill_tc_workspace_bytes(int BH, int64_t N, int64_t F, int d_K, int d_V
 cudaError_t launch_prefill_tc(const DeviceBasis &basis, int BH, int64_t N, int d_V,
                               const void *q, const void *k, const void *v, float *out,
                               float *S, float *Z, bool state_in, void *ws, size_t ws_bytes,
-                              int *flags, cudaStream_t stream, const HostIO *io);
+                              int *flags, cudaStream_t stream, const HostIO *io, float *den_out = nullptr);
 // Library-owned copy streams of the current device (non-blocking), created once.
 cudaError_t device_copy_streams(cudaStream_t *h2d, cudaStream_t *d2h);
 

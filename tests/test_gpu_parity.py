@@ -385,11 +385,16 @@ def _check_grads(sata, oracle_mod, B, H, N, d_K, d_V, P, seed, heads=None):
     return dq, dk, dv
 
 
+@pytest.mark.parametrize("path", list(PATHS))
 @pytest.mark.parametrize("d_K,d_V,P,N", [(16, 16, 4, 100), (8, 8, 4, 77), (32, 32, 4, 70),
                                          (64, 64, 4, 130), (16, 32, 3, 65), (12, 8, 2, 50),
                                          (8, 8, 5, 40), (4, 4, 1, 33), (128, 128, 2, 37)])
-def test_backward_matches_oracle(sata, oracle_mod, d_K, d_V, P, N):
+def test_backward_matches_oracle(sata, oracle_mod, path, d_K, d_V, P, N):
+    """auto: the recomputed forward runs on tensor cores for d_K = d_V in
+    {16, 32, 64}, P <= 4; cuda_core: always on CUDA cores."""
+    _set_path(sata, path)
     _check_grads(sata, oracle_mod, 1, 2, N, d_K, d_V, P, seed=5000 + d_K + P * 3 + N)
+    _set_path(sata, "auto")
 
 
 def test_backward_single_token(sata):
@@ -409,12 +414,20 @@ def test_backward_several_segments(sata, oracle_mod):
     _check_grads(sata, oracle_mod, 2, 4, 3000, 64, 64, 4, seed=5100, heads=[(0, 0), (1, 3)])
 
 
-def test_backward_is_deterministic_and_linear_in_dy(sata):
+@pytest.mark.parametrize("path", list(PATHS))
+def test_backward_is_deterministic_and_linear_in_dy(sata, path):
+    """Bitwise repeatable with SATA_OPT_DETERMINISTIC = 1 (the recomputed
+    forward may run on tensor cores), and linear in dy."""
+    _set_path(sata, path)
     q, k, v = (x.cuda() for x in wl.random_inputs(1, 2, 200, 16, 16, seed=5200))
     dy1 = wl.random_cotangent(1, 2, 200, 16, seed=5201).cuda()
     dy2 = wl.random_cotangent(1, 2, 200, 16, seed=5202).cuda()
-    a = sata.prefill_backward(q, k, v, dy1, 4)
-    b = sata.prefill_backward(q, k, v, dy1, 4)
+    sata.sata_set_option(sata.SATA_OPT_DETERMINISTIC, 1)
+    try:
+        a = sata.prefill_backward(q, k, v, dy1, 4)
+        b = sata.prefill_backward(q, k, v, dy1, 4)
+    finally:
+        sata.sata_set_option(sata.SATA_OPT_DETERMINISTIC, 0)
     for x, y in zip(a, b):
         assert torch.equal(x, y)
     c = sata.prefill_backward(q, k, v, dy2, 4)
