@@ -473,14 +473,9 @@ bwd_finish_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__re
             float x = 0.f;
             for (int i = 0; i < d_K; ++i) x = fmaf(xq[t * d_K + i], xk[s * d_K + i], x);
             x *= inv_c;
-            // Horner forms of T_P(x) = sum_{p<P} x^p / p! and of T_{P-1}(x)
-            float h = 1.f;
-            for (int p = P - 1; p >= 1; --p) h = fmaf(h, x / (float)p, 1.f);
-            float hd = 0.f;
-            if (P > 1) {
-                hd = 1.f;
-                for (int p = P - 2; p >= 1; --p) hd = fmaf(hd, x / (float)p, 1.f);
-            }
+            // T_P(x) = sum_{p<P} x^p / p! and its derivative T_{P-1}(x) (T_0 = 0)
+            const float h = simt::taylor_exp(x, P);
+            const float hd = simt::taylor_exp(x, P - 1);
             float dw = 0.f;
             for (int j = 0; j < DV1; ++j) dw = fmaf(xr[t * DV1 + j], xu[s * DV1 + j], dw);
             wd = dw * hd * inv_c;

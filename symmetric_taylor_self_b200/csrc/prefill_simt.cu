@@ -192,10 +192,7 @@ simt_finish_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
             float x = 0.f;
             for (int i = 0; i < d_K; ++i) x = fmaf(xq[t * d_K + i], xk[s * d_K + i], x);
             x *= inv_c;
-            // Horner form of sum_{p<P} x^p / p!
-            float h = 1.f;
-            for (int p = P - 1; p >= 1; --p) h = fmaf(h, x / (float)p, 1.f);
-            w = h;
+            w = simt::taylor_exp(x, P);   // sum_{p<P} x^p / p!
         }
         W[e] = w;
     }

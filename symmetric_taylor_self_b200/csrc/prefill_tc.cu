@@ -952,10 +952,13 @@ tc_finish_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__res
     const int t = tid;                               // token row = TMEM lane
     const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
     // ---- W row t: polynomial, causal mask, power-of-two scale into the fp16 range
+    // Horner form of sum_{p<P} x^p / p!, x = sv / c: h <- 1 + h * sv * (1 / (c p)), P <= 4
+    const float cp1 = inv_c, cp2 = inv_c * 0.5f, cp3 = inv_c * (1.f / 3.f);
     auto wval = [&](float sv, int s) -> float {
-        const float x = sv * inv_c;
-        float h = 1.f;   // Horner form of sum_{p<P} x^p / p!
-        for (int pp = P - 1; pp >= 1; --pp) h = fmaf(h, x / (float)pp, 1.f);
+        float h = 1.f;
+        if (P > 3) h = fmaf(h, sv * cp3, 1.f);
+        if (P > 2) h = fmaf(h, sv * cp2, 1.f);
+        if (P > 1) h = fmaf(h, sv * cp1, 1.f);
         return (s <= t && t < nt) ? h : 0.f;
     };
     float wmax = 0.f;

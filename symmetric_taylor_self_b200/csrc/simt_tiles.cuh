@@ -14,6 +14,16 @@ constexpr int kThreads = 256;
 constexpr int kTF = 128;   // features per CTA
 constexpr int kL = 32;     // chunk length
 
+// T_n(x) = sum_{p<n} x^p / p! (n <= 8) in Horner form, h <- 1 + h x / p; the
+// steps are unrolled so each 1/p is a compile-time constant (no division).
+__device__ __forceinline__ float taylor_exp(float x, int n) {
+    float h = n > 0 ? 1.f : 0.f;
+#pragma unroll
+    for (int p = 7; p >= 1; --p)
+        if (p < n) h = fmaf(h, x * (1.f / p), 1.f);
+    return h;
+}
+
 // Register-tiled contraction out[t][m] = coef[m] * sum_j X[m][j] * Y[t][j] over
 // the j < DV1 columns (X: a tile's state rows, Y: the chunk's r or u rows):
 // thread (warp, lane) owns t = warp + 8b (b < 4) and m = lane + 32a (a < 4).
