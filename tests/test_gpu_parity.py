@@ -388,7 +388,8 @@ def _check_grads(sata, oracle_mod, B, H, N, d_K, d_V, P, seed, heads=None):
 @pytest.mark.parametrize("path", list(PATHS))
 @pytest.mark.parametrize("d_K,d_V,P,N", [(16, 16, 4, 100), (8, 8, 4, 77), (32, 32, 4, 70),
                                          (64, 64, 4, 130), (16, 32, 3, 65), (12, 8, 2, 50),
-                                         (8, 8, 5, 40), (4, 4, 1, 33), (128, 128, 2, 37)])
+                                         (8, 8, 5, 40), (4, 4, 1, 33), (128, 128, 2, 37),
+                                         (6, 8, 7, 29), (32, 4, 4, 140)])
 def test_backward_matches_oracle(sata, oracle_mod, path, d_K, d_V, P, N):
     """auto: the recomputed forward runs on tensor cores for d_K = d_V in
     {16, 32, 64}, P <= 4; cuda_core: always on CUDA cores."""
@@ -469,8 +470,9 @@ def test_backward_workload_full_size(sata, oracle_mod, name):
 
 # ------------------------------------------------ sequence split (row f4) ----
 
-@pytest.mark.parametrize("d,lens", [(32, (300, 212)), (64, (128, 257, 100)), (16, (64, 64, 64, 65))])
-def test_sequence_split_emulated_ranks(sata, oracle_mod, d, lens):
+@pytest.mark.parametrize("d,lens,P", [(32, (300, 212), 4), (64, (128, 257, 100), 4), (16, (64, 64, 64, 65), 4),
+                                     (8, (50, 1, 77), 5)])
+def test_sequence_split_emulated_ranks(sata, oracle_mod, d, lens, P):
     """The product steps of the sequence split on one GPU, its ranks run one
     after another in this process (no kernel waits on another rank): segment
     states, the exclusive prefix in rank order (sata_state_accumulate), then
@@ -486,21 +488,33 @@ def test_sequence_split_emulated_ranks(sata, oracle_mod, d, lens):
     segs = [(qc[:, :, a:b].contiguous(), kc[:, :, a:b].contiguous(), vc[:, :, a:b].contiguous())
             for a, b in zip(bounds[:-1], bounds[1:])]
     impl = seqsplit.LibraryImpl()
-    gathered = [impl.tensors(impl.segment_state(*sg, 4)) for sg in segs]
+    gathered = [impl.tensors(impl.segment_state(*sg, P)) for sg in segs]
     ys, st = [], None
     for r, sg in enumerate(segs):
-        st = seqsplit.exclusive_prefix(impl, (1, 2, d, d, 4), gathered, r, list(lens), qc.device)
+        st = seqsplit.exclusive_prefix(impl, (1, 2, d, d, P), gathered, r, list(lens), qc.device)
         assert st.tokens == bounds[r]
-        ys.append(impl.prefill(*sg, 4, st))
+        ys.append(impl.prefill(*sg, P, st))
     y = torch.cat(ys, dim=2)
     torch.cuda.synchronize()
     assert sata.sata_sync_status() == 0
-    ref = _oracle_heads(oracle_mod, q, k, v, 4, [(0, 0), (0, 1)])
+    ref = _oracle_heads(oracle_mod, q, k, v, P, [(0, 0), (0, 1)])
     _check_heads(y, ref, what=f"split d={d} {lens}")
-    whole = sata.State(1, 2, d, d, 4)
-    y1 = sata.prefill(qc, kc, vc, P=4, state=whole)
+    whole = sata.State(1, 2, d, d, P)
+    y1 = sata.prefill(qc, kc, vc, P=P, state=whole)
     torch.cuda.synchronize()
     assert (y - y1).abs().max().item() <= 1e-3 * y1.abs().max().item()
     assert st.tokens == N
     for got, want in ((st.S, whole.S), (st.Z, whole.Z)):
         assert (got - want).abs().max().item() <= 1e-4 * want.abs().max().item()
+
+
+def test_state_accumulate_adds_and_counts(sata):
+    """sata_state_accumulate: S += dS, Z += dZ elementwise, tokens += n."""
+    st = sata.State(2, 3, 8, 16, 4)
+    dS = torch.randn_like(st.S)
+    dZ = torch.randn_like(st.Z)
+    sata.sata_state_accumulate(st.st, dS, dZ, 7)
+    sata.sata_state_accumulate(st.st, dS, dZ, 5)
+    torch.cuda.synchronize()
+    assert st.tokens == 12
+    assert torch.allclose(st.S, 2 * dS, rtol=0, atol=1e-6) and torch.allclose(st.Z, 2 * dZ, rtol=0, atol=1e-6)
