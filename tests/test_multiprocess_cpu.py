@@ -182,3 +182,26 @@ def test_sequence_split_exchange_gloo(lens):
         np.testing.assert_allclose(S_last[0, h], Sr, rtol=1e-10, atol=1e-12)
         np.testing.assert_allclose(Z_last[0, h], Zr, rtol=1e-10, atol=1e-12)
         assert tokens == sum(lens)
+
+
+def test_reference_arm_json_line(monkeypatch, capsys):
+    """The oracle arm on rank 0 prints one JSON line with the contract's keys."""
+    import json
+
+    sys.path.insert(0, ROOT)
+    import bench
+
+    monkeypatch.setenv("RANK", "0")
+    monkeypatch.setenv("WORLD_SIZE", "1")
+    monkeypatch.setattr(sys, "argv", ["bench.py", "--impl", "reference", "--steps", "1", "--warmup", "0",
+                                      "--cpu-seconds", "1"])
+    assert bench.main() == 0
+    lines = capsys.readouterr().out.strip().splitlines()
+    assert len(lines) == 1
+    line = json.loads(lines[0])
+    for key in ("impl", "metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step",
+                "higher_is_better", "scaling", "vs_baseline", "dtype", "data", "config", "cpu_baseline", "e2e"):
+        assert key in line, key
+    assert line["impl"] == "reference" and line["value"] > 0
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] >= 1
+    assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["value"] == line["value"]
