@@ -47,7 +47,10 @@ using simt::kL;
 using simt::contract_rows;
 using simt::readout_cols;
 using simt::update_rows;
-constexpr int kMaxComp = kMaxP - 2;   // indices left of a top-degree feature after removing one
+constexpr int kMaxComp = kMaxP - 2;
+// Row stride (floats) of r = [dy / den | -(dy . y) / den]: d_V + 1 rounded up
+// to a multiple of 4, so every row starts on a 16-byte boundary.
+__host__ __device__ constexpr int r_stride(int d_V) { return (d_V + 1 + 3) / 4 * 4; }   // indices left of a top-degree feature after removing one
 constexpr size_t kPartialBudget = size_t(2) << 30;  // bytes of partials per segment
 
 // Features are dealt to the kTF-feature tiles round-robin: tile tau holds the
@@ -154,19 +157,49 @@ __device__ __forceinline__ float feature(const float *x, uint32_t w, uint32_t hi
     return v;
 }
 
-// J_phi(x~)^T applied to one token's tile values `val`: the sum over the
-// tile's features f containing index i of val[f] * d phi_f / d x_i.
-__device__ __forceinline__ float jac_t(const uint32_t *off, const uint64_t *ent, int i, const float *x,
-                                       const float *val, int ncomp) {
+// J_phi(x~)^T applied to the tile values of kJT consecutive tokens: for index
+// i, acc[j] = sum over the tile's features f containing i of
+// val[j][f] * d phi_f / d x_i at token j (x~ rows of DK1 values, val rows of
+// kTF).  Each list entry is decoded once and applied to all kJT tokens, whose
+// loads are independent of each other.
+constexpr int kJT = 8;
+__device__ __forceinline__ void jac_t(const uint32_t *off, const uint64_t *ent, int i, const float *x, int DK1,
+                                      const float *val, int ncomp, float (&acc)[kJT]) {
+#pragma unroll
+    for (int j = 0; j < kJT; ++j) acc[j] = 0.f;
     const uint32_t b = off[i], e = off[i + 1];
-    float acc = 0.f;
     for (uint32_t n = b; n < e; ++n) {
         const uint64_t u = ent[n];
-        float d = (float)((u >> 8) & 255);
-        for (int m = 0; m < ncomp; ++m) d *= x[(u >> (16 + 8 * m)) & 255];
-        acc = fmaf(val[u & 255], d, acc);
+        const int m = (int)(u & 255);
+        const float mult = (float)((u >> 8) & 255);
+        int ci[kMaxComp];
+#pragma unroll
+        for (int c = 0; c < kMaxComp; ++c) ci[c] = (int)((u >> (16 + 8 * c)) & 255);
+#pragma unroll
+        for (int j = 0; j < kJT; ++j) {
+            float d = mult;
+#pragma unroll
+            for (int c = 0; c < kMaxComp; ++c)
+                if (c < ncomp) d *= x[j * DK1 + ci[c]];
+            acc[j] = fmaf(val[j * kTF + m], d, acc[j]);
+        }
     }
-    return acc;
+}
+
+// The Jacobian products of one chunk: items (index i, group of kJT tokens),
+// kL / kJT groups per index; the results go to out[t * ld + i] for t < nt.
+__device__ __forceinline__ void jac_chunk(const uint32_t *off, const uint64_t *ent, const float *x, int DK1,
+                                          const float *val, int ncomp, int d_K, int nt, float *out, int64_t ld) {
+    constexpr int G = kL / kJT;
+    for (int item = threadIdx.x; item < d_K * G; item += kThreads) {
+        const int i = item / G, tb = (item % G) * kJT;
+        if (tb >= nt) continue;
+        float acc[kJT];
+        jac_t(off, ent, i, x + tb * DK1, DK1, val + tb * kTF, ncomp, acc);
+#pragma unroll
+        for (int j = 0; j < kJT; ++j)
+            if (tb + j < nt) __stcs(out + (int64_t)(tb + j) * ld + i, acc[j]);
+    }
 }
 
 // Loads one chunk: x~q, x~k [kL][d_K+1] (last column 1), u = [v | 1] and r
@@ -175,26 +208,118 @@ __device__ __forceinline__ void load_chunk(const __nv_bfloat16 *q, const __nv_bf
                                            const __nv_bfloat16 *v, const float *r, int64_t row0,
                                            int nt, int d_K, int d_V, float *xq, float *xk, float *xu,
                                            float *xr) {
-    const int DK1 = d_K + 1, DV1 = d_V + 1;
-    for (int e = threadIdx.x; e < kL * DK1; e += kThreads) {
-        const int t = e / DK1, i = e % DK1;
-        float a = 0.f, b = 0.f;
-        if (t < nt) {
-            a = i < d_K ? __bfloat162float(q[(row0 + t) * d_K + i]) : 1.f;
-            b = i < d_K ? __bfloat162float(k[(row0 + t) * d_K + i]) : 1.f;
+    const int DK1 = d_K + 1, DV1 = d_V + 1, RW = r_stride(d_V);
+    if ((d_K & 7) == 0 && (d_V & 7) == 0) {
+        // 16-byte loads: 8 bf16 of q, k or v, or 4 floats of r, per load; all of a
+        // thread's loads are issued before its stores
+        constexpr int U = (kL * (kMaxDK / 8) + kThreads - 1) / kThreads;
+        const int nq = kL * (d_K / 8), nv = kL * (d_V / 8), nr = kL * (RW / 4);
+        uint4 bq[U], bk[U], bv[U];
+        float4 br[2 * U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int e = threadIdx.x + u * kThreads;
+            bq[u] = bk[u] = bv[u] = make_uint4(0, 0, 0, 0);
+            if (e < nq && e / (d_K / 8) < nt) {
+                const int64_t off = (row0 + e / (d_K / 8)) * d_K + (e % (d_K / 8)) * 8;
+                bq[u] = *reinterpret_cast<const uint4 *>(q + off);
+                bk[u] = *reinterpret_cast<const uint4 *>(k + off);
+            }
+            if (e < nv && e / (d_V / 8) < nt)
+                bv[u] = *reinterpret_cast<const uint4 *>(v + (row0 + e / (d_V / 8)) * d_V + (e % (d_V / 8)) * 8);
         }
-        xq[e] = a;
-        xk[e] = b;
+#pragma unroll
+        for (int u = 0; u < 2 * U; ++u) {
+            const int e = threadIdx.x + u * kThreads;
+            br[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (e < nr && e / (RW / 4) < nt)
+                br[u] = *reinterpret_cast<const float4 *>(r + (row0 + e / (RW / 4)) * RW + (e % (RW / 4)) * 4);
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int e = threadIdx.x + u * kThreads;
+            if (e < nq) {
+                const int t = e / (d_K / 8), i = (e % (d_K / 8)) * 8;
+                const __nv_bfloat16 *hq = reinterpret_cast<const __nv_bfloat16 *>(&bq[u]);
+                const __nv_bfloat16 *hk = reinterpret_cast<const __nv_bfloat16 *>(&bk[u]);
+#pragma unroll
+                for (int w = 0; w < 8; ++w) {
+                    xq[t * DK1 + i + w] = __bfloat162float(hq[w]);
+                    xk[t * DK1 + i + w] = __bfloat162float(hk[w]);
+                }
+            }
+            if (e < nv) {
+                const int t = e / (d_V / 8), j = (e % (d_V / 8)) * 8;
+                const __nv_bfloat16 *hv = reinterpret_cast<const __nv_bfloat16 *>(&bv[u]);
+#pragma unroll
+                for (int w = 0; w < 8; ++w) xu[t * DV1 + j + w] = __bfloat162float(hv[w]);
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < 2 * U; ++u) {
+            const int e = threadIdx.x + u * kThreads;
+            if (e < nr) {
+                const int t = e / (RW / 4), j = (e % (RW / 4)) * 4;
+                const float x4[4] = {br[u].x, br[u].y, br[u].z, br[u].w};
+#pragma unroll
+                for (int w = 0; w < 4; ++w)
+                    if (j + w < DV1) xr[t * DV1 + j + w] = x4[w];
+            }
+        }
+        for (int t = threadIdx.x; t < kL; t += kThreads) {   // the constant columns
+            const float one = t < nt ? 1.f : 0.f;
+            xq[t * DK1 + d_K] = one;
+            xk[t * DK1 + d_K] = one;
+            xu[t * DV1 + d_V] = one;
+        }
+        return;
     }
-    for (int e = threadIdx.x; e < kL * DV1; e += kThreads) {
-        const int t = e / DV1, j = e % DV1;
-        float a = 0.f, b = 0.f;
-        if (t < nt) {
-            a = j < d_V ? __bfloat162float(v[(row0 + t) * d_V + j]) : 1.f;
-            b = r[(row0 + t) * DV1 + j];
+    // other head sizes: element loads, every element a thread owns loaded
+    // before any is stored, so the global loads are in flight together
+    constexpr int U = (kL * (kMaxDK + 1) + kThreads - 1) / kThreads;
+    static_assert(kMaxDV <= kMaxDK, "one bound for both loops");
+    float a[U], b[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+        const int e = threadIdx.x + u * kThreads;
+        a[u] = 0.f;
+        b[u] = 0.f;
+        if (e < kL * DK1) {
+            const int t = e / DK1, i = e % DK1;
+            if (t < nt) {
+                a[u] = i < d_K ? __bfloat162float(q[(row0 + t) * d_K + i]) : 1.f;
+                b[u] = i < d_K ? __bfloat162float(k[(row0 + t) * d_K + i]) : 1.f;
+            }
         }
-        xu[e] = a;
-        xr[e] = b;
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+        const int e = threadIdx.x + u * kThreads;
+        if (e < kL * DK1) {
+            xq[e] = a[u];
+            xk[e] = b[u];
+        }
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+        const int e = threadIdx.x + u * kThreads;
+        a[u] = 0.f;
+        b[u] = 0.f;
+        if (e < kL * DV1) {
+            const int t = e / DV1, j = e % DV1;
+            if (t < nt) {
+                a[u] = j < d_V ? __bfloat162float(v[(row0 + t) * d_V + j]) : 1.f;
+                b[u] = r[(row0 + t) * RW + j];
+            }
+        }
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+        const int e = threadIdx.x + u * kThreads;
+        if (e < kL * DV1) {
+            xu[e] = a[u];
+            xr[e] = b[u];
+        }
     }
 }
 
@@ -238,12 +363,12 @@ bwd_r_kernel(const float *__restrict__ dy, const float *__restrict__ y, const fl
     float s = 0.f;
     for (int j = lane; j < d_V; j += 32) {
         const float g = dy[row * d_V + j] * inv;
-        r[row * (d_V + 1) + j] = g;
+        r[row * r_stride(d_V) + j] = g;
         s = fmaf(g, y[row * d_V + j], s);
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-    if (lane == 0) r[row * (d_V + 1) + d_V] = -s;
+    if (lane == 0) r[row * r_stride(d_V) + d_V] = -s;
 }
 
 // Shared-memory layout of the two scan kernels (floats after the tables).
@@ -322,11 +447,8 @@ bwd_q_scan_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__re
         }
         contract_rows<DV1>(Sx, xr, ts.coef, val);   // a (.) S r_t (zero rows past nt)
         __syncthreads();
-        for (int e = tid; e < nt * d_K; e += kThreads) {
-            const int t = e / d_K, i = e % d_K;
-            partials[(((int64_t)tile * BH + bh) * Tseg + c0 + t) * d_K + i] =
-                jac_t(ts.off, ts.ent, i, xq + t * DK1, val + t * kTF, ncomp);
-        }
+        jac_chunk(ts.off, ts.ent, xq, DK1, val, ncomp, d_K, nt,
+                  partials + (((int64_t)tile * BH + bh) * Tseg + c0) * d_K, d_K);
         update_rows<DV1>(Sx, phik, xu, nt);          // S += phi(K)^T U
     }
     __syncthreads();
@@ -384,11 +506,8 @@ bwd_kv_scan_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
         }
         contract_rows<DV1>(Gx, xu, ts.coef, val);   // a (.) G u_s
         __syncthreads();
-        for (int e = tid; e < nt * d_K; e += kThreads) {
-            const int t = e / d_K, i = e % d_K;
-            partials[(((int64_t)tile * BH + bh) * Tseg + c0 + t) * DKV + i] =
-                jac_t(ts.off, ts.ent, i, xk + t * DK1, val + t * kTF, ncomp);
-        }
+        jac_chunk(ts.off, ts.ent, xk, DK1, val, ncomp, d_K, nt,
+                  partials + (((int64_t)tile * BH + bh) * Tseg + c0) * DKV, DKV);
         {   // dv partial: (a (.) phi(k_s))^T G[:, :d_V]
             constexpr int JV = (DV + 31) / 32;
             float acc[4][JV];
@@ -400,7 +519,7 @@ bwd_kv_scan_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
                 for (int n = 0; n < JV; ++n) {
                     const int j = lane + 32 * n;
                     if (t < nt && j < DV)
-                        partials[(((int64_t)tile * BH + bh) * Tseg + c0 + t) * DKV + d_K + j] = acc[b][n];
+                        __stcs(partials + (((int64_t)tile * BH + bh) * Tseg + c0 + t) * DKV + d_K + j, acc[b][n]);
                 }
             }
         }
@@ -460,7 +579,7 @@ bwd_finish_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__re
         float a = 0.f, b = 0.f;
         if (t < nt) {
             a = j < d_V ? __bfloat162float(v[(row0 + t) * d_V + j]) : 1.f;
-            b = r[(row0 + t) * DV1 + j];
+            b = r[(row0 + t) * r_stride(d_V) + j];
         }
         xu[e] = a;
         xr[e] = b;
@@ -540,7 +659,7 @@ BwdLayout bwd_layout(int BH, int64_t N, int64_t F, int d_K, int d_V, int P, bool
     L.off_y = L.off_state + round256((size_t)BH * F * (d_V + 1) * sizeof(float));
     L.off_den = L.off_y + round256((size_t)BH * N * d_V * sizeof(float));
     L.off_r = L.off_den + round256((size_t)BH * N * sizeof(float));
-    L.total = L.off_r + round256((size_t)BH * N * (d_V + 1) * sizeof(float));
+    L.total = L.off_r + round256((size_t)BH * N * r_stride(d_V) * sizeof(float));
     return L;
 }
 
