@@ -412,7 +412,7 @@ def main():
     # ---------------- backward of the prefill ----------------
     bwd = None
     if not args.no_backward:
-        bwd = bench_backward(torch, sata, wl, args, world, dev, stream, clocks)
+        bwd = bench_backward(torch, sata, wl, args, world, dev, stream, peaks, peaks_src)
 
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
@@ -525,7 +525,7 @@ def backward_flops(d_K, d_V, P):
     return {"bwd_q_scan": 4 * F * (d_V + 1), "bwd_kv_scan": 4 * F * (d_V + 1) + 2 * F * d_V}
 
 
-def bench_backward(torch, sata, wl, args, world, dev, stream, clocks):
+def bench_backward(torch, sata, wl, args, world, dev, stream, peaks, peaks_src):
     w = wl.WORKLOADS[args.backward_workload]
     (q, k, v), _ = wl.make_inputs(w)
     qd, kd, vd, dy = q.to(dev), k.to(dev), v.to(dev), wl.cotangent(w).to(dev)
@@ -551,8 +551,9 @@ def bench_backward(torch, sata, wl, args, world, dev, stream, clocks):
         raise RuntimeError("device status after the backward")
     value = job_throughput(w.B * w.N, args.steps, world, ms)
     per_tok = backward_flops(w.d_K, w.d_V, w.P)
-    sm_ghz = (clocks.get("sm_max_mhz") or 1965.0) / 1000.0
-    alu_peak = NUM_SMS * FP32_LANES_PER_SM * 2 * sm_ghz / 1000.0
+    # the scans' contractions run on tensor cores with tf32 operands: the tf32 dense
+    # peak is the measured bf16 peak times the nominal ratio 1.1 / 2.25
+    tf32_peak = peaks["bf16_tflops"] * 1.1 / 2.25
     roof = None
     scans = {k_: stats[k_] for k_ in per_tok if k_ in stats}
     if scans:
@@ -560,10 +561,11 @@ def bench_backward(torch, sata, wl, args, world, dev, stream, clocks):
         n_l, ms_l = scans[dom]
         flops_per_launch = per_tok[dom] * w.B * w.H * w.N * args.steps / n_l
         achieved = flops_per_launch / (ms_l / n_l / 1000.0) / 1e12
-        roof = {"bound": "alu", "achieved": achieved, "peak": alu_peak, "unit": "TFLOP/s",
-                "frac": achieved / alu_peak, "kernel": dom, "launches_per_step": n_l / args.steps,
+        roof = {"bound": "tensor", "achieved": achieved, "peak": tf32_peak, "unit": "TFLOP/s",
+                "frac": achieved / tf32_peak, "kernel": dom, "launches_per_step": n_l / args.steps,
                 "ms_per_launch": ms_l / n_l, "algorithmic_flops_per_launch": flops_per_launch,
-                "peak_kind": "fp32 FMA: 148 SMs x 128 lanes x 2 FLOP x max SM clock",
+                "peak_kind": f"tf32 dense = {peaks_src} bf16 burst x 1.1/2.25 (nominal ratio); each fp32 "
+                             "product is three tf32 products (split operands), not credited",
                 "traffic": ncu_traffic(dom)}
     return {"metric": "SATA prefill backward tokens/s (dq, dk, dv)", "value": value, "unit": "tokens/s",
             "steps": args.steps, "ms_per_step": ms / args.steps,

@@ -36,6 +36,7 @@
 #include <vector>
 
 #include "sata_internal.h"
+#include "mma_tf32.cuh"
 #include "simt_tiles.cuh"
 
 namespace sata {
@@ -44,9 +45,6 @@ namespace {
 using simt::kThreads;
 using simt::kTF;
 using simt::kL;
-using simt::contract_rows;
-using simt::readout_cols;
-using simt::update_rows;
 constexpr int kMaxComp = kMaxP - 2;
 // Row stride (floats) of r = [dy / den | -(dy . y) / den]: d_V + 1 rounded up
 // to a multiple of 4, so every row starts on a 16-byte boundary.
@@ -164,7 +162,7 @@ __device__ __forceinline__ float feature(const float *x, uint32_t w, uint32_t hi
 // loads are independent of each other.
 constexpr int kJT = 8;
 __device__ __forceinline__ void jac_t(const uint32_t *off, const uint64_t *ent, int i, const float *x, int DK1,
-                                      const float *val, int ncomp, float (&acc)[kJT]) {
+                                      const float *val, int ldv, int ncomp, float (&acc)[kJT]) {
 #pragma unroll
     for (int j = 0; j < kJT; ++j) acc[j] = 0.f;
     const uint32_t b = off[i], e = off[i + 1];
@@ -181,7 +179,7 @@ __device__ __forceinline__ void jac_t(const uint32_t *off, const uint64_t *ent, 
 #pragma unroll
             for (int c = 0; c < kMaxComp; ++c)
                 if (c < ncomp) d *= x[j * DK1 + ci[c]];
-            acc[j] = fmaf(val[j * kTF + m], d, acc[j]);
+            acc[j] = fmaf(val[j * ldv + m], d, acc[j]);
         }
     }
 }
@@ -189,25 +187,32 @@ __device__ __forceinline__ void jac_t(const uint32_t *off, const uint64_t *ent, 
 // The Jacobian products of one chunk: items (index i, group of kJT tokens),
 // kL / kJT groups per index; the results go to out[t * ld + i] for t < nt.
 __device__ __forceinline__ void jac_chunk(const uint32_t *off, const uint64_t *ent, const float *x, int DK1,
-                                          const float *val, int ncomp, int d_K, int nt, float *out, int64_t ld) {
+                                          const float *val, int ldv, int ncomp, int d_K, int nt, float *out,
+                                          int64_t ld) {
     constexpr int G = kL / kJT;
     for (int item = threadIdx.x; item < d_K * G; item += kThreads) {
         const int i = item / G, tb = (item % G) * kJT;
         if (tb >= nt) continue;
         float acc[kJT];
-        jac_t(off, ent, i, x + tb * DK1, DK1, val + tb * kTF, ncomp, acc);
+        jac_t(off, ent, i, x + tb * DK1, DK1, val + tb * ldv, ldv, ncomp, acc);
 #pragma unroll
         for (int j = 0; j < kJT; ++j)
             if (tb + j < nt) __stcs(out + (int64_t)(tb + j) * ld + i, acc[j]);
     }
 }
 
+// Zeroes columns n .. w-1 of the kL rows of stride w.
+__device__ __forceinline__ void zero_pad(float *x, int w, int n) {
+    for (int e = threadIdx.x; e < kL * (w - n); e += kThreads) x[(e / (w - n)) * w + n + e % (w - n)] = 0.f;
+}
+
 // Loads one chunk: x~q, x~k [kL][d_K+1] (last column 1), u = [v | 1] and r
-// [kL][d_V+1]; rows past the end are zero.
+// (d_V + 1 values per row, row strides wu and wr, zero padded); rows past the
+// end are zero.
 __device__ __forceinline__ void load_chunk(const __nv_bfloat16 *q, const __nv_bfloat16 *k,
                                            const __nv_bfloat16 *v, const float *r, int64_t row0,
-                                           int nt, int d_K, int d_V, float *xq, float *xk, float *xu,
-                                           float *xr) {
+                                           int nt, int d_K, int d_V, float *xq, float *xk, float *xu, int wu,
+                                           float *xr, int wr) {
     const int DK1 = d_K + 1, DV1 = d_V + 1, RW = r_stride(d_V);
     if ((d_K & 7) == 0 && (d_V & 7) == 0) {
         // 16-byte loads: 8 bf16 of q, k or v, or 4 floats of r, per load; all of a
@@ -252,7 +257,7 @@ __device__ __forceinline__ void load_chunk(const __nv_bfloat16 *q, const __nv_bf
                 const int t = e / (d_V / 8), j = (e % (d_V / 8)) * 8;
                 const __nv_bfloat16 *hv = reinterpret_cast<const __nv_bfloat16 *>(&bv[u]);
 #pragma unroll
-                for (int w = 0; w < 8; ++w) xu[t * DV1 + j + w] = __bfloat162float(hv[w]);
+                for (int w = 0; w < 8; ++w) xu[t * wu + j + w] = __bfloat162float(hv[w]);
             }
         }
 #pragma unroll
@@ -263,15 +268,17 @@ __device__ __forceinline__ void load_chunk(const __nv_bfloat16 *q, const __nv_bf
                 const float x4[4] = {br[u].x, br[u].y, br[u].z, br[u].w};
 #pragma unroll
                 for (int w = 0; w < 4; ++w)
-                    if (j + w < DV1) xr[t * DV1 + j + w] = x4[w];
+                    if (j + w < DV1) xr[t * wr + j + w] = x4[w];
             }
         }
         for (int t = threadIdx.x; t < kL; t += kThreads) {   // the constant columns
             const float one = t < nt ? 1.f : 0.f;
             xq[t * DK1 + d_K] = one;
             xk[t * DK1 + d_K] = one;
-            xu[t * DV1 + d_V] = one;
+            xu[t * wu + d_V] = one;
         }
+        zero_pad(xu, wu, DV1);
+        zero_pad(xr, wr, DV1);
         return;
     }
     // other head sizes: element loads, every element a thread owns loaded
@@ -317,10 +324,12 @@ __device__ __forceinline__ void load_chunk(const __nv_bfloat16 *q, const __nv_bf
     for (int u = 0; u < U; ++u) {
         const int e = threadIdx.x + u * kThreads;
         if (e < kL * DV1) {
-            xu[e] = a[u];
-            xr[e] = b[u];
+            xu[(e / DV1) * wu + e % DV1] = a[u];
+            xr[(e / DV1) * wr + e % DV1] = b[u];
         }
     }
+    zero_pad(xu, wu, DV1);
+    zero_pad(xr, wr, DV1);
 }
 
 // Shared-memory image of one tile: its features' packed words and weights, its
@@ -372,16 +381,22 @@ bwd_r_kernel(const float *__restrict__ dy, const float *__restrict__ y, const fl
 }
 
 // Shared-memory layout of the two scan kernels (floats after the tables).
+// The three contractions run on tensor cores (mma_tf32.cuh); row strides
+// follow its bank rules: the state [kTF][WS] and the contraction's token rows
+// [kL][WA] are read with rows over g, the update's token rows [kL][WB] and
+// feature columns [kL][kFeatC] with rows over c, the dv readout's feature rows
+// [kL][kFeatG] with rows over g.
 struct ScanSmem {
     static size_t tables(int d_K, int max_entries) {
         size_t b = (size_t)(max_entries > 0 ? max_entries : 1) * sizeof(uint64_t);
         b += ((size_t)(d_K + 1) + 2 * kTF) * sizeof(uint32_t) + kTF * sizeof(float);
         return (b + 15) / 16 * 16;
     }
-    static size_t bytes(int d_K, int d_V, int nphi, int max_entries) {
+    static size_t bytes(int d_K, int d_V, bool kv, int max_entries) {
+        const size_t WS = mma32::stride_g(d_V + 1), WA = mma32::stride_g(d_V + 1), WB = mma32::stride_c(d_V + 1);
+        const size_t feat = kv ? (size_t)kL * (mma32::kFeatG + mma32::kFeatC) : (size_t)2 * kL * mma32::kFeatC;
         return tables(d_K, max_entries) +
-               sizeof(float) * ((size_t)kTF * (d_V + 1) + 2 * kL * (d_K + 1) + 2 * kL * (d_V + 1) +
-                                (size_t)nphi * kL * kTF);
+               sizeof(float) * ((size_t)kTF * WS + 2 * kL * (d_K + 1) + kL * (WA + WB) + feat);
     }
 };
 
@@ -405,7 +420,7 @@ __device__ __forceinline__ TileSmem carve_tables(uint8_t *base, int d_K, int max
 // dq partials of one feature tile of one head over the tokens [t0, t0 + T):
 // forward over the chunks with the tile's rows of S = sum phi(k) u^T.
 template <int DV>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kThreads, DV <= 64 ? 2 : 1)   // two CTAs per SM where shared memory allows
 bwd_q_scan_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k,
                   const __nv_bfloat16 *__restrict__ v, const float *__restrict__ r,
                   float *__restrict__ state, const uint32_t *__restrict__ packed,
@@ -413,18 +428,20 @@ bwd_q_scan_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__re
                   const uint32_t *__restrict__ jac_off, const uint64_t *__restrict__ jac_ent, int d_K,
                   int max_entries, int ncomp, int64_t F, int64_t N, int64_t t0, int T, int Tseg,
                   int load_state, float *__restrict__ partials) {
-    constexpr int DV1 = DV + 1;
+    constexpr int DV1 = DV + 1, KC = mma32::cols8(DV1);
+    constexpr int WS = mma32::stride_g(DV1), WA = mma32::stride_g(DV1), WB = mma32::stride_c(DV1);
+    constexpr int FC = mma32::kFeatC;
     extern __shared__ __align__(16) uint8_t smem_raw[];
     const int DK1 = d_K + 1;
     float *fs;
     const TileSmem ts = carve_tables(smem_raw, d_K, max_entries, &fs);
-    float *Sx = fs;                    // [kTF][DV1]
-    float *xq = Sx + kTF * DV1;        // [kL][DK1]
+    float *Sx = fs;                    // [kTF][WS]  state rows, zero padded
+    float *xq = Sx + kTF * WS;         // [kL][DK1]
     float *xk = xq + kL * DK1;
-    float *xu = xk + kL * DK1;         // [kL][DV1]
-    float *xr = xu + kL * DV1;
-    float *phik = xr + kL * DV1;       // [kL][kTF]
-    float *val = phik + kL * kTF;      // [kL][kTF]
+    float *xr = xk + kL * DK1;         // [kL][WA]   r rows (contraction operand)
+    float *xu = xr + kL * WA;          // [kL][WB]   u rows (update operand)
+    float *phik = xu + kL * WB;        // [kL][FC]
+    float *val = phik + kL * FC;       // [kL][FC]
 
     const int64_t bh = blockIdx.x;
     const int BH = gridDim.x;
@@ -432,29 +449,29 @@ bwd_q_scan_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__re
     const int nf = (int)((F - tile + ntiles - 1) / ntiles);
     const int tid = threadIdx.x;
     load_tile(ts, packed, packed_hi, coef, jac_off, jac_ent, tile, ntiles, nf, d_K);
-    for (int e = tid; e < kTF * DV1; e += kThreads) {
-        const int m = e / DV1, j = e % DV1;
-        Sx[e] = (load_state && m < nf) ? state[(bh * F + tile + (int64_t)m * ntiles) * DV1 + j] : 0.f;
+    for (int e = tid; e < kTF * WS; e += kThreads) {
+        const int m = e / WS, j = e % WS;
+        Sx[e] = (load_state && m < nf && j < DV1) ? state[(bh * F + tile + (int64_t)m * ntiles) * DV1 + j] : 0.f;
     }
     for (int c0 = 0; c0 < T; c0 += kL) {
         const int nt = min(kL, T - c0);
         __syncthreads();
-        load_chunk(q, k, v, r, bh * N + t0 + c0, nt, d_K, DV, xq, xk, xu, xr);
+        load_chunk(q, k, v, r, bh * N + t0 + c0, nt, d_K, DV, xq, xk, xu, WB, xr, WA);
         __syncthreads();
         for (int e = tid; e < kL * kTF; e += kThreads) {
             const int t = e / kTF, m = e % kTF;
-            phik[e] = (t < nt && m < nf) ? feature(xk + t * DK1, ts.pk[m], ts.hi[m]) : 0.f;
+            phik[t * FC + m] = (t < nt && m < nf) ? feature(xk + t * DK1, ts.pk[m], ts.hi[m]) : 0.f;
         }
-        contract_rows<DV1>(Sx, xr, ts.coef, val);   // a (.) S r_t (zero rows past nt)
+        mma32::contract_rows<KC>(Sx, WS, xr, WA, ts.coef, val, FC);   // a (.) S r_t (zero rows past nt)
         __syncthreads();
-        jac_chunk(ts.off, ts.ent, xq, DK1, val, ncomp, d_K, nt,
+        jac_chunk(ts.off, ts.ent, xq, DK1, val, FC, ncomp, d_K, nt,
                   partials + (((int64_t)tile * BH + bh) * Tseg + c0) * d_K, d_K);
-        update_rows<DV1>(Sx, phik, xu, nt);          // S += phi(K)^T U
+        mma32::update_rows<KC / 8>(Sx, WS, phik, FC, xu, WB);        // S += phi(K)^T U
     }
     __syncthreads();
     for (int e = tid; e < nf * DV1; e += kThreads) {
         const int m = e / DV1, j = e % DV1;
-        state[(bh * F + tile + (int64_t)m * ntiles) * DV1 + j] = Sx[e];
+        state[(bh * F + tile + (int64_t)m * ntiles) * DV1 + j] = Sx[m * WS + j];
     }
 }
 
@@ -462,7 +479,7 @@ bwd_q_scan_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__re
 // [t0, t0 + T): backward over the chunks with the tile's rows of
 // G = sum phi(q) r^T over the tokens after the chunk.
 template <int DV>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kThreads, DV <= 64 ? 2 : 1)
 bwd_kv_scan_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k,
                    const __nv_bfloat16 *__restrict__ v, const float *__restrict__ r,
                    float *__restrict__ state, const uint32_t *__restrict__ packed,
@@ -470,71 +487,63 @@ bwd_kv_scan_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
                    const uint32_t *__restrict__ jac_off, const uint64_t *__restrict__ jac_ent, int d_K,
                    int max_entries, int ncomp, int64_t F, int64_t N, int64_t t0, int T, int Tseg,
                    int load_state, float *__restrict__ partials) {
-    constexpr int DV1 = DV + 1;
+    constexpr int DV1 = DV + 1, KC = mma32::cols8(DV1);
+    constexpr int WS = mma32::stride_g(DV1), WA = mma32::stride_g(DV1), WB = mma32::stride_c(DV1);
+    constexpr int FC = mma32::kFeatC, FG = mma32::kFeatG;
     extern __shared__ __align__(16) uint8_t smem_raw[];
     const int DK1 = d_K + 1, DKV = d_K + DV;
     float *fs;
     const TileSmem ts = carve_tables(smem_raw, d_K, max_entries, &fs);
-    float *Gx = fs;                    // [kTF][DV1]
-    float *xq = Gx + kTF * DV1;        // [kL][DK1]
+    float *Gx = fs;                    // [kTF][WS]  G rows, zero padded
+    float *xq = Gx + kTF * WS;         // [kL][DK1]
     float *xk = xq + kL * DK1;
-    float *xu = xk + kL * DK1;         // [kL][DV1]
-    float *xr = xu + kL * DV1;
-    float *pka = xr + kL * DV1;        // [kL][kTF]  a (.) phi(k)
-    float *val = pka + kL * kTF;       // [kL][kTF]  a (.) G u, then phi(q)
+    float *xu = xk + kL * DK1;         // [kL][WA]   u rows (contraction operand)
+    float *xr = xu + kL * WA;          // [kL][WB]   r rows (update operand)
+    float *pka = xr + kL * WB;         // [kL][FG]   a (.) phi(k)
+    float *val = pka + kL * FG;        // [kL][FC]   a (.) G u, then phi(q)
 
     const int64_t bh = blockIdx.x;
     const int BH = gridDim.x;
     const int tile = blockIdx.y, ntiles = gridDim.y;
     const int nf = (int)((F - tile + ntiles - 1) / ntiles);
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int tid = threadIdx.x;
     load_tile(ts, packed, packed_hi, coef, jac_off, jac_ent, tile, ntiles, nf, d_K);
-    for (int e = tid; e < kTF * DV1; e += kThreads) {
-        const int m = e / DV1, j = e % DV1;
-        Gx[e] = (load_state && m < nf) ? state[(bh * F + tile + (int64_t)m * ntiles) * DV1 + j] : 0.f;
+    for (int e = tid; e < kTF * WS; e += kThreads) {
+        const int m = e / WS, j = e % WS;
+        Gx[e] = (load_state && m < nf && j < DV1) ? state[(bh * F + tile + (int64_t)m * ntiles) * DV1 + j] : 0.f;
     }
     const int nchunks = (T + kL - 1) / kL;
     for (int ci = nchunks - 1; ci >= 0; --ci) {
         const int c0 = ci * kL;
         const int nt = min(kL, T - c0);
         __syncthreads();
-        load_chunk(q, k, v, r, bh * N + t0 + c0, nt, d_K, DV, xq, xk, xu, xr);
+        load_chunk(q, k, v, r, bh * N + t0 + c0, nt, d_K, DV, xq, xk, xu, WA, xr, WB);
         __syncthreads();
         for (int e = tid; e < kL * kTF; e += kThreads) {
             const int t = e / kTF, m = e % kTF;
-            pka[e] = (t < nt && m < nf) ? ts.coef[m] * feature(xk + t * DK1, ts.pk[m], ts.hi[m]) : 0.f;
+            pka[t * FG + m] = (t < nt && m < nf) ? ts.coef[m] * feature(xk + t * DK1, ts.pk[m], ts.hi[m]) : 0.f;
         }
-        contract_rows<DV1>(Gx, xu, ts.coef, val);   // a (.) G u_s
+        mma32::contract_rows<KC>(Gx, WS, xu, WA, ts.coef, val, FC);   // a (.) G u_s
         __syncthreads();
-        jac_chunk(ts.off, ts.ent, xk, DK1, val, ncomp, d_K, nt,
+        jac_chunk(ts.off, ts.ent, xk, DK1, val, FC, ncomp, d_K, nt,
                   partials + (((int64_t)tile * BH + bh) * Tseg + c0) * DKV, DKV);
-        {   // dv partial: (a (.) phi(k_s))^T G[:, :d_V]
-            constexpr int JV = (DV + 31) / 32;
-            float acc[4][JV];
-            readout_cols<JV, DV1>(pka, Gx, DV, acc);
-#pragma unroll
-            for (int b = 0; b < 4; ++b) {
-                const int t = warp + 8 * b;
-#pragma unroll
-                for (int n = 0; n < JV; ++n) {
-                    const int j = lane + 32 * n;
-                    if (t < nt && j < DV)
-                        __stcs(partials + (((int64_t)tile * BH + bh) * Tseg + c0 + t) * DKV + d_K + j, acc[b][n]);
-                }
-            }
-        }
+        // dv partial: (a (.) phi(k_s))^T G[:, :d_V]
+        float *dvp = partials + (((int64_t)tile * BH + bh) * Tseg + c0) * DKV + d_K;
+        mma32::readout_cols<mma32::cols8(DV) / 8>(pka, FG, Gx, WS, [&](int t, int j, float x) {
+            if (t < nt && j < DV) __stcs(dvp + (int64_t)t * DKV + j, x);
+        });
         __syncthreads();
         for (int e = tid; e < kL * kTF; e += kThreads) {   // phi(q) over the consumed values
             const int t = e / kTF, m = e % kTF;
-            val[e] = (t < nt && m < nf) ? feature(xq + t * DK1, ts.pk[m], ts.hi[m]) : 0.f;
+            val[t * FC + m] = (t < nt && m < nf) ? feature(xq + t * DK1, ts.pk[m], ts.hi[m]) : 0.f;
         }
         __syncthreads();
-        update_rows<DV1>(Gx, val, xr, nt);          // G += phi(Q)^T R
+        mma32::update_rows<KC / 8>(Gx, WS, val, FC, xr, WB);         // G += phi(Q)^T R
     }
     __syncthreads();
     for (int e = tid; e < nf * DV1; e += kThreads) {
         const int m = e / DV1, j = e % DV1;
-        state[(bh * F + tile + (int64_t)m * ntiles) * DV1 + j] = Gx[e];
+        state[(bh * F + tile + (int64_t)m * ntiles) * DV1 + j] = Gx[m * WS + j];
     }
 }
 
@@ -729,8 +738,8 @@ cudaError_t launch_prefill_backward(const DeviceBasis &basis, int BH, int64_t N,
     launch_end(kBwdR, stream);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
 
-    const size_t smemQ = ScanSmem::bytes(d_K, d_V, 2, max_ent);
-    const size_t smemKV = ScanSmem::bytes(d_K, d_V, 2, max_ent);
+    const size_t smemQ = ScanSmem::bytes(d_K, d_V, false, max_ent);
+    const size_t smemKV = ScanSmem::bytes(d_K, d_V, true, max_ent);
     const size_t smemF = sizeof(float) * ((size_t)2 * kL * d_K + 2 * kL * (d_V + 1) + 2 * kL * kL);
     if ((e = cudaFuncSetAttribute(q_scan, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   (int)smemQ)) != cudaSuccess)
