@@ -211,8 +211,9 @@ SATA_API int sata_prefill_host(const void *q, const void *k, const void *v, floa
  * over the sequence with S gives dq and one pass backward with
  * G = sum_t phi(q_t) [dy_t / den_t | -(dy_t . y_t) / den_t]^T gives dk and dv.
  * The recomputed forward takes the prefill's path (tensor cores where
- * sata_prefill_ex would use them, keeping den); the two gradient scans run on
- * CUDA cores in fp32 for every supported shape.
+ * sata_prefill_ex would use them, keeping den); the two gradient scans run for
+ * every supported shape, their contractions on tensor cores with tf32 operands
+ * split into high and low parts (fp32-level accuracy).
  *   q, k: bf16 [B][H][N][d_K];  v: bf16 [B][H][N][d_V]  (the forward's inputs)
  *   dy:   fp32 [B][H][N][d_V]
  *   dq, dk: fp32 [B][H][N][d_K];  dv: fp32 [B][H][N][d_V]  (overwritten)

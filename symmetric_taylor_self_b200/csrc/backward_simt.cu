@@ -1,5 +1,5 @@
-// Backward pass of the causal prefill on CUDA cores (fp32): the gradients of a
-// loss L with respect to q, k and v, given dL/dy for every output.
+// Backward pass of the causal prefill (fp32-accurate): the gradients of a loss
+// L with respect to q, k and v, given dL/dy for every output.
 //
 // The method's pages define no backward pass; they expect the attention to be
 // trained inside ordinary Transformer pipelines ([CC-TAYLOR] "Comparison with
