@@ -615,9 +615,8 @@ bwd_finish_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__re
     __syncthreads();
     for (int e = tid; e < nt * d_K; e += kThreads) {
         const int t = e / d_K, i = e % d_K;
-        float a = 0.f;
-        for (int tile = 0; tile < ntiles; ++tile)
-            a += partials[(((int64_t)tile * BH + bh) * Tseg + c0 + t) * PW + i];
+        const float a = simt::sum_strided(partials + ((int64_t)bh * Tseg + c0 + t) * PW + i, ntiles,
+                                          (int64_t)BH * Tseg * PW);
         float b = 0.f;
         if (!KV) {
             for (int s = 0; s <= t; ++s) b = fmaf(Wd[t * kL + s], xk[s * d_K + i], b);
@@ -629,9 +628,8 @@ bwd_finish_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__re
     if (KV) {
         for (int e = tid; e < nt * d_V; e += kThreads) {
             const int s = e / d_V, j = e % d_V;
-            float a = 0.f;
-            for (int tile = 0; tile < ntiles; ++tile)
-                a += partials[(((int64_t)tile * BH + bh) * Tseg + c0 + s) * PW + d_K + j];
+            const float a = simt::sum_strided(partials + ((int64_t)bh * Tseg + c0 + s) * PW + d_K + j, ntiles,
+                                              (int64_t)BH * Tseg * PW);
             float b = 0.f;
             for (int u = s; u < nt; ++u) b = fmaf(Ww[u * kL + s], xr[u * DV1 + j], b);
             dv[(row0 + s) * d_V + j] = a + b;

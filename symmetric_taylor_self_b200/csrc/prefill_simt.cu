@@ -78,23 +78,7 @@ simt_scan_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__res
     for (int c0 = 0; c0 < T; c0 += kL) {
         const int nt = min(kL, T - c0);
         __syncthreads();
-        for (int e = tid; e < kL * DK1; e += kThreads) {
-            const int t = e / DK1, i = e % DK1;
-            float a = 0.f, b = 0.f;
-            if (t < nt) {
-                const int64_t row = (bh * N + t0 + c0 + t) * d_K;
-                a = i < d_K ? __bfloat162float(q[row + i]) : 1.f;
-                b = i < d_K ? __bfloat162float(k[row + i]) : 1.f;
-            }
-            xq[e] = a;
-            xk[e] = b;
-        }
-        for (int e = tid; e < kL * DV1; e += kThreads) {
-            const int t = e / DV1, j = e % DV1;
-            float a = 0.f;
-            if (t < nt) a = j < d_V ? __bfloat162float(v[(bh * N + t0 + c0 + t) * d_V + j]) : 1.f;
-            xv[e] = a;
-        }
+        simt::load_qkv_chunk(q, k, v, bh * N + t0 + c0, nt, d_K, d_V, xq, xk, xv);
         __syncthreads();
         for (int e = tid; e < kL * kTF; e += kThreads) {
             const int t = e / kTF, f = e % kTF;
@@ -199,9 +183,8 @@ simt_finish_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
     __syncthreads();
     for (int e = tid; e < nt * DV1; e += kThreads) {
         const int t = e / DV1, j = e % DV1;
-        float a = 0.f;
-        for (int tile = 0; tile < ntiles; ++tile)
-            a += partials[(((int64_t)tile * BH + bh) * Tseg + c0 + t) * DV1 + j];
+        const float a = simt::sum_strided(partials + ((int64_t)bh * Tseg + c0 + t) * DV1 + j, ntiles,
+                                          (int64_t)BH * Tseg * DV1);
         float b = 0.f;
         for (int s = 0; s <= t; ++s) b = fmaf(W[t * kL + s], xv[s * DV1 + j], b);
         acc[e] = a + b;

@@ -7,6 +7,10 @@
 // d_V, so the 32 lanes of a warp reading 32 different rows hit 32 banks.
 #pragma once
 
+#include <cuda_bf16.h>
+
+#include "sata_internal.h"
+
 namespace sata {
 namespace simt {
 
@@ -22,6 +26,115 @@ __device__ __forceinline__ float taylor_exp(float x, int n) {
     for (int p = 7; p >= 1; --p)
         if (p < n) h = fmaf(h, x * (1.f / p), 1.f);
     return h;
+}
+
+// Loads one chunk of kL token rows starting at row0 into shared memory:
+// x~q, x~k [kL][d_K + 1] (last column 1) and [v | 1] [kL][d_V + 1]; rows past nt
+// are zero.  16-byte loads (8 bf16) when d_K and d_V are multiples of 8, else
+// element loads; either way all of a thread's loads are issued before its
+// stores, so they are in flight together.
+__device__ __forceinline__ void load_qkv_chunk(const __nv_bfloat16 *q, const __nv_bfloat16 *k,
+                                               const __nv_bfloat16 *v, int64_t row0, int nt, int d_K, int d_V,
+                                               float *xq, float *xk, float *xv) {
+    const int DK1 = d_K + 1, DV1 = d_V + 1;
+    if ((d_K & 7) == 0 && (d_V & 7) == 0) {
+        constexpr int U = (kL * (kMaxDK / 8) + kThreads - 1) / kThreads;
+        const int nq = kL * (d_K / 8), nv = kL * (d_V / 8);
+        uint4 bq[U], bk[U], bv[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int e = threadIdx.x + u * kThreads;
+            bq[u] = bk[u] = bv[u] = make_uint4(0, 0, 0, 0);
+            if (e < nq && e / (d_K / 8) < nt) {
+                const int64_t off = (row0 + e / (d_K / 8)) * d_K + (e % (d_K / 8)) * 8;
+                bq[u] = *reinterpret_cast<const uint4 *>(q + off);
+                bk[u] = *reinterpret_cast<const uint4 *>(k + off);
+            }
+            if (e < nv && e / (d_V / 8) < nt)
+                bv[u] = *reinterpret_cast<const uint4 *>(v + (row0 + e / (d_V / 8)) * d_V + (e % (d_V / 8)) * 8);
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int e = threadIdx.x + u * kThreads;
+            if (e < nq) {
+                const int t = e / (d_K / 8), i = (e % (d_K / 8)) * 8;
+                const __nv_bfloat16 *hq = reinterpret_cast<const __nv_bfloat16 *>(&bq[u]);
+                const __nv_bfloat16 *hk = reinterpret_cast<const __nv_bfloat16 *>(&bk[u]);
+#pragma unroll
+                for (int w = 0; w < 8; ++w) {
+                    xq[t * DK1 + i + w] = __bfloat162float(hq[w]);
+                    xk[t * DK1 + i + w] = __bfloat162float(hk[w]);
+                }
+            }
+            if (e < nv) {
+                const int t = e / (d_V / 8), j = (e % (d_V / 8)) * 8;
+                const __nv_bfloat16 *hv = reinterpret_cast<const __nv_bfloat16 *>(&bv[u]);
+#pragma unroll
+                for (int w = 0; w < 8; ++w) xv[t * DV1 + j + w] = __bfloat162float(hv[w]);
+            }
+        }
+        for (int t = threadIdx.x; t < kL; t += kThreads) {   // the constant columns
+            const float one = t < nt ? 1.f : 0.f;
+            xq[t * DK1 + d_K] = one;
+            xk[t * DK1 + d_K] = one;
+            xv[t * DV1 + d_V] = one;
+        }
+        return;
+    }
+    constexpr int U = (kL * (kMaxDK + 1) + kThreads - 1) / kThreads;
+    static_assert(kMaxDV <= kMaxDK, "one bound for both loops");
+    float a[U], b[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+        const int e = threadIdx.x + u * kThreads;
+        a[u] = 0.f;
+        b[u] = 0.f;
+        if (e < kL * DK1) {
+            const int t = e / DK1, i = e % DK1;
+            if (t < nt) {
+                a[u] = i < d_K ? __bfloat162float(q[(row0 + t) * d_K + i]) : 1.f;
+                b[u] = i < d_K ? __bfloat162float(k[(row0 + t) * d_K + i]) : 1.f;
+            }
+        }
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+        const int e = threadIdx.x + u * kThreads;
+        if (e < kL * DK1) {
+            xq[e] = a[u];
+            xk[e] = b[u];
+        }
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+        const int e = threadIdx.x + u * kThreads;
+        a[u] = 0.f;
+        if (e < kL * DV1) {
+            const int t = e / DV1, j = e % DV1;
+            if (t < nt) a[u] = j < d_V ? __bfloat162float(v[(row0 + t) * d_V + j]) : 1.f;
+        }
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+        const int e = threadIdx.x + u * kThreads;
+        if (e < kL * DV1) xv[e] = a[u];
+    }
+}
+
+// sum_{g < n} p[g * stride] in a fixed order, eight loads in flight: eight
+// running sums over g mod 8, then the tail, then a fixed pairwise combination.
+__device__ __forceinline__ float sum_strided(const float *__restrict__ p, int n, int64_t stride) {
+    float s[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    int g = 0;
+    for (; g + 8 <= n; g += 8) {
+        float x[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) x[u] = p[(int64_t)(g + u) * stride];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) s[u] += x[u];
+    }
+    for (; g < n; ++g) s[0] += p[(int64_t)g * stride];
+    return ((s[0] + s[1]) + (s[2] + s[3])) + ((s[4] + s[5]) + (s[6] + s[7]));
 }
 
 // Register-tiled contraction out[t][m] = coef[m] * sum_j X[m][j] * Y[t][j] over
