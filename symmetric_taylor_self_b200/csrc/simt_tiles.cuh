@@ -1,10 +1,12 @@
-// Register-tiled building blocks of the CUDA-core scans (prefill and its
-// backward): 256 threads, tiles of kTF = 128 features, chunks of kL = 32 tokens.
-// Thread (warp, lane) owns tokens t = warp + 8b (b < 4) and features
-// m = lane + 32a (a < 4) or value columns; every operand row is read from shared
-// memory once per thread and reused across the thread's register tile.
-// Shared-memory rows of d_V + 1 floats have an odd stride for every supported
-// d_V, so the 32 lanes of a warp reading 32 different rows hit 32 banks.
+// Building blocks of the chunked scans that run outside the tensor-core
+// prefill (the CUDA-core prefill and the backward): 256 threads, tiles of
+// kTF = 128 features, chunks of kL = 32 tokens.  The chunk loader, the
+// truncated series, the fixed-order strided sum, and the CUDA-core prefill's
+// register-tiled contractions: thread (warp, lane) owns tokens t = warp + 8b
+// (b < 4) and features m = lane + 32a (a < 4) or value columns, and reuses every
+// shared-memory operand across that tile.  Shared-memory rows of d_V + 1 floats
+// have an odd stride for every supported d_V, so the 32 lanes of a warp reading
+// 32 different rows hit 32 banks.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -135,32 +137,6 @@ __device__ __forceinline__ float sum_strided(const float *__restrict__ p, int n,
     }
     for (; g < n; ++g) s[0] += p[(int64_t)g * stride];
     return ((s[0] + s[1]) + (s[2] + s[3])) + ((s[4] + s[5]) + (s[6] + s[7]));
-}
-
-// Register-tiled contraction out[t][m] = coef[m] * sum_j X[m][j] * Y[t][j] over
-// the j < DV1 columns (X: a tile's state rows, Y: the chunk's r or u rows):
-// thread (warp, lane) owns t = warp + 8b (b < 4) and m = lane + 32a (a < 4).
-template <int DV1>
-__device__ __forceinline__ void contract_rows(const float *X, const float *Y, const float *coef, float *out) {
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    float acc[4][4] = {};
-#pragma unroll 4
-    for (int j = 0; j < DV1; ++j) {
-        float x[4], y[4];
-#pragma unroll
-        for (int a = 0; a < 4; ++a) x[a] = X[(lane + 32 * a) * DV1 + j];
-#pragma unroll
-        for (int b = 0; b < 4; ++b) y[b] = Y[(warp + 8 * b) * DV1 + j];
-#pragma unroll
-        for (int b = 0; b < 4; ++b)
-#pragma unroll
-            for (int a = 0; a < 4; ++a) acc[b][a] = fmaf(y[b], x[a], acc[b][a]);
-    }
-#pragma unroll
-    for (int b = 0; b < 4; ++b)
-#pragma unroll
-        for (int a = 0; a < 4; ++a)
-            out[(warp + 8 * b) * kTF + lane + 32 * a] = coef[lane + 32 * a] * acc[b][a];
 }
 
 // Register-tiled rank-nt update X[m][j] += sum_t A[t][m] * Y[t][j]: thread
