@@ -205,3 +205,22 @@ def test_reference_arm_json_line(monkeypatch, capsys):
     assert line["impl"] == "reference" and line["value"] > 0
     assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] >= 1
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["value"] == line["value"]
+
+
+def test_sequence_split_single_rank_without_process_group():
+    """Without a process group the split runs as one rank: no exchange, an empty
+    prefix, and the outputs of one prefill."""
+    import numpy as np
+
+    sys.path.insert(0, ROOT)
+    import oracle
+    from symmetric_taylor_self_b200 import seqsplit
+    from symmetric_taylor_self_b200 import workloads as wl
+
+    q, k, v = wl.random_inputs(1, 2, 37, 3, 2, seed=91)
+    y, st = seqsplit.prefill_sequence_split(q, k, v, P=4, impl=_OracleImpl())
+    assert st["tokens"] == 37
+    for h in range(2):
+        yr, _, Sr, Zr = oracle.scan(q[0, h], k[0, h], v[0, h], 4)
+        np.testing.assert_allclose(y[0, h].numpy(), yr, rtol=1e-12, atol=1e-12)
+        np.testing.assert_allclose(st["S"][0, h].numpy(), Sr, rtol=1e-12, atol=1e-12)
