@@ -217,10 +217,12 @@ __device__ __forceinline__ void load_chunk(const __nv_bfloat16 *q, const __nv_bf
     if ((d_K & 7) == 0 && (d_V & 7) == 0) {
         // 16-byte loads: 8 bf16 of q, k or v, or 4 floats of r, per load; all of a
         // thread's loads are issued before its stores
-        constexpr int U = (kL * (kMaxDK / 8) + kThreads - 1) / kThreads;
+        constexpr int U = (kL * (kMaxDK / 8) + kThreads - 1) / kThreads;             // q, k, v pieces
+        constexpr int UR = (kL * (r_stride(kMaxDV) / 4) + kThreads - 1) / kThreads;  // r pieces
+        static_assert(kMaxDV <= kMaxDK, "one bound for q, k and v");
         const int nq = kL * (d_K / 8), nv = kL * (d_V / 8), nr = kL * (RW / 4);
         uint4 bq[U], bk[U], bv[U];
-        float4 br[2 * U];
+        float4 br[UR];
 #pragma unroll
         for (int u = 0; u < U; ++u) {
             const int e = threadIdx.x + u * kThreads;
@@ -234,7 +236,7 @@ __device__ __forceinline__ void load_chunk(const __nv_bfloat16 *q, const __nv_bf
                 bv[u] = *reinterpret_cast<const uint4 *>(v + (row0 + e / (d_V / 8)) * d_V + (e % (d_V / 8)) * 8);
         }
 #pragma unroll
-        for (int u = 0; u < 2 * U; ++u) {
+        for (int u = 0; u < UR; ++u) {
             const int e = threadIdx.x + u * kThreads;
             br[u] = make_float4(0.f, 0.f, 0.f, 0.f);
             if (e < nr && e / (RW / 4) < nt)
@@ -261,7 +263,7 @@ __device__ __forceinline__ void load_chunk(const __nv_bfloat16 *q, const __nv_bf
             }
         }
 #pragma unroll
-        for (int u = 0; u < 2 * U; ++u) {
+        for (int u = 0; u < UR; ++u) {
             const int e = threadIdx.x + u * kThreads;
             if (e < nr) {
                 const int t = e / (RW / 4), j = (e % (RW / 4)) * 4;

@@ -389,7 +389,8 @@ def _check_grads(sata, oracle_mod, B, H, N, d_K, d_V, P, seed, heads=None):
 @pytest.mark.parametrize("d_K,d_V,P,N", [(16, 16, 4, 100), (8, 8, 4, 77), (32, 32, 4, 70),
                                          (64, 64, 4, 130), (16, 32, 3, 65), (12, 8, 2, 50),
                                          (8, 8, 5, 40), (4, 4, 1, 33), (128, 128, 2, 37),
-                                         (6, 8, 7, 29), (32, 4, 4, 140)])
+                                         (6, 8, 7, 29), (32, 4, 4, 140), (128, 128, 2, 100),
+                                         (64, 128, 2, 70)])
 def test_backward_matches_oracle(sata, oracle_mod, path, d_K, d_V, P, N):
     """auto: the recomputed forward runs on tensor cores for d_K = d_V in
     {16, 32, 64}, P <= 4; cuda_core: always on CUDA cores."""
