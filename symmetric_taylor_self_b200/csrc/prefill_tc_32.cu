@@ -1,0 +1,8 @@
+// Tensor-core prefill instances: d_K = 32, d_V = 16, d_K = 32, d_V = 32, d_K = 32, d_V = 64.
+#include "prefill_tc_kernels.cuh"
+
+namespace sata {
+SATA_TC_DEFINE(32, 16)
+SATA_TC_DEFINE(32, 32)
+SATA_TC_DEFINE(32, 64)
+}  // namespace sata

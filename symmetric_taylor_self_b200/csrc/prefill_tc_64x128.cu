@@ -1,0 +1,6 @@
+// Tensor-core prefill instances: d_K = 64, d_V = 128.
+#include "prefill_tc_kernels.cuh"
+
+namespace sata {
+SATA_TC_DEFINE(64, 128)
+}  // namespace sata

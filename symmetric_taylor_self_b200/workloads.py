@@ -112,10 +112,11 @@ def cotangent(w: Workload):
     return random_cotangent(w.B, w.H, w.N, w.d_V, seed=w.seed * 2 ** 20 + 2 ** 19)
 
 
-def random_inputs(B, H, N, d_K, d_V, seed, dtype=torch.bfloat16, scale=1.0):
-    """Free-form seeded N(0, scale^2) inputs [B, H, N, d] for edge-case tests."""
+def random_inputs(B, H, N, d_K, d_V, seed, dtype=torch.bfloat16, scale=1.0, vscale=1.0):
+    """Free-form seeded inputs [B, H, N, d] for edge-case tests: q, k ~ N(0, scale^2),
+    v ~ N(0, vscale^2)."""
     g = torch.Generator("cpu").manual_seed(seed)
     q = torch.randn(B, H, N, d_K, generator=g) * scale
     k = torch.randn(B, H, N, d_K, generator=g) * scale
-    v = torch.randn(B, H, N, d_V, generator=g)
+    v = torch.randn(B, H, N, d_V, generator=g) * vscale
     return q.to(dtype), k.to(dtype), v.to(dtype)

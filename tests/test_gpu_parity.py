@@ -87,11 +87,15 @@ def test_prefill_and_decode_higher_P(sata, oracle_mod, d, P, N):
     _check_heads(yall, _oracle_heads(oracle_mod, q, k, v, P, [(0, 0), (0, 1)]), what=f"d={d} P={P}")
 
 
-@pytest.mark.parametrize("d_K,d_V,N", [(32, 64, 150), (64, 16, 140), (128, 128, 20), (12, 8, 90)])
-def test_prefill_and_decode_other_head_sizes(sata, oracle_mod, d_K, d_V, N):
-    """Head sizes outside the tensor-core set (d_K != d_V, d = 128, odd d_K) run on
-    the CUDA-core prefill; prefill plus two decode steps against the oracle."""
+@pytest.mark.parametrize("d_K,d_V,N,tc", [(32, 64, 150, True), (64, 16, 140, True), (128, 128, 20, True),
+                                          (128, 128, 300, True), (64, 128, 200, True), (128, 64, 260, True),
+                                          (16, 64, 140, True), (12, 8, 90, False)])
+def test_prefill_and_decode_other_head_sizes(sata, oracle_mod, d_K, d_V, N, tc):
+    """d_K != d_V and d = 128 run on the tensor-core prefill (d_K, d_V in
+    {16, 32, 64, 128}); odd or small head sizes on the CUDA-core prefill.
+    Prefill plus two decode steps against the oracle."""
     _set_path(sata, "auto")
+    sata.sata_reset_kernel_stats()
     B, H, steps = 1, 1, 2
     q, k, v = wl.random_inputs(B, H, N + steps, d_K, d_V, seed=1300 + d_K + d_V)
     st = sata.State(B, H, d_K, d_V, 4)
@@ -102,6 +106,7 @@ def test_prefill_and_decode_other_head_sizes(sata, oracle_mod, d_K, d_V, N):
     torch.cuda.synchronize()
     assert sata.sata_sync_status() == 0
     yall = torch.cat([y, torch.stack(ys, dim=2)], dim=2)
+    assert ("tc_scan" in sata.sata_kernel_stats()) == tc
     _check_heads(yall, _oracle_heads(oracle_mod, q, k, v, 4, [(0, 0)]), what=f"d_K={d_K} d_V={d_V}")
 
 
@@ -305,7 +310,10 @@ def test_prefill_host_matches_device_and_oracle(sata, oracle_mod, path, d, N):
     assert sata.sata_sync_status() == 0
     assert torch.isfinite(yh).all()
     scale = y_dev.abs().max().item()
-    assert (yh - y_dev.cpu()).abs().max().item() <= 1e-6 * scale
+    # The host path runs the sequence as token segments, each with its own power-of-two
+    # operand prescale (from that segment's maxima), so the fp16 roundings of tiny operands
+    # differ from the one-segment device call: agreement to 1e-4, both within the oracle bar.
+    assert (yh - y_dev.cpu()).abs().max().item() <= 1e-4 * scale
     _check_heads(yh, _oracle_heads(oracle_mod, q, k, v, 4, [(0, 1)]), what=f"host d={d} N={N}")
 
 
@@ -355,15 +363,47 @@ def test_bounded_wait_reports_timeout(sata):
     sata.sata_set_option(sata.SATA_OPT_PREFILL_PATH, 0)
 
 
-def test_out_of_range_inputs_are_reported(sata):
+@pytest.mark.parametrize("d_K,d_V,scale,vscale", [(32, 32, 100.0, 1.0), (32, 32, 1e-3, 1.0), (64, 64, 30.0, 1e4),
+                                                (16, 16, 1.0, 1e-4), (64, 64, 1e-2, 300.0)])
+def test_tensor_core_path_any_input_range(sata, oracle_mod, d_K, d_V, scale, vscale):
+    """The pages put no bound on q, k, v and the accuracy depends on the input
+    statistics ([CC-TAYLOR] "Precision vs efficiency"): the tensor-core path
+    prescales each head's q/c, k and v by powers of two, so inputs far from
+    N(0, 1) keep their accuracy.  Gated per token on the well-conditioned
+    tokens (kappa <= 8, as everywhere), against the oracle's direct form."""
     sata.sata_set_option(sata.SATA_OPT_PREFILL_PATH, 2)
-    q, k, v = wl.random_inputs(1, 1, 64, 32, 32, seed=9, scale=100.0)
-    sata.prefill(q.cuda(), k.cuda(), v.cuda(), P=4)
-    assert sata.sata_sync_status() == sata.SATA_ERANGE
-    q, k, v = wl.random_inputs(1, 1, 64, 32, 32, seed=9)
-    sata.prefill(q.cuda(), k.cuda(), v.cuda(), P=4)
-    assert sata.sata_sync_status() == 0
-    sata.sata_set_option(sata.SATA_OPT_PREFILL_PATH, 0)
+    try:
+        N = 300
+        q, k, v = wl.random_inputs(1, 2, N, d_K, d_V, seed=9 + d_K, scale=scale, vscale=vscale)
+        y = sata.prefill(q.cuda(), k.cuda(), v.cuda(), P=4)
+        torch.cuda.synchronize()
+        assert sata.sata_sync_status() == 0
+        for h in range(2):
+            yr, den, kappa = oracle_mod.direct(q[0, h], k[0, h], v[0, h], 4)
+            err, excl, _ = token_rel_err(y[0, h].double().cpu().numpy(), yr, kappa)
+            assert err <= TOL, f"scale {scale}/{vscale} head {h}: {err:.3e}"
+            assert excl < N // 2
+    finally:
+        sata.sata_set_option(sata.SATA_OPT_PREFILL_PATH, 0)
+
+
+def test_non_finite_inputs_are_reported(sata):
+    """An infinite input cannot be represented: the call reports SATA_ERANGE at
+    sync and the affected head's outputs are not finite (never silent); the other
+    head and the next call are unaffected."""
+    sata.sata_set_option(sata.SATA_OPT_PREFILL_PATH, 2)
+    try:
+        q, k, v = wl.random_inputs(1, 2, 200, 32, 32, seed=19)
+        k[0, 1, 50, 3] = float("inf")
+        y = sata.prefill(q.cuda(), k.cuda(), v.cuda(), P=4)
+        assert sata.sata_sync_status() == sata.SATA_ERANGE
+        assert not torch.isfinite(y[0, 1]).all()
+        assert torch.isfinite(y[0, 0]).all()
+        k[0, 1, 50, 3] = 0.0
+        sata.prefill(q.cuda(), k.cuda(), v.cuda(), P=4)
+        assert sata.sata_sync_status() == 0
+    finally:
+        sata.sata_set_option(sata.SATA_OPT_PREFILL_PATH, 0)
 
 
 # ------------------------------------------------------------ backward ----
