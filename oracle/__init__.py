@@ -63,6 +63,10 @@ def _load():
             lib.oracle_direct.restype = ctypes.c_int
             lib.oracle_direct.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_double,
                                           ctypes.c_longlong, _dp, _dp, _dp, _dp, _dp, _dp]
+            lib.oracle_direct_at.restype = ctypes.c_int
+            lib.oracle_direct_at.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_double,
+                                             ctypes.c_longlong, _dp, _dp, _dp, ctypes.c_longlong, ctypes.c_void_p,
+                                             _dp, _dp, _dp]
             lib.oracle_direct_grad.restype = ctypes.c_int
             lib.oracle_direct_grad.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_double,
                                                ctypes.c_longlong, _dp, _dp, _dp, _dp, _dp, _dp, _dp]
@@ -163,6 +167,25 @@ def direct(q, k, v, P: int, c: float | None = None):
     kappa = np.zeros(T)
     _check(_load().oracle_direct(dK, dV, P, c, T, _ptr(q), _ptr(k), _ptr(v), _ptr(y), _ptr(den),
                                  _ptr(kappa)), "direct")
+    return y, den, kappa
+
+
+def direct_at(q, k, v, P: int, ts, c: float | None = None):
+    """``direct`` at the token indices ``ts`` only, for one head: (y [n, d_V], den, kappa).
+
+    Each output costs O(t d), so tokens deep into a long sequence can be checked."""
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    T, dK = q.shape
+    dV = v.shape[1]
+    c = default_c(dK) if c is None else float(c)
+    idx = np.ascontiguousarray(np.asarray(ts, dtype=np.int64))
+    n = idx.shape[0]
+    y = np.zeros((n, dV))
+    den = np.zeros(n)
+    kappa = np.zeros(n)
+    _check(_load().oracle_direct_at(dK, dV, P, c, T, _ptr(q), _ptr(k), _ptr(v), n,
+                                    idx.ctypes.data_as(ctypes.c_void_p), _ptr(y), _ptr(den), _ptr(kappa)),
+           "direct_at")
     return y, den, kappa
 
 

@@ -243,6 +243,50 @@ int oracle_direct(int dK, int dV, int P, double c, long long T,
 }
 
 /*
+ * The masked direct form above at a few chosen tokens only: for each of the n
+ * token indices ts[i] (0 <= ts[i] < T), y[i] = sum_{s<=t} w_ts v_s / sum_{s<=t} w_ts
+ * with the same weights w_ts = sum_{p<P} (q_t . k_s / c)^p / p!, summed in the
+ * same order as oracle_direct; den[i] and kappa[i] as there (either may be NULL).
+ * Each output costs O(t (d_K + d_V)), so outputs deep into a long sequence can be
+ * checked without the whole O(T^2) table.  y is [n][d_V].
+ */
+int oracle_direct_at(int dK, int dV, int P, double c, long long T,
+                     const double *q, const double *k, const double *v,
+                     long long n, const long long *ts, double *y, double *den, double *kappa) {
+    if (dK < 1 || dV < 1 || P < 1 || T < 0 || n < 0) return -1;
+    if (n > 0 && (!q || !k || !v || !ts || !y)) return -1;
+    double *num = (double *)malloc(sizeof(double) * dV);
+    if (!num) return -2;
+    for (long long i = 0; i < n; ++i) {
+        const long long t = ts[i];
+        if (t < 0 || t >= T) {
+            free(num);
+            return -1;
+        }
+        double dn = 0.0, absw = 0.0;
+        for (int j = 0; j < dV; ++j) num[j] = 0.0;
+        for (long long s = 0; s <= t; ++s) {
+            double x = 0.0;
+            for (int a = 0; a < dK; ++a) x += q[t * dK + a] * k[s * dK + a];
+            x /= c;
+            double w = 0.0, term = 1.0;
+            for (int p = 0; p < P; ++p) {
+                w += term;
+                term = term * x / (double)(p + 1);
+            }
+            dn += w;
+            absw += fabs(w);
+            for (int j = 0; j < dV; ++j) num[j] += w * v[s * dV + j];
+        }
+        for (int j = 0; j < dV; ++j) y[i * dV + j] = num[j] / dn;
+        if (den) den[i] = dn;
+        if (kappa) kappa[i] = absw / fabs(dn);
+    }
+    free(num);
+    return 0;
+}
+
+/*
  * Gradient of the loss L = sum_t dy_t . y_t with respect to q, k and v, for the
  * masked direct form above.  The pages define no backward pass; they expect the
  * attention to be trained inside ordinary Transformer pipelines ([CC-TAYLOR]

@@ -72,11 +72,16 @@ namespace sata {
 namespace {
 
 constexpr int kL = 128;                    // chunk length (tokens)
+// Readout sums of a (head, chunk): [DQ][128 tokens][4] fp32, DQ = ceil((d_V + 1) / 4) quads of
+// columns (V columns, then the Z column, zero padding): a thread adds its token's quad with
+// one vector reduction, and 32 consecutive tokens cover 512 contiguous bytes.
+__host__ __device__ constexpr int sum_quads(int DV) { return (DV + 1 + 3) / 4; }
 constexpr int kNMax = 208;                 // widest unit: TMEM state + readout + P2(q) <= 512 columns
 constexpr int kScanWarps = 13;          // at most 4 warps per SM sub-partition: 128 registers each
 constexpr int kScanThreads = kScanWarps * 32;
-// warp roles: MMA issuer (one thread, both contractions), k side (4, thread = token), q side (4,
-// thread = token = TMEM lane), state conversion (4, thread = pair row = TMEM lane)
+// warp roles: MMA issuer (one thread, both contractions, in chunk order), k side (4, thread =
+// token), q side (4, thread = token = TMEM lane), state conversion (4, thread = pair row = TMEM
+// lane)
 constexpr int kWarpI = 0, kWarpK0 = 1, kWarpQ0 = 5, kWarpC0 = 9;
 constexpr int64_t kDefaultWaitNs = 2000000000LL;   // 2 s per wait
 constexpr size_t kPartialBudget = size_t(4) << 30;  // fixed-order mode: unit partials per segment
@@ -91,8 +96,9 @@ struct Cfg {
     static constexpr int XW = DK / 2 + 1;        // half2 words of a token row x~ = (x, 1)
     static constexpr int NPAIR = (D + 1) * (D + 2) / 2;
     static constexpr int NPT = (NPAIR + 127) / 128;
-    // TMEM columns: state, readout accumulator, P2(q) operand (two fp16 per column)
-    static constexpr int COL_S = 0, COL_R = NMAX, COL_AQ = 2 * NMAX;
+    // TMEM columns: state, readout accumulator (32-aligned: the drain reads 32 columns at a
+    // time), P2(q) operand (two fp16 per column)
+    static constexpr int COL_S = 0, COL_R = (NMAX + 31) / 32 * 32, COL_AQ = COL_R + NMAX;
     // shared memory: P2(k) operand x2 (128-byte swizzled MN-major), W and the state operand
     // B x2 (MN-major core matrices, K groups of 8 rows LBO bytes apart)
     static constexpr int AK_BYTES = 128 * 128 * 2;
@@ -201,6 +207,17 @@ __device__ __forceinline__ void tc_ld16(uint32_t taddr, uint32_t *r) {
         "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
         : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
           "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr)
+        : "memory");
+}
+__device__ __forceinline__ void tc_ld32(uint32_t taddr, uint32_t *r) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
         : "r"(taddr)
         : "memory");
 }
@@ -523,23 +540,15 @@ __global__ void tc_state_stats_kernel(const float *__restrict__ S, const float *
 
 // ----------------------------------------------------------------- scan ----
 
-// q side: P2(q) (64 registers) of a token row already in registers, and q~_l of each slot.
-template <int DK, int DV>
-__device__ __forceinline__ void q_prep(const ScanParams &p, int64_t bh, int ktile, const int *sl, int cl, int t,
-                                       const uint32_t (&x)[Cfg<DK, DV>::XW], uint32_t (&pq)[64],
-                                       float (&ql)[Cfg<DK, DV>::NL]) {
-    using C = Cfg<DK, DV>;
+// Token row t of chunk cl into registers, with x~_l of each slot (half2 broadcasts).
+template <int DK, int NX, int NL>
+__device__ __forceinline__ void fetch_row(const __half *x16, const ScanParams &p, int64_t bh, const int *sl, int cl,
+                                          int t, uint32_t (&x)[NX], uint32_t (&xl)[NL]) {
     const bool valid = (int64_t)(p.c0 + cl) * kL + t < p.N;
-    const uint4 *cr = chunk_rows<DK>(p.q16, bh, p.nch, p.c0 + cl);
-    p2q_dispatch<DK, 0, C::NPT>(ktile, x, pq);
+    const uint4 *cr = chunk_rows<DK>(x16, bh, p.nch, p.c0 + cl);
+    load_row<DK>(cr, t, valid, x);
 #pragma unroll
-    for (int s = 0; s < C::NL; ++s) ql[s] = h_lo(row_half2(cr, t, sl[s], DK, valid));
-}
-// q side: prefetch token row t of chunk cl into registers.
-template <int DK, int NX>
-__device__ __forceinline__ void q_row(const ScanParams &p, int64_t bh, int cl, int t, uint32_t (&x)[NX]) {
-    const bool valid = (int64_t)(p.c0 + cl) * kL + t < p.N;
-    load_row<DK>(chunk_rows<DK>(p.q16, bh, p.nch, p.c0 + cl), t, valid, x);
+    for (int s = 0; s < NL; ++s) xl[s] = row_half2(cr, t, sl[s], DK, valid);
 }
 
 // q side: readout R of chunk cl (TMEM, this warp's lanes), combined over the slots with
@@ -555,7 +564,8 @@ __device__ __forceinline__ void q_drain(const ScanParams &p, int64_t bh, int64_t
     const int sg = state_sigma(cl, e_ms, E, p.P);
     const float upv = pow2f_sat(sg + ev), upz = pow2f_sat(sg);
     const bool valid = (int64_t)(p.c0 + cl) * kL + t < p.N;
-    float *dst = p.part + ((part_base + cl) * (DV + 1)) * kL + t;
+    constexpr int DQ = sum_quads(DV);
+    float4 *dst = reinterpret_cast<float4 *>(p.part) + (part_base + cl) * DQ * kL + t;
     float den = 0.f;
     {
         uint32_t rz[16];
@@ -565,40 +575,44 @@ __device__ __forceinline__ void q_drain(const ScanParams &p, int64_t bh, int64_t
         for (int s = 0; s < NL; ++s)
             if (s < nl) den = fmaf(qv[s], __uint_as_float(rz[s]), den);
     }
-    // one 16-column group at a time: combine the slots, then add (or store) the group
+    // 32 columns at a time (16 when d_V = 16): one load per slot, combined, then the columns'
+    // quads added (or stored)
+    constexpr int GW = DV >= 32 ? 32 : 16;
 #pragma unroll 1
-    for (int g = 0; g < DV / 16; ++g) {
-        float acc[16];
+    for (int g = 0; g < DV / GW; ++g) {
+        float acc[GW];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) acc[i] = 0.f;
+        for (int i = 0; i < GW; ++i) acc[i] = 0.f;
 #pragma unroll
         for (int s = 0; s < NL; ++s) {
             if (s < nl) {
-                uint32_t r0[16];
-                tc_ld16(tm + C::COL_R + s * DV + 16 * g, r0);
+                uint32_t ra[GW];
+                if constexpr (GW == 32) tc_ld32(tm + C::COL_R + s * DV + GW * g, ra);
+                else tc_ld16(tm + C::COL_R + s * DV + GW * g, ra);
                 tc_wait_ld();
 #pragma unroll
-                for (int i = 0; i < 16; ++i) acc[i] = fmaf(qv[s], __uint_as_float(r0[i]), acc[i]);
+                for (int i = 0; i < GW; ++i) acc[i] = fmaf(qv[s], __uint_as_float(ra[i]), acc[i]);
             }
         }
-        if (g == DV / 16 - 1) {   // every column read: the next readout may overwrite R
+        if (g == DV / GW - 1) {   // every column read: the next readout may overwrite R
             tc_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(rf_bar);
         }
         if (valid) {
-            if (p.red_atomic) {
 #pragma unroll
-                for (int i = 0; i < 16; ++i) atomicAdd(dst + (16 * g + i) * kL, acc[i] * upv);
-            } else {
-#pragma unroll
-                for (int i = 0; i < 16; ++i) dst[(16 * g + i) * kL] = acc[i] * upv;
+            for (int i4 = 0; i4 < GW / 4; ++i4) {
+                const float4 val = make_float4(acc[4 * i4] * upv, acc[4 * i4 + 1] * upv, acc[4 * i4 + 2] * upv,
+                                               acc[4 * i4 + 3] * upv);
+                if (p.red_atomic) atomicAdd(dst + (GW / 4 * g + i4) * kL, val);
+                else dst[(GW / 4 * g + i4) * kL] = val;
             }
         }
     }
-    if (valid) {
-        if (p.red_atomic) atomicAdd(dst + DV * kL, den * upz);
-        else dst[DV * kL] = den * upz;
+    if (valid) {   // the Z column opens the last quad (its other columns are padding)
+        const float4 val = make_float4(den * upz, 0.f, 0.f, 0.f);
+        if (p.red_atomic) atomicAdd(dst + (DV / 4) * kL, val);
+        else dst[(DV / 4) * kL] = val;
     }
 }
 
@@ -668,6 +682,7 @@ __global__ void __launch_bounds__(kScanThreads, 1) tc_scan_kernel(const ScanPara
             if (i == C::B_AKF || i == C::B_SR || i == C::B_BSF || i == C::B_BSF + 1 || i == C::B_AQF ||
                 i == C::B_RF)
                 cnt = 4;
+
             mbar_init(BAR(i), cnt);
         }
         *abort_flag = 0;
@@ -731,22 +746,18 @@ __global__ void __launch_bounds__(kScanThreads, 1) tc_scan_kernel(const ScanPara
         // Per chunk: P2(k) from the prefetched k row once its buffer is free, then the v row is
         // requested and lands while the update of the previous chunk completes, then W, then
         // the next chunk's k row is requested.
-        uint32_t x[C::XW];
-        if (p.nc > 0) load_row<DK>(chunk_rows<DK>(p.k16, bh, p.nch, p.c0), t, (int64_t)p.c0 * kL + t < p.N, x);
+        uint32_t x[C::XW], kl[NL];   // this chunk's k row and k~_l (half2 broadcasts), prefetched
+        if (p.nc > 0) fetch_row<DK>(p.k16, p, bh, sl, 0, t, x, kl);
         bool ok = true;
         for (int cl = 0; cl < p.nc && ok; ++cl) {
-            const bool valid = (int64_t)(p.c0 + cl) * kL + t < p.N;
-            const uint4 *kcr = chunk_rows<DK>(p.k16, bh, p.nch, p.c0 + cl);
             const int b = cl & 1;
             // P2(k) into its double buffer once the update of chunk cl-2 has read it
             if (cl >= 2 && !(ok = W.wait(BAR(C::B_AKE + b), ((cl >> 1) - 1) & 1))) break;
             p2k_dispatch<DK>(ktile, x, smem + C::OFF_AK + b * C::AK_BYTES, t,
                              std::make_integer_sequence<int, C::NPT>{});
-            uint32_t kl[NL];   // k~_l of each slot, half2 broadcast; 0 past the sequence end
-#pragma unroll
-            for (int s = 0; s < NL; ++s) kl[s] = row_half2(kcr, t, sl[s], DK, valid);
             uint4 vr[DV / 8];
             {
+                const bool valid = (int64_t)(p.c0 + cl) * kL + t < p.N;
                 const uint4 *vcr = chunk_rows<DV>(p.v16, bh, p.nch, p.c0 + cl);
 #pragma unroll
                 for (int i = 0; i < DV / 8; ++i) vr[i] = valid ? __ldg(vcr + i * 128 + t) : make_uint4(0, 0, 0, 0);
@@ -778,9 +789,9 @@ __global__ void __launch_bounds__(kScanThreads, 1) tc_scan_kernel(const ScanPara
                 }
                 *reinterpret_cast<uint4 *>(wrow + z8 * 128) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
             }
-            if (cl + 1 < p.nc)
-                load_row<DK>(chunk_rows<DK>(p.k16, bh, p.nch, p.c0 + cl + 1), t,
-                             (int64_t)(p.c0 + cl + 1) * kL + t < p.N, x);
+            if (cl + 1 < p.nc) {
+                fetch_row<DK>(p.k16, p, bh, sl, cl + 1, t, x, kl);
+            }
             fence_proxy_async();
             __syncwarp();
             // test hook: one producer signal withheld, so the issuer's wait expires
@@ -792,14 +803,13 @@ __global__ void __launch_bounds__(kScanThreads, 1) tc_scan_kernel(const ScanPara
         const int t = quarter * 32 + lane;               // token row of the chunk = TMEM lane
         const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
         const int64_t part_base = p.red_atomic ? (int64_t)bh * p.nc : ((int64_t)bh * p.G + u) * p.nc;
-        uint32_t pq[64];
-        float ql[NL], qlp[NL];
-        uint32_t x[C::XW];   // the token row of the next chunk, prefetched
+        uint32_t pq[64], xl[NL];
+        float qlp[NL];
         bool ok = true;
         if (p.nc > 0) {
-            q_row<DK>(p, bh, 0, t, x);
-            q_prep<DK, DV>(p, bh, ktile, sl, 0, t, x, pq, ql);
-            if (p.nc > 1) q_row<DK>(p, bh, 1, t, x);
+            uint32_t x[C::XW];
+            fetch_row<DK>(p.q16, p, bh, sl, 0, t, x, xl);
+            p2q_dispatch<DK, 0, C::NPT>(ktile, x, pq);
         }
         for (int cl = 0; cl < p.nc; ++cl) {
             if (cl > 0 && !(ok = W.wait(BAR(C::B_RD), (cl - 1) & 1))) break;
@@ -813,11 +823,14 @@ __global__ void __launch_bounds__(kScanThreads, 1) tc_scan_kernel(const ScanPara
             if (cl > 0) q_drain<DK, DV>(p, bh, part_base, nl, e_ms, E, he.ev, cl - 1, t, lane, tmem + lane_off,
                                         BAR(C::B_RF), qlp);
 #pragma unroll
-            for (int s = 0; s < NL; ++s) qlp[s] = ql[s];
-            // unconditional, so that pq is provably dead during the drain above (the last
-            // iteration computes an unused operand)
-            q_prep<DK, DV>(p, bh, ktile, sl, cl + 1 < p.nc ? cl + 1 : cl, t, x, pq, ql);
-            if (cl + 2 < p.nc) q_row<DK>(p, bh, cl + 2, t, x);
+            for (int s = 0; s < NL; ++s) qlp[s] = h_lo(xl[s]);
+            {   // the next chunk's operand (its row is read after the drain, which needs the
+                // registers; the load overlaps the readout now running).  Unconditional, so that
+                // pq is provably dead during the drain (the last iteration builds an unused one).
+                uint32_t x[C::XW];
+                fetch_row<DK>(p.q16, p, bh, sl, cl + 1 < p.nc ? cl + 1 : cl, t, x, xl);
+                p2q_dispatch<DK, 0, C::NPT>(ktile, x, pq);
+            }
         }
         if (ok && p.nc > 0 && W.wait(BAR(C::B_RD), (p.nc - 1) & 1))
             q_drain<DK, DV>(p, bh, part_base, nl, e_ms, E, he.ev, p.nc - 1, t, lane, tmem + lane_off, BAR(C::B_RF), qlp);
@@ -963,7 +976,7 @@ __global__ void __launch_bounds__(kScanThreads, 1) tc_scan_kernel(const ScanPara
 template <int DV>
 __global__ void __launch_bounds__(256)
 tc_reduce_kernel(const float4 *__restrict__ part, float4 *__restrict__ red, int BH, int G, int nc) {
-    const int64_t per_head = (int64_t)nc * (DV + 1) * (kL / 4);
+    const int64_t per_head = (int64_t)nc * sum_quads(DV) * kL;
     const int64_t total = (int64_t)BH * per_head;
     for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < total; e += (int64_t)gridDim.x * blockDim.x) {
         const int64_t bh = e / per_head, rem = e % per_head;
@@ -1166,14 +1179,14 @@ tc_finish_kernel(const __half *__restrict__ q16, const __half *__restrict__ k16,
     float *stg = reinterpret_cast<float *>(sm);
     if (ok) {
         const float upz = pow2f_sat(e_t), upv = pow2f_sat(e_t + he.ev);
-        const float *rp = red + ((bh * nc + cl) * (DV + 1)) * kL + t;
+        const float4 *rp = reinterpret_cast<const float4 *>(red) + (bh * nc + cl) * sum_quads(DV) * kL + t;
         float inv;
         bool finite = true;
         {   // denominator: column DV
             uint32_t rr[16];
             tc_ld16(tmem + 128 + lane_off + DV, rr);
             tc_wait_ld();
-            const float den = fmaf(__uint_as_float(rr[0]), upz, rp[DV * kL]);
+            const float den = fmaf(__uint_as_float(rr[0]), upz, rp[(DV / 4) * kL].x);
             inv = 1.f / den;
             finite = fabsf(inv) <= FLT_MAX;
             if (den_out && t < nt) den_out[bh * N + t0 + t] = den;   // kept for the backward pass
@@ -1185,11 +1198,12 @@ tc_finish_kernel(const __half *__restrict__ q16, const __half *__restrict__ k16,
             tc_wait_ld();
 #pragma unroll
             for (int i4 = 0; i4 < 4; ++i4) {
+                const float4 sv = rp[(c16 * 4 + i4) * kL];
+                const float sq[4] = {sv.x, sv.y, sv.z, sv.w};
                 float o[4];
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
-                    const int j = c16 * 16 + 4 * i4 + i;
-                    o[i] = fmaf(__uint_as_float(rr[4 * i4 + i]), upv, rp[j * kL]) * inv;
+                    o[i] = fmaf(__uint_as_float(rr[4 * i4 + i]), upv, sq[i]) * inv;
                     finite = finite && fabsf(o[i]) <= FLT_MAX;
                 }
                 *reinterpret_cast<float4 *>(stg + t * F::STG + c16 * 16 + 4 * i4) = make_float4(o[0], o[1], o[2], o[3]);
@@ -1355,7 +1369,7 @@ bool make_plan(int BH, int64_t N, int64_t F, int P, bool need_state, int min_seg
     pl.nchunks = (int)((N + kL - 1) / kL);
     int64_t nseg = min_segments;
     if (deterministic) {
-        const size_t per_chunk = (size_t)BH * pl.G * (DV + 1) * kL * sizeof(float);
+        const size_t per_chunk = (size_t)BH * pl.G * sum_quads(DV) * kL * 16;
         int64_t seg = (int64_t)(kPartialBudget / per_chunk);
         if (seg < 1) seg = 1;
         const int64_t need = (pl.nchunks + seg - 1) / seg;
@@ -1371,9 +1385,9 @@ bool make_plan(int BH, int64_t N, int64_t F, int P, bool need_state, int min_seg
     pl.off_k16 = pl.off_q16 + align256(rows * DK * 2);
     pl.off_v16 = pl.off_k16 + align256(rows * DK * 2);
     pl.off_red = pl.off_v16 + align256(rows * DV * 2);
-    pl.off_part = pl.off_red + align256((size_t)BH * (DV + 1) * kL * sizeof(float) * pl.nc_seg);
+    pl.off_part = pl.off_red + align256((size_t)BH * sum_quads(DV) * kL * 16 * pl.nc_seg);
     pl.off_state = pl.off_part +
-                   (deterministic ? align256((size_t)BH * pl.G * (DV + 1) * kL * sizeof(float) * pl.nc_seg) : 0);
+                   (deterministic ? align256((size_t)BH * pl.G * sum_quads(DV) * kL * 16 * pl.nc_seg) : 0);
     pl.total = pl.off_state + (need_state && pl.nseg > 1 ? align256((size_t)BH * F * (DV + 1) * sizeof(float)) : 0);
     return true;
 }
@@ -1496,7 +1510,7 @@ cudaError_t run(const DeviceBasis &basis, int BH, int64_t N, const void *q, cons
         sp.unit_fidx = (const int32_t *)(tab + up.off_fidx);
         sp.S = S;
         sp.Z = Z;
-        if (!det && (e = cudaMemsetAsync(red, 0, (size_t)BH * ncs * (DV + 1) * kL * sizeof(float), stream)) !=
+        if (!det && (e = cudaMemsetAsync(red, 0, (size_t)BH * ncs * sum_quads(DV) * kL * 16, stream)) !=
                         cudaSuccess)
             return e;
         sp.part = det ? part : red;
@@ -1520,7 +1534,7 @@ cudaError_t run(const DeviceBasis &basis, int BH, int64_t N, const void *q, cons
         launch_end(kTcScan, stream);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
         if (det) {   // the units' partials summed in a fixed order
-            const int64_t rwork = (int64_t)BH * ncs * (DV + 1) * (kL / 4);
+            const int64_t rwork = (int64_t)BH * ncs * sum_quads(DV) * kL;
             launch_begin(kTcReduce, stream);
             tc_reduce_kernel<DV><<<(int)((rwork + 255) / 256 < 148 * 32 ? (rwork + 255) / 256 : 148 * 32), 256, 0,
                                    stream>>>((const float4 *)part, (float4 *)red, BH, pl.G, ncs);

@@ -97,7 +97,13 @@ def test_size_queries(lib):
     S, Z = sata_state_bytes(1, 8, 64, 64, 4)
     assert S == 8 * 47905 * 64 * 4 and Z == 8 * 47905 * 4
     assert (S + Z) // 8 // 4 == 3113825           # (d_V + 1) binom(67, 3) per head
-    assert sata_workspace_bytes(1, 8, 65536, 64, 64, 4) > 0
+    ws = sata_workspace_bytes(1, 8, 65536, 64, 64, 4)
+    # prefill_d64 in the default mode: the prescaled fp16 rows (201 MB) and the L2-resident
+    # readout sums of one segment (143 MB); no per-unit partial buffer
+    rows = 8 * 65536 * (64 + 64 + 64) * 2
+    sums = 8 * 512 * 17 * 128 * 16
+    assert rows + sums <= ws < rows + sums + (1 << 20)
+    assert ws < 0.6e9
     from symmetric_taylor_self_b200 import sata_backward_workspace_bytes as bwb
     small, big = bwb(1, 1, 1000, 16, 16, 4), bwb(1, 1, 100000, 16, 16, 4)
     # y, den and r are kept for every token: at least (2 d_V + 2) fp32 values per token

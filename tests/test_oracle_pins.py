@@ -172,6 +172,26 @@ def test_direct_pairwise_weights_by_hand(oracle_mod):
     np.testing.assert_allclose(ys, y, rtol=1e-14)
 
 
+@pytest.mark.parametrize("dK,dV,P,T", [(2, 3, 4, 40), (8, 8, 4, 64), (3, 5, 2, 33)])
+def test_direct_at_selected_tokens(oracle_mod, dK, dV, P, T):
+    """direct_at (outputs at chosen tokens only) equals the full direct table at
+    those tokens, in any order and with repeats, and the P = 1 running mean at
+    selected tokens; an index outside [0, T) is rejected."""
+    rng = np.random.default_rng(dK * 10 + P)
+    q, k, v = _inputs(rng, T, dK, dV)
+    y, den, kappa = oracle_mod.direct(q, k, v, P)
+    ts = [T - 1, 0, T // 2, T // 2, 1]
+    ya, dena, kappaa = oracle_mod.direct_at(q, k, v, P, ts)
+    np.testing.assert_array_equal(ya, y[ts])
+    np.testing.assert_array_equal(dena, den[ts])
+    np.testing.assert_array_equal(kappaa, kappa[ts])
+    y1, _, _ = oracle_mod.direct_at(q, k, v, 1, ts)
+    want = (np.cumsum(v, axis=0) / np.arange(1, T + 1)[:, None])[ts]
+    np.testing.assert_allclose(y1, want, rtol=1e-12)
+    with pytest.raises(RuntimeError):
+        oracle_mod.direct_at(q, k, v, P, [T])
+
+
 def test_P1_is_running_mean(oracle_mod):
     rng = np.random.default_rng(1)
     q, k, v = _inputs(rng, 50, 4, 3)
