@@ -47,13 +47,14 @@ def parse():
     ap.add_argument("--impl", choices=["sata", "reference"], default="sata")
     ap.add_argument("--workload", default="prefill_d64")
     ap.add_argument("--decode-workload", default="decode_d32")
-    ap.add_argument("--decode-steps", type=int, default=256)
+    ap.add_argument("--decode-steps", type=int, default=None, help="default: all of the workload's")
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--backward-workload", default="backward_d64")
     ap.add_argument("--no-backward", action="store_true")
     ap.add_argument("--only", choices=["all", "prefill", "decode", "backward"], default="all",
                     help="run one part only (reduced workloads for profiler captures)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extra", action="store_true", help="skip the other prefill workloads")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--path", choices=["auto", "cuda_core", "tensor_core"], default="auto")
     ap.add_argument("--seq-split", action="store_true",
@@ -173,7 +174,8 @@ def flops_per_token(d_K, d_V, P):
     return num * F // (d_K + 1)
 
 
-KERNEL_SOURCES = {"tc_scan": "prefill_tc.cu", "simt_scan": "prefill_simt.cu", "decode_stream": "decode.cu"}
+# prefill workloads measured beside the headline one (lines under "extra")
+EXTRA_WORKLOADS = ("tiny_d8", "prefill_d16", "prefill_d32", "prefill_d128", "prefill_d64_dv32", "prefill_d16_p6")
 
 
 # ---------------------------------------------------------- distributed ----
@@ -360,33 +362,8 @@ def main():
     value = job_throughput(tokens_per_step, args.steps, world, ms)
     launches = sum(n for n, _ in stats.values())
 
-    # roofline of the dominant kernel
-    dom = max(stats, key=lambda n: stats[n][1]) if stats else None
-    flops_tok_head = flops_per_token(w.d_K, w.d_V, w.P)
-    alg_flops_step = flops_tok_head * w.B * w.H * w.N
-    roof = None
-    if dom:
-        n_l, ms_l = stats[dom]
-        per_launch_ms = ms_l / n_l
-        flops_per_launch = alg_flops_step * args.steps / n_l
-        achieved = flops_per_launch / (per_launch_ms / 1000.0) / 1e12
-        if dom.startswith("tc"):
-            roof = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                    "peak_kind": f"{peaks_src} bf16 dense burst (fp16 operands run at the bf16 rate)"}
-        else:
-            sm_ghz = (clocks.get("sm_max_mhz") or 1965.0) / 1000.0
-            alu_peak = NUM_SMS * FP32_LANES_PER_SM * 2 * sm_ghz / 1000.0
-            roof = {"bound": "alu", "achieved": achieved, "peak": alu_peak, "unit": "TFLOP/s",
-                    "peak_kind": "fp32 FMA: 148 SMs x 128 lanes x 2 FLOP x max SM clock"}
-        roof["frac"] = roof["achieved"] / roof["peak"]
-        roof["kernel"] = dom
-        roof["launches_per_step"] = n_l / args.steps
-        roof["ms_per_launch"] = per_launch_ms
-        roof["algorithmic_flops_per_launch"] = flops_per_launch
-        tr = ncu_traffic(dom)
-        roof["traffic"] = tr
-        if tr is None:
-            roof["traffic_note"] = "no ncu capture of the current kernel source"
+    roof = prefill_roofline(stats, w, args.steps, peaks, peaks_src, clocks)
+    dom = roof["kernel"] if roof else None
 
     # ---------------- e2e through host buffers ----------------
     e2e = None
@@ -414,6 +391,14 @@ def main():
     if not args.no_backward:
         bwd = bench_backward(torch, sata, wl, args, world, dev, stream, peaks, peaks_src)
 
+    # ---------------- the other prefill workloads ----------------
+    extra = []
+    for name in ([] if args.no_extra else EXTRA_WORKLOADS):
+        e = bench_extra(torch, sata, wl, name, args, world, dev, stream, peaks, peaks_src)
+        if rank == 0 and world == 1 and not args.no_cpu_baseline:
+            e["cpu_baseline"] = cpu_oracle_rate(wl.WORKLOADS[name], min(args.cpu_seconds, 4.0))
+        extra.append(e)
+
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True,
@@ -425,7 +410,7 @@ def main():
                    "l2": f"inputs {in_bytes / 1e6:.0f} MB + output {out_bytes / 1e6:.0f} MB per step > 126 MB L2",
                    "path": args.path},
         "roofline": roof, "gpu_launches": launches, "clocks": clocks, "e2e": e2e, "decode": dec,
-        "backward": bwd,
+        "backward": bwd, "extra": extra,
         "kernel_ms": {k_: {"launches": n, "ms": t} for k_, (n, t) in stats.items()},
         "peaks_source": peaks_src,
     }
@@ -437,6 +422,74 @@ def main():
         import torch.distributed as dist
         dist.destroy_process_group()
     return 0
+
+
+def prefill_roofline(stats, w, steps, peaks, peaks_src, clocks):
+    """Roofline of the prefill's dominant kernel: algorithmic FLOPs of the
+    workload per launch over its mean CUDA-event duration."""
+    if not stats:
+        return None
+    dom = max(stats, key=lambda n: stats[n][1])
+    n_l, ms_l = stats[dom]
+    per_launch_ms = ms_l / n_l
+    flops_per_launch = flops_per_token(w.d_K, w.d_V, w.P) * w.B * w.H * w.N * steps / n_l
+    achieved = flops_per_launch / (per_launch_ms / 1000.0) / 1e12
+    if dom.startswith("tc"):
+        roof = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                "peak_kind": f"{peaks_src} bf16 dense burst (fp16 operands run at the bf16 rate)"}
+    else:
+        sm_ghz = ((clocks or {}).get("sm_max_mhz") or 1965.0) / 1000.0
+        alu_peak = NUM_SMS * FP32_LANES_PER_SM * 2 * sm_ghz / 1000.0
+        roof = {"bound": "alu", "achieved": achieved, "peak": alu_peak, "unit": "TFLOP/s",
+                "peak_kind": "fp32 FMA: 148 SMs x 128 lanes x 2 FLOP x max SM clock"}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    roof["kernel"] = dom
+    roof["launches_per_step"] = n_l / steps
+    roof["ms_per_launch"] = per_launch_ms
+    roof["algorithmic_flops_per_launch"] = flops_per_launch
+    tr = ncu_traffic(dom)
+    roof["traffic"] = tr
+    if tr is None:
+        roof["traffic_note"] = "no ncu capture of the current kernel source"
+    return roof
+
+
+def bench_extra(torch, sata, wl, name, args, world, dev, stream, peaks, peaks_src):
+    """One more prefill workload, each timed step preceded (outside its events)
+    by a 256 MB write that flushes L2, since some of these inputs fit in L2."""
+    w = wl.WORKLOADS[name]
+    (q, k, v), _ = wl.make_inputs(w)
+    qd, kd, vd = q.to(dev), k.to(dev), v.to(dev)
+    out = torch.empty((w.B, w.H, w.N, w.d_V), dtype=torch.float32, device=dev)
+    flush = torch.empty(64 << 20, dtype=torch.float32, device=dev)
+
+    def step():
+        sata.sata_prefill_ex(qd, kd, vd, out, w.B, w.H, w.N, w.d_K, w.d_V, w.P, None, None, stream)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    sata.sata_reset_kernel_stats()
+    sata.sata_set_option(sata.SATA_OPT_TIME_KERNELS, 1)
+    total = 0.0
+    for _ in range(args.steps):
+        with torch.cuda.stream(stream):
+            flush.fill_(1.0)
+        total += timed(torch, world, step, 1, 0, stream)
+    stats = sata.sata_kernel_stats()
+    sata.sata_set_option(sata.SATA_OPT_TIME_KERNELS, 0)
+    if sata.sata_sync_status(stream) != 0:
+        raise RuntimeError(f"device status after {name}")
+    roof = prefill_roofline(stats, w, args.steps, peaks, peaks_src, None)
+    line = {"metric": "SATA prefill tokens/s", "workload": f"{w.name}: B={w.B} H={w.H} N={w.N} d_K={w.d_K} "
+            f"d_V={w.d_V} P={w.P} F={w.F}", "value": job_throughput(w.B * w.N, args.steps, world, total),
+            "unit": "tokens/s", "steps": args.steps, "ms_per_step": total / args.steps,
+            "dtype": "f16" if roof and roof["kernel"].startswith("tc") else "f32",
+            "l2": "L2 flushed (256 MB write) before each timed step", "roofline": roof,
+            "gpu_launches": sum(n for n, _ in stats.values()),
+            "kernel_ms": {k_: {"launches": n, "ms": t} for k_, (n, t) in stats.items()}}
+    del qd, kd, vd, out, flush
+    return line
 
 
 def run_seq_split(torch, sata, wl, args, rank, world):
@@ -474,7 +527,7 @@ def run_seq_split(torch, sata, wl, args, rank, world):
                                       f"states all-gathered, exclusive prefix, prefill from the prefix",
                        "l2": "inputs and state exchange larger than L2 at this size"},
             "roofline": None, "e2e": None, "clocks": clocks,
-            "note": "two prefills of each rank's segment plus the state all-gather; see DESIGN"}
+            "note": "two prefills of each rank's segment plus the state all-gather"}
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -577,32 +630,34 @@ def bench_backward(torch, sata, wl, args, world, dev, stream, peaks, peaks_src):
 
 
 def bench_decode(torch, sata, wl, args, world, dev, stream, peaks, peaks_src):
+    """The decode workload as stated: the seeded per-head inputs of workloads.py,
+    an N-token prefill into the state, then every decode step timed.  Warm-up
+    steps run first on the same state, which is then rebuilt by the prefill."""
     w = wl.WORKLOADS[args.decode_workload]
-    g = torch.Generator(device=dev).manual_seed(w.seed)
-    shp = (w.B, w.H, w.N)
-    q = torch.randn(*shp, w.d_K, generator=g, device=dev).to(torch.bfloat16)
-    k = torch.randn(*shp, w.d_K, generator=g, device=dev).to(torch.bfloat16)
-    v = torch.randn(*shp, w.d_V, generator=g, device=dev).to(torch.bfloat16)
-    D = min(args.decode_steps, w.steps)
-    qs = torch.randn(D, w.B, w.H, w.d_K, generator=g, device=dev).to(torch.bfloat16)
-    ks = torch.randn(D, w.B, w.H, w.d_K, generator=g, device=dev).to(torch.bfloat16)
-    vs = torch.randn(D, w.B, w.H, w.d_V, generator=g, device=dev).to(torch.bfloat16)
+    (q, k, v), (qs, ks, vs) = wl.make_inputs(w)
+    D = w.steps if args.decode_steps is None else min(args.decode_steps, w.steps)
+    q, k, v = q.to(dev), k.to(dev), v.to(dev)
+    qs, ks, vs = qs[:D].to(dev), ks[:D].to(dev), vs[:D].to(dev)
     st = sata.State(w.B, w.H, w.d_K, w.d_V, w.P, device=dev, stream=stream)
-    with torch.cuda.stream(stream):
-        sata.prefill(q, k, v, P=w.P, state=st, stream=stream)
-    del q, k, v
     outs = torch.empty((D, w.B, w.H, w.d_V), dtype=torch.float32, device=dev)
+
+    def rebuild():
+        sata.sata_state_init(st.st, w.B, w.H, w.d_K, w.d_V, w.P, st.S, st.Z, stream)
+        with torch.cuda.stream(stream):
+            sata.prefill(q, k, v, P=w.P, state=st, stream=stream)
+
+    rebuild()
+    for i in range(min(8, D)):
+        sata.sata_decode_step(st.st, qs[i], ks[i], vs[i], outs[i])
+    rebuild()
     torch.cuda.synchronize()
     it = [0]
 
     def step():
-        i = it[0] % D
+        i = it[0]
         it[0] += 1
         sata.sata_decode_step(st.st, qs[i], ks[i], vs[i], outs[i])
 
-    for _ in range(8):
-        step()
-    torch.cuda.synchronize()
     sata.sata_reset_kernel_stats()
     sata.sata_set_option(sata.SATA_OPT_TIME_KERNELS, 1)
     ms = timed(torch, world, step, D, 0, stream)
@@ -626,7 +681,7 @@ def bench_decode(torch, sata, wl, args, world, dev, stream, peaks, peaks_src):
     return {"metric": "SATA decode tokens/s", "value": value, "unit": "tokens/s", "steps": D,
             "ms_per_step": ms / D,
             "workload": f"{w.name}: B={w.B} H={w.H} d_K={w.d_K} d_V={w.d_V} P={w.P} F={F}, state from a "
-                        f"{w.N}-token prefill; inputs drawn on the GPU (torch generator, N(0,1))",
+                        f"{w.N}-token prefill, then steps 1..{D} timed; seeded per-head N(0,1) bf16 inputs",
             "l2": f"state {state_bytes / 2 / 1e9:.2f} GB > 126 MB L2", "roofline": roof,
             "gpu_launches": sum(n for n, _ in stats.values()),
             "kernel_ms": {k_: {"launches": n, "ms": t} for k_, (n, t) in stats.items()}}

@@ -40,13 +40,19 @@
  *     (P is a tunable hyperparameter: [CC-TAYLOR] "Precision and efficiency
  *     trade-off" (精度与效率的权衡); [CC-HW] "Taylor-expansion trade-off between
  *     precision and efficiency" (精度与效率的泰勒展开权衡) weighs P = 8).  The
- *     tensor-core prefill serves d_K = d_V in
- *     {16, 32, 64} with P <= 4; every other supported shape runs on the CUDA-core
- *     prefill (fp32).  sata_decode_step_static takes P <= 4.  Other values return
- *     SATA_EUNSUPPORTED.  There is no CPU fallback.
+ *     tensor-core prefill serves P <= 4 with (d_K, d_V) one of (16|32, 16|32|64),
+ *     (64, 16|32|64|128) and (128, 64|128); every other supported shape runs on
+ *     the CUDA-core prefill (fp32).  sata_decode_step_static takes P <= 4.  Other
+ *     values return SATA_EUNSUPPORTED.  There is no CPU fallback.
+ *   - The tensor-core prefill scales each head's rows by powers of two before its
+ *     fp16 operands are formed (exact), so every finite bf16 input is in range;
+ *     only a non-finite input, or an output beyond the fp32 range, sets the
+ *     range flag (SATA_ERANGE at the next sata_sync_status).
  *   - The library-owned workspaces are shared by all calls on a device: calls
  *     that may overlap on different streams must pass their own workspace
- *     (sata_prefill_ex) or be ordered by the caller.
+ *     (sata_prefill_ex) or be ordered by the caller.  That includes calls made
+ *     from different host threads: the library serialises the sizing and
+ *     allocation of a workspace, not the kernels that use it.
  *   - The first call for a given (device, d_K, P) uploads the basis tables with
  *     synchronous copies; make it before capturing a CUDA graph.
  */
@@ -73,7 +79,7 @@ enum sata_status {
     SATA_ECUDA = -3,         /* CUDA runtime or launch error; see sata_last_cuda_error() */
     SATA_ETIMEOUT = -4,      /* a bounded device-side wait expired (reported at sync) */
     SATA_ENOMEM = -5,        /* internal workspace allocation failed, or too small */
-    SATA_ERANGE = -6,        /* inputs exceed the prefill's fp16 operand range (at sync) */
+    SATA_ERANGE = -6,        /* tensor-core prefill: a non-finite input or output (at sync) */
     SATA_EALIGN = -7         /* a device pointer is not 16-byte aligned */
 };
 
@@ -129,7 +135,9 @@ SATA_API void sata_shutdown(void);
 SATA_API int sata_state_bytes(int B, int H, int d_K, int d_V, int P, size_t *S_bytes, size_t *Z_bytes);
 
 /* Fill *st for caller-owned device buffers S, Z (sizes from sata_state_bytes)
- * and zero them on `stream` (an empty context).  tokens = 0. */
+ * and zero them on `stream`: the empty context, Z_0 = 0 and S_0 = 0, from which
+ * the recurrence of [CC-TAYLOR] "Feature maps and linear attention"
+ * (特征映射与线性注意力) accumulates phi(k_t) and phi(k_t) v_t^T.  tokens = 0. */
 SATA_API int sata_state_init(sata_state *st, int B, int H, int d_K, int d_V, int P,
                     float *S, float *Z, void *stream);
 
@@ -254,11 +262,15 @@ SATA_API int sata_decode_step(sata_state *st, const void *q, const void *k, cons
  * state, inputs and outputs, as above.  Its partial sums live in a 4 MiB static
  * device array compiled into the library, and it derives the basis
  * arithmetically instead of from tables.
- *   Limit: B*H*ceil(F/1024)*(d_V+1) <= 1,048,576 fp32 values (about 1500 heads
- *   at d_K = d_V = 32).  Beyond that it returns SATA_ENOMEM without launching.
- *   The first call on each device looks up the array's device address (once);
- *   make it before any stream capture.  All calls share the array: calls that
- *   overlap on the GPU race.  Nothing in it needs clearing between calls.
+ *   Limit: B*H*ceil(F/1024)*(d_V+1) <= 1,048,576 fp32 values: about 4500 heads
+ *   at d_K = d_V = 32 (7 x 33 values a head), about 340 at d_K = d_V = 64
+ *   (47 x 65).  Beyond that it returns SATA_ENOMEM without launching.
+ *   The first call in each device context looks up the array's device address
+ *   (a context that replaces it, after cudaDeviceReset, looks it up again);
+ *   make that call before any stream capture.  All calls share the array, from
+ *   every host thread: calls that overlap on the GPU race.  Nothing in it needs
+ *   clearing between calls.  Same kernels as sata_decode_step, so the two give
+ *   the same result.
  * Returns SATA_OK or a negative status as sata_decode_step; st->tokens += 1.
  */
 SATA_API int sata_decode_step_static(sata_state *st, const void *q, const void *k, const void *v, float *out);

@@ -22,7 +22,7 @@
 //   dq_t += dx_ts k_s / c,  dk_s += dx_ts q_t / c,  dv_s += w_ts g_t.
 //
 // Kernels, in stream order:
-//   forward (prefill_simt.cu) -> y and den;  bwd_r -> r;
+//   forward on the prefill's own path (tensor-core or CUDA-core) -> y and den;  bwd_r -> r;
 //   bwd_q_scan: per feature tile, forward over the chunks with S: dq partials;
 //   bwd_finish<dq>: sum the tiles' partials, add the intra-chunk part;
 //   bwd_kv_scan: per feature tile, backward over the chunks with G: dk, dv partials;

@@ -262,7 +262,7 @@ const char *sata_status_string(int status) {
         case SATA_ECUDA: return "SATA_ECUDA: CUDA runtime or launch error";
         case SATA_ETIMEOUT: return "SATA_ETIMEOUT: a bounded device-side wait expired";
         case SATA_ENOMEM: return "SATA_ENOMEM: workspace allocation failed or too small";
-        case SATA_ERANGE: return "SATA_ERANGE: inputs outside the prefill operand range";
+        case SATA_ERANGE: return "SATA_ERANGE: a non-finite input or output in the tensor-core prefill";
         case SATA_EALIGN: return "SATA_EALIGN: device pointer not 16-byte aligned";
         default: return "unknown sata status";
     }

@@ -17,6 +17,8 @@ Recipe (one per (b, h) head, so any head can be regenerated alone):
 from __future__ import annotations
 
 import math
+import os
+from concurrent.futures import ThreadPoolExecutor
 from dataclasses import dataclass, field
 
 import torch
@@ -54,6 +56,14 @@ WORKLOADS = {
                             oracle_heads=((0, 0),), oracle_tokens=2048),
     "decode_d32": Workload("decode_d32", B=64, H=32, N=8192, d_K=32, d_V=32, P=4, seed=4,
                            steps=1024, oracle_heads=((0, 0), (63, 31), (17, 5), (40, 22))),
+    # other head sizes and degrees: d = 128 (the state size worked out on the
+    # "Fixed-size hidden state" page), d_K != d_V, and P = 6
+    "prefill_d128": Workload("prefill_d128", B=1, H=8, N=16384, d_K=128, d_V=128, P=4, seed=7,
+                             oracle_heads=((0, 0),), oracle_tokens=256),
+    "prefill_d64_dv32": Workload("prefill_d64_dv32", B=1, H=8, N=32768, d_K=64, d_V=32, P=4, seed=8,
+                                 oracle_heads=((0, 0),), oracle_tokens=1024),
+    "prefill_d16_p6": Workload("prefill_d16_p6", B=1, H=8, N=4096, d_K=16, d_V=16, P=6, seed=9,
+                               oracle_heads=((0, 0),), oracle_tokens=1024),
     # backward pass of the prefill (gradients of q, k, v): the prefill_d64 head
     # shape over 4096 tokens; the upstream gradient dy is N(0, 1) (cotangent())
     "backward_d64": Workload("backward_d64", B=1, H=8, N=4096, d_K=64, d_V=64, P=4, seed=5,
@@ -92,9 +102,14 @@ def make_inputs(w: Workload, dtype=torch.bfloat16):
     q = torch.empty(w.B, w.H, T, w.d_K, dtype=dtype)
     k = torch.empty(w.B, w.H, T, w.d_K, dtype=dtype)
     v = torch.empty(w.B, w.H, T, w.d_V, dtype=dtype)
-    for b in range(w.B):
-        for h in range(w.H):
-            q[b, h], k[b, h], v[b, h] = head_inputs(w, b, h, dtype)
+
+    def fill(bh):
+        b, h = divmod(bh, w.H)
+        q[b, h], k[b, h], v[b, h] = head_inputs(w, b, h, dtype)
+
+    # heads are independent draws (one generator each): fill them on host threads
+    with ThreadPoolExecutor(max_workers=min(16, len(os.sched_getaffinity(0)))) as ex:
+        list(ex.map(fill, range(w.B * w.H)))
     pre = (q[:, :, :w.N].contiguous(), k[:, :, :w.N].contiguous(), v[:, :, :w.N].contiguous())
     dec = tuple(x[:, :, w.N:].permute(2, 0, 1, 3).contiguous() for x in (q, k, v))
     return pre, dec

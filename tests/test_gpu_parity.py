@@ -157,6 +157,33 @@ def test_prefill_workload_d64(sata, oracle_mod):
         assert excl <= 2
 
 
+@pytest.mark.parametrize("name", ["prefill_d128", "prefill_d64_dv32", "prefill_d16_p6"])
+def test_prefill_workload_other_shapes(sata, oracle_mod, name):
+    """The benchmark's other prefill workloads (d = 128, d_K != d_V, P = 6) at
+    full size, in its launch configuration: the first tokens of head 0 against
+    the oracle's recurrence, and on every head a sample of tokens out to the end
+    of the sequence against the direct form."""
+    _set_path(sata, "auto")
+    w = wl.WORKLOADS[name]
+    (q, k, v), _ = wl.make_inputs(w)
+    sata.sata_reset_kernel_stats()
+    y = sata.prefill(q.cuda(), k.cuda(), v.cuda(), P=w.P)
+    torch.cuda.synchronize()
+    assert sata.sata_sync_status() == 0
+    assert ("tc_scan" in sata.sata_kernel_stats()) == (w.P <= 4)
+    ref = _oracle_heads(oracle_mod, q, k, v, w.P, list(w.oracle_heads), T=w.oracle_tokens)
+    _check_heads(y, ref, T=w.oracle_tokens, what=f"{name} head 0, first {w.oracle_tokens} tokens")
+    rng = np.random.default_rng(w.seed)
+    ts = sorted({w.oracle_tokens, w.N // 2 - 1, w.N // 2, w.N - 1,
+                 *rng.integers(w.oracle_tokens, w.N, 6).tolist()})
+    yc = y.cpu()
+    for h in range(w.H):
+        yr, _, kappa = oracle_mod.direct_at(q[0, h], k[0, h], v[0, h], w.P, ts)
+        err, excl, _ = token_rel_err(yc[0, h, ts].double().numpy(), yr, kappa)
+        assert err <= TOL, f"{name} head {h}, tokens {ts}: {err:.3e}"
+        assert excl <= 2
+
+
 @pytest.mark.parametrize("mode", ["deterministic", "atomic", "host"])
 def test_prefill_d64_internal_segments(sata, oracle_mod, mode):
     """d = 64, P = 4 with 64 heads: in the fixed-order mode the partial buffer
