@@ -691,7 +691,15 @@ bool scan_kernels(int d_V, ScanFn *fq, ScanFn *fkv) {
 
 }  // namespace
 
+// The gradient scans run on tensor cores (backward_tc.cuh) where the forward does,
+// unless the fixed-order mode asks for bitwise repeatable results (their sums use
+// atomics); elsewhere on the CUDA-core scans below.
+static bool backward_on_tc(int d_K, int d_V, int P, bool use_tc) {
+    return use_tc && g_opt_deterministic == 0 && prefill_backward_tc_supported(d_K, d_V, P);
+}
+
 size_t prefill_backward_workspace_bytes(int BH, int64_t N, int64_t F, int d_K, int d_V, int P, bool use_tc) {
+    if (backward_on_tc(d_K, d_V, P, use_tc)) return prefill_backward_tc_workspace_bytes(BH, N, F, d_K, d_V, P);
     return bwd_layout(BH, N, F, d_K, d_V, P, use_tc).total;
 }
 
@@ -701,6 +709,8 @@ cudaError_t launch_prefill_backward(const DeviceBasis &basis, int BH, int64_t N,
                                     bool use_tc, int *flags, cudaStream_t stream) {
     const int d_K = basis.d_K, P = basis.P;
     const int64_t F = basis.F;
+    if (backward_on_tc(d_K, d_V, P, use_tc))
+        return launch_prefill_backward_tc(basis, BH, N, d_V, q, k, v, dy, dq, dk, dv, ws, ws_bytes, flags, stream);
     const BwdLayout L = bwd_layout(BH, N, F, d_K, d_V, P, use_tc);
     if (ws_bytes < L.total) return cudaErrorInvalidValue;
     const int ntiles = (int)((F + kTF - 1) / kTF);

@@ -37,4 +37,25 @@ cudaError_t launch_prefill_tc(const DeviceBasis &basis, int BH, int64_t N, int d
     return cudaErrorNotSupported;
 }
 
+bool prefill_backward_tc_supported(int d_K, int d_V, int P) { return prefill_tc_supported(d_K, d_V, P); }
+
+size_t prefill_backward_tc_workspace_bytes(int BH, int64_t N, int64_t F, int d_K, int d_V, int P) {
+#define SATA_TC_CASE(a, b) \
+    if (d_K == a && d_V == b) return tc_bwd_workspace_##a##_##b(BH, N, F, P);
+    SATA_TC_SHAPES(SATA_TC_CASE)
+#undef SATA_TC_CASE
+    return 0;
+}
+
+cudaError_t launch_prefill_backward_tc(const DeviceBasis &basis, int BH, int64_t N, int d_V, const void *q,
+                                       const void *k, const void *v, const float *dy, float *dq, float *dk,
+                                       float *dv, void *ws, size_t ws_bytes, int *flags, cudaStream_t stream) {
+#define SATA_TC_CASE(a, b)                                                                                     \
+    if (basis.d_K == a && d_V == b)                                                                            \
+        return tc_bwd_run_##a##_##b(basis, BH, N, q, k, v, dy, dq, dk, dv, ws, ws_bytes, flags, stream);
+    SATA_TC_SHAPES(SATA_TC_CASE)
+#undef SATA_TC_CASE
+    return cudaErrorNotSupported;
+}
+
 }  // namespace sata

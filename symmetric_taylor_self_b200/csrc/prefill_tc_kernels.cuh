@@ -137,7 +137,17 @@ struct ScanParams {
     int BH, G, c0, nc, nch, P;
     int load_state, store_state, stall_chunk;
     float inv_c;
+    int lc;                          // floor(log2 c): the readout operand's scale bound
     int64_t wait_ns;
+    // gradient scans (JAC kernels) only: Z-column values per token (prescaled fp16, chunk-
+    // interleaved [BH][nch][128]; null: the constant 1), whether the Z columns carry the
+    // column prescale, the readout's per-token multipliers (fp32 [BH][N][mult_stride], true
+    // frame) and the sums [BH][d_K][N] the drain adds into
+    const __half *zval16 = nullptr;
+    int zscaled = 0;
+    const float *mult = nullptr;
+    int mult_stride = 0;
+    float *sums_jac = nullptr;
 };
 
 // ----------------------------------------------------------------- PTX ----
@@ -270,13 +280,26 @@ __device__ __forceinline__ HeadExp head_exps(const float *st) {
 // Exponent sigma_c of the readout operand's scale before chunk cl of this call:
 // |S'| < 2^e_ms + 128 cl + 1 (every prescaled feature and value is at most 1 in
 // magnitude, e_ms bounds the prescaled incoming state), and a degree-p row carries
-// C/p! 2^(p E) <= 2^max(0, (P-1) E), so |B| < 2^15 for every row.
-__device__ __forceinline__ int state_sigma(int cl, int e_ms, int E, int P) {
+// C/p! c^-p 2^(p E) <= 2^(p (E - lc)) <= 2^max(0, (P-1)(E - lc)) (C/p! <= 1, lc =
+// floor(log2 c)), so |B| < 2^15 for every row.  The bound is tight for the rows that
+// reach it; a looser one would push the small rows of B into fp16's subnormal range.
+__device__ __forceinline__ int state_sigma_rows(int cl, int e_ms, int e_row) {
     const uint32_t tok = (uint32_t)cl * kL + 1u;
     const int e_tok = 32 - __clz(tok);
     const int eb = (e_ms > e_tok ? e_ms : e_tok) + 1;
-    const int s = eb + ((P - 1) * E > 0 ? (P - 1) * E : 0) - 15;
+    const int s = eb + e_row - 15;
     return s < -120 ? -120 : (s > 120 ? 120 : s);
+}
+__device__ __forceinline__ int state_sigma(int cl, int e_ms, int E, int P, int lc) {
+    const int r = (P - 1) * (E - lc);
+    return state_sigma_rows(cl, e_ms, r > 0 ? r : 0);
+}
+// The same for a gradient scan: a pair row of degree p' <= P - 2 carries
+// C/p'! c^-(p'+1) 2^(p' E + e_k) <= 2^(p' (E - lc) + e_k - lc) (the slot index is a
+// key-side factor only; the derivative's 1/c is in the row).
+__device__ __forceinline__ int jac_sigma(int cl, int E, int ek, int P, int lc) {
+    const int r = (P - 2) * (E - lc);
+    return state_sigma_rows(cl, -1000, (r > 0 ? r : 0) + ek - lc);
 }
 
 struct Waiter {
@@ -561,7 +584,7 @@ __device__ __forceinline__ void q_drain(const ScanParams &p, int64_t bh, int64_t
     using C = Cfg<DK, DV>;
     constexpr int NL = C::NL;
     tc_after();
-    const int sg = state_sigma(cl, e_ms, E, p.P);
+    const int sg = state_sigma(cl, e_ms, E, p.P, p.lc);
     const float upv = pow2f_sat(sg + ev), upz = pow2f_sat(sg);
     const bool valid = (int64_t)(p.c0 + cl) * kL + t < p.N;
     constexpr int DQ = sum_quads(DV);
@@ -616,6 +639,73 @@ __device__ __forceinline__ void q_drain(const ScanParams &p, int64_t bh, int64_t
     }
 }
 
+// Gradient scan (JAC) drain: R of chunk cl holds, per slot s (index i_s) and column j,
+// sum_pairs P2(a_t) B[pair, (s, j)]; the token's output for slot s is its contraction with
+// the token's multipliers m_t (fp32, true frame): sum_{j < d_V} m_t[j] R[t, (s, j)] +
+// m_t[d_V] R[t, Z_s], added into sums[bh][i_s][token].  Arrives on rf_bar once every column
+// is read.
+template <int DK, int DV>
+__device__ __forceinline__ void q_drain_jac(const ScanParams &p, int64_t bh, int nl, int E, int ek, int ev, int cl,
+                                            int t, int lane, uint32_t tm, uint32_t rf_bar, const int *sl) {
+    using C = Cfg<DK, DV>;
+    constexpr int NL = C::NL;
+    tc_after();
+    const int sg = jac_sigma(cl, E, ek, p.P, p.lc);
+    const float upv = pow2f_sat(sg + ev), upz = pow2f_sat(sg + (p.zscaled ? ev : 0));
+    const int64_t tok = (int64_t)(p.c0 + cl) * kL + t;
+    const bool valid = tok < p.N;
+    const float *m = p.mult + (bh * p.N + (valid ? tok : 0)) * p.mult_stride;
+    float acc[NL], accz[NL];
+    {
+        uint32_t rz[16];
+        tc_ld16(tm + C::COL_R + nl * DV, rz);
+        tc_wait_ld();
+        const float mz = valid ? __ldg(m + DV) : 0.f;
+#pragma unroll
+        for (int s = 0; s < NL; ++s) {
+            acc[s] = 0.f;
+            accz[s] = mz * __uint_as_float(rz[s]);
+        }
+    }
+    constexpr int GW = DV >= 32 ? 32 : 16;
+#pragma unroll 1
+    for (int g = 0; g < DV / GW; ++g) {
+        float mv[GW];
+#pragma unroll
+        for (int i4 = 0; i4 < GW / 4; ++i4) {
+            const float4 x = valid ? __ldg(reinterpret_cast<const float4 *>(m + GW * g) + i4)
+                                   : make_float4(0.f, 0.f, 0.f, 0.f);
+            mv[4 * i4] = x.x;
+            mv[4 * i4 + 1] = x.y;
+            mv[4 * i4 + 2] = x.z;
+            mv[4 * i4 + 3] = x.w;
+        }
+#pragma unroll
+        for (int s = 0; s < NL; ++s) {
+            if (s < nl) {
+                uint32_t ra[GW];
+                if constexpr (GW == 32) tc_ld32(tm + C::COL_R + s * DV + GW * g, ra);
+                else tc_ld16(tm + C::COL_R + s * DV + GW * g, ra);
+                tc_wait_ld();
+                float a = acc[s];
+#pragma unroll
+                for (int i = 0; i < GW; ++i) a = fmaf(mv[i], __uint_as_float(ra[i]), a);
+                acc[s] = a;
+            }
+        }
+        if (g == DV / GW - 1) {   // every column read: the next readout may overwrite R
+            tc_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(rf_bar);
+        }
+    }
+    if (valid) {
+#pragma unroll
+        for (int s = 0; s < NL; ++s)
+            if (s < nl) atomicAdd(p.sums_jac + (bh * DK + sl[s]) * p.N + tok, fmaf(acc[s], upv, accz[s] * upz));
+    }
+}
+
 // conversion: 16 fp32 state columns of one slot's V part -> 8 packed fp16 words, scaled by f.
 __device__ __forceinline__ void conv_v(const uint32_t (&rr)[16], float f, uint32_t (&hp)[8]) {
 #pragma unroll
@@ -649,7 +739,12 @@ __device__ __forceinline__ int frame_exp(int n, int nl, const int (&dg)[NL], int
     return -(seli(dg, s_out) * ek);
 }
 
-template <int DK, int DV>
+// JAC = false: the prefill scan (features of degree < P, den from the Z columns).
+// JAC = true: a gradient scan of the backward pass: pair rows of degree <= P - 2 (the
+// derivative T_{P-1} of the Taylor weight), slots index the key-side vector as a value
+// dimension, the Z columns take zval16 (or 1), and the drain contracts each slot's
+// columns with the token's multipliers (q_drain_jac).  Fresh state only.
+template <int DK, int DV, bool JAC = false>
 __global__ void __launch_bounds__(kScanThreads, 1) tc_scan_kernel(const ScanParams p) {
     using C = Cfg<DK, DV>;
     constexpr int NL = C::NL;
@@ -774,6 +869,17 @@ __global__ void __launch_bounds__(kScanThreads, 1) tc_scan_kernel(const ScanPara
                         *reinterpret_cast<uint4 *>(wrow + (s * (DV / 8) + i) * 128) = hmul2x4(vr[i], kl[s]);
                 }
             }
+            uint32_t zv = 0x3C003C00u;   // the Z columns' factor: 1, or the token's value (JAC)
+            if constexpr (JAC) {
+                if (p.zval16) {
+                    const bool valid = (int64_t)(p.c0 + cl) * kL + t < p.N;
+                    const uint32_t h =
+                        valid ? (uint32_t)__ldg(reinterpret_cast<const unsigned short *>(p.zval16) +
+                                                ((int64_t)bh * p.nch + p.c0 + cl) * kL + t)
+                              : 0u;
+                    zv = h | (h << 16);
+                }
+            }
             for (int z8 = nl * (DV / 8); z8 < NU / 8; ++z8) {
                 uint32_t w4[4];
 #pragma unroll
@@ -782,8 +888,9 @@ __global__ void __launch_bounds__(kScanThreads, 1) tc_scan_kernel(const ScanPara
                     uint32_t lo = 0, hi = 0;
 #pragma unroll
                     for (int s = 0; s < NL; ++s) {
-                        lo = (s == s0 && s < nl) ? (kl[s] & 0xFFFFu) : lo;
-                        hi = (s == s1 && s < nl) ? (kl[s] & 0xFFFFu) : hi;
+                        const uint32_t kz = JAC ? hmul2u(kl[s], zv) : kl[s];
+                        lo = (s == s0 && s < nl) ? (kz & 0xFFFFu) : lo;
+                        hi = (s == s1 && s < nl) ? (kz & 0xFFFFu) : hi;
                     }
                     w4[j] = lo | (hi << 16);
                 }
@@ -820,8 +927,13 @@ __global__ void __launch_bounds__(kScanThreads, 1) tc_scan_kernel(const ScanPara
             tc_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(BAR(C::B_AQF));
-            if (cl > 0) q_drain<DK, DV>(p, bh, part_base, nl, e_ms, E, he.ev, cl - 1, t, lane, tmem + lane_off,
-                                        BAR(C::B_RF), qlp);
+            if (cl > 0) {
+                if constexpr (JAC)
+                    q_drain_jac<DK, DV>(p, bh, nl, E, he.ek, he.ev, cl - 1, t, lane, tmem + lane_off, BAR(C::B_RF), sl);
+                else
+                    q_drain<DK, DV>(p, bh, part_base, nl, e_ms, E, he.ev, cl - 1, t, lane, tmem + lane_off,
+                                    BAR(C::B_RF), qlp);
+            }
 #pragma unroll
             for (int s = 0; s < NL; ++s) qlp[s] = h_lo(xl[s]);
             {   // the next chunk's operand (its row is read after the drain, which needs the
@@ -832,8 +944,13 @@ __global__ void __launch_bounds__(kScanThreads, 1) tc_scan_kernel(const ScanPara
                 p2q_dispatch<DK, 0, C::NPT>(ktile, x, pq);
             }
         }
-        if (ok && p.nc > 0 && W.wait(BAR(C::B_RD), (p.nc - 1) & 1))
-            q_drain<DK, DV>(p, bh, part_base, nl, e_ms, E, he.ev, p.nc - 1, t, lane, tmem + lane_off, BAR(C::B_RF), qlp);
+        if (ok && p.nc > 0 && W.wait(BAR(C::B_RD), (p.nc - 1) & 1)) {
+            if constexpr (JAC)
+                q_drain_jac<DK, DV>(p, bh, nl, E, he.ek, he.ev, p.nc - 1, t, lane, tmem + lane_off, BAR(C::B_RF), sl);
+            else
+                q_drain<DK, DV>(p, bh, part_base, nl, e_ms, E, he.ev, p.nc - 1, t, lane, tmem + lane_off, BAR(C::B_RF),
+                                qlp);
+        }
         tc_before();
     } else {
         // ------------------------------------------------ state -> fp16 readout operand
@@ -850,7 +967,9 @@ __global__ void __launch_bounds__(kScanThreads, 1) tc_scan_kernel(const ScanPara
             cf[s] = s < nl ? p.unit_coef[at] : 0.f;
             fi[s] = s < nl ? p.unit_fidx[at] : -1;
             dg[s] = ppair + (sl[s] < DK);               // degree of feature (pair r, l_s)
-            pe[s] = dg[s] * E;
+            // prefill: the feature's degree on both sides; gradient scan: the pair's degree on
+            // both sides, the slot on the key side only
+            pe[s] = JAC ? (dg[s] - 1) * E + he.ek : dg[s] * E;
             for (int i = 0; i < dg[s]; ++i) cf[s] *= p.inv_c;   // alpha_p = 1 / (p! c^p)
         }
         constexpr int NG = C::NG;
@@ -886,7 +1005,7 @@ __global__ void __launch_bounds__(kScanThreads, 1) tc_scan_kernel(const ScanPara
             // B double buffer: the readout of chunk cl-2 has read it
             if (cl >= 2 && !(ok = W.wait(BAR(C::B_BSE + b), ((cl >> 1) - 1) & 1))) break;
             tc_after();
-            const int sg = state_sigma(cl, e_ms, E, p.P);
+            const int sg = JAC ? jac_sigma(cl, E, he.ek, p.P, p.lc) : state_sigma(cl, e_ms, E, p.P, p.lc);
             float sc[NL];
 #pragma unroll
             for (int s = 0; s < NL; ++s) sc[s] = cf[s] * pow2f_sat(pe[s] - sg);
@@ -1243,6 +1362,13 @@ struct UnitPlan {
 
 size_t align256(size_t x) { return (x + 255) / 256 * 256; }
 
+// floor(log2 c), c = sqrt(d_K): the largest e with 2^(2e) <= d_K.
+int floor_log2_c(int d_K) {
+    int e = 0;
+    while ((int64_t)1 << (2 * (e + 1)) <= d_K) ++e;
+    return e;
+}
+
 bool build_unit_plan(int D, int P, int NL, UnitPlan &up) {
     HostBasis hb;
     if (!build_basis_host(D, P, hb)) return false;
@@ -1528,6 +1654,7 @@ cudaError_t run(const DeviceBasis &basis, int BH, int64_t N, const void *q, cons
         sp.store_state = (s + 1 < nseg || !own_state) ? 1 : 0;
         sp.stall_chunk = stall;
         sp.inv_c = inv_c;
+        sp.lc = floor_log2_c(DK);
         sp.wait_ns = wait_ns;
         launch_begin(kTcScan, stream);
         tc_scan_kernel<DK, DV><<<BH * pl.G, kScanThreads, C::SMEM, stream>>>(sp);

@@ -1,4 +1,4 @@
-// The (d_K, d_V) instances of the tensor-core prefill and their entry points.
+// The (d_K, d_V) instances of the tensor-core prefill and backward, and their entry points.
 #pragma once
 
 #include <cstddef>
@@ -22,4 +22,11 @@ namespace sata {
                                  float *den_out);
 SATA_TC_SHAPES(SATA_TC_DECLARE)
 #undef SATA_TC_DECLARE
+#define SATA_TC_BWD_DECLARE(a, b)                                                                               \
+    size_t tc_bwd_workspace_##a##_##b(int BH, int64_t N, int64_t F, int P);                                      \
+    cudaError_t tc_bwd_run_##a##_##b(const DeviceBasis &basis, int BH, int64_t N, const void *q, const void *k, \
+                                     const void *v, const float *dy, float *dq, float *dk, float *dv, void *ws, \
+                                     size_t ws_bytes, int *flags, cudaStream_t stream);
+SATA_TC_SHAPES(SATA_TC_BWD_DECLARE)
+#undef SATA_TC_BWD_DECLARE
 }  // namespace sata

@@ -67,7 +67,7 @@ const void *device_table(uint64_t key, size_t bytes, const std::function<void(ui
 // Kernel identities for launch statistics.
 enum KernelId {
     kDecodeStream = 0, kDecodeFinish, kSimtScan, kSimtFinish, kTcPrep, kTcScan, kTcFinish, kTcReduce,
-    kBwdR, kBwdQScan, kBwdKVScan, kBwdFinish, kStateAdd, kNumKernels
+    kBwdR, kBwdQScan, kBwdKVScan, kBwdFinish, kStateAdd, kBwdTcPrep, kBwdTcScan, kBwdTcFinish, kNumKernels
 };
 const char *kernel_name(int id);
 // Call around every kernel launch: begin() records a start event when timing is
@@ -99,6 +99,14 @@ cudaError_t launch_prefill_simt(const DeviceBasis &basis, int BH, int64_t N, int
 // S += dS (nS floats), Z += dZ (nZ floats), on `stream`.
 cudaError_t launch_state_add(float *S, float *Z, const float *dS, const float *dZ, int64_t nS, int64_t nZ,
                              cudaStream_t stream);
+
+// ---- backward of the prefill on tensor cores (backward_tc.cuh via prefill_tc.cu) ----
+// Shapes of the tensor-core prefill; the gradient scans add into their sums with atomics.
+bool prefill_backward_tc_supported(int d_K, int d_V, int P);
+size_t prefill_backward_tc_workspace_bytes(int BH, int64_t N, int64_t F, int d_K, int d_V, int P);
+cudaError_t launch_prefill_backward_tc(const DeviceBasis &basis, int BH, int64_t N, int d_V, const void *q,
+                                       const void *k, const void *v, const float *dy, float *dq, float *dk,
+                                       float *dv, void *ws, size_t ws_bytes, int *flags, cudaStream_t stream);
 
 // ---- backward of the prefill, CUDA-core path (backward_simt.cu) ----
 size_t prefill_backward_workspace_bytes(int BH, int64_t N, int64_t F, int d_K, int d_V, int P, bool use_tc);
