@@ -570,21 +570,30 @@ def run_part(torch, sata, wl, args, world):
 
 
 def backward_flops(d_K, d_V, P):
-    """Algorithmic FLOPs per token and head of the backward's two scans (the
-    feature-form contractions; the Jacobian products and features not counted):
-    dq scan: S r_t and the S update, 2 x 2F(d_V+1);
-    dk/dv scan: G u_s, the dv readout 2F d_V, the G update: 4F(d_V+1) + 2F d_V."""
+    """Algorithmic FLOPs per token and head of the backward's gradient scans (the
+    feature-form contractions; the features, the pairs inside a chunk and the
+    recomputed forward not counted).
+    Tensor-core path: dq and dk each update and read a state of F2 x d_K x (d_V + 1)
+    values, F2 = binom(d_K + P - 2, P - 2) the features of T_{P-1}: 2 x 2 F2 d_K (d_V + 1)
+    each; dv is the prefill's scan on the reversed sequence (flops_per_token).
+    CUDA-core path: dq scan: S r_t and the S update, 2 x 2F(d_V+1); dk/dv scan: G u_s,
+    the dv readout 2F d_V, the G update: 4F(d_V+1) + 2F d_V."""
     F = math.comb(d_K + P - 1, P - 1)
-    return {"bwd_q_scan": 4 * F * (d_V + 1), "bwd_kv_scan": 4 * F * (d_V + 1) + 2 * F * d_V}
+    F2 = math.comb(d_K + P - 2, P - 2) if P >= 2 else 0
+    return {"bwd_tc_scan": 8 * F2 * d_K * (d_V + 1) + flops_per_token(d_K, d_V, P),
+            "bwd_q_scan": 4 * F * (d_V + 1), "bwd_kv_scan": 4 * F * (d_V + 1) + 2 * F * d_V}
 
 
 def bench_backward(torch, sata, wl, args, world, dev, stream, peaks, peaks_src):
+    """The backward workload; each timed step is preceded (outside its events) by a
+    256 MB write that flushes L2, since the step's working set is close to its size."""
     w = wl.WORKLOADS[args.backward_workload]
     (q, k, v), _ = wl.make_inputs(w)
     qd, kd, vd, dy = q.to(dev), k.to(dev), v.to(dev), wl.cotangent(w).to(dev)
     dq = torch.empty((w.B, w.H, w.N, w.d_K), dtype=torch.float32, device=dev)
     dk = torch.empty_like(dq)
     dv = torch.empty((w.B, w.H, w.N, w.d_V), dtype=torch.float32, device=dev)
+    flush = torch.empty(64 << 20, dtype=torch.float32, device=dev)
 
     def step():
         sata.sata_prefill_backward(qd, kd, vd, dy, dq, dk, dv, w.B, w.H, w.N, w.d_K, w.d_V, w.P, None,
@@ -597,19 +606,36 @@ def bench_backward(torch, sata, wl, args, world, dev, stream, peaks, peaks_src):
     torch.cuda.synchronize()
     sata.sata_reset_kernel_stats()
     sata.sata_set_option(sata.SATA_OPT_TIME_KERNELS, 1)
-    ms = timed(torch, world, step, args.steps, 0, stream)
+    ms = 0.0
+    for _ in range(args.steps):
+        with torch.cuda.stream(stream):
+            flush.fill_(1.0)
+        ms += timed(torch, world, step, 1, 0, stream)
     stats = sata.sata_kernel_stats()
     sata.sata_set_option(sata.SATA_OPT_TIME_KERNELS, 0)
     if sata.sata_sync_status(stream) != 0:
         raise RuntimeError("device status after the backward")
     value = job_throughput(w.B * w.N, args.steps, world, ms)
     per_tok = backward_flops(w.d_K, w.d_V, w.P)
-    # the scans' contractions run on tensor cores with tf32 operands: the tf32 dense
-    # peak is the measured bf16 peak times the nominal ratio 1.1 / 2.25
-    tf32_peak = peaks["bf16_tflops"] * 1.1 / 2.25
     roof = None
     scans = {k_: stats[k_] for k_ in per_tok if k_ in stats}
-    if scans:
+    if "bwd_tc_scan" in scans:
+        # three launches a step (dq, dk, dv) of different sizes: the step's scan FLOPs over
+        # the step's scan time, i.e. the mean over the three
+        n_l, ms_l = scans["bwd_tc_scan"]
+        flops_per_launch = per_tok["bwd_tc_scan"] * w.B * w.H * w.N * args.steps / n_l
+        achieved = flops_per_launch / (ms_l / n_l / 1000.0) / 1e12
+        roof = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                "frac": achieved / peaks["bf16_tflops"], "kernel": "bwd_tc_scan",
+                "launches_per_step": n_l / args.steps, "ms_per_launch": ms_l / n_l,
+                "algorithmic_flops_per_launch": flops_per_launch,
+                "peak_kind": f"{peaks_src} bf16 dense burst (fp16 operands run at the bf16 rate); FLOPs and "
+                             "time are the mean over the step's dq, dk and dv scans",
+                "traffic": ncu_traffic("bwd_tc_scan")}
+    elif scans:
+        # the CUDA-core gradient scans' contractions run on tensor cores with tf32 operands:
+        # the tf32 dense peak is the measured bf16 peak times the nominal ratio 1.1 / 2.25
+        tf32_peak = peaks["bf16_tflops"] * 1.1 / 2.25
         dom = max(scans, key=lambda n: scans[n][1])
         n_l, ms_l = scans[dom]
         flops_per_launch = per_tok[dom] * w.B * w.H * w.N * args.steps / n_l
@@ -624,7 +650,7 @@ def bench_backward(torch, sata, wl, args, world, dev, stream, peaks, peaks_src):
             "steps": args.steps, "ms_per_step": ms / args.steps,
             "workload": f"{w.name}: B={w.B} H={w.H} N={w.N} d_K={w.d_K} d_V={w.d_V} P={w.P} F={w.F}; "
                         f"dy N(0,1) fp32; the step recomputes the forward on the prefill's path",
-            "l2": "each step writes more than 1 GB of partial sums, far above the 126 MB L2",
+            "l2": "L2 flushed (256 MB write) before each timed step",
             "roofline": roof, "gpu_launches": sum(n for n, _ in stats.values()),
             "kernel_ms": {k_: {"launches": n, "ms": t} for k_, (n, t) in stats.items()}}
 

@@ -215,22 +215,28 @@ SATA_API int sata_prefill_host(const void *q, const void *k, const void *v, floa
  * "Comparison with other methods", "Future directions"); this is the exact
  * gradient of the forward as defined in [CC-TAYLOR] "Feature maps and linear
  * attention", y_t = num_t / den_t, computed in the same chunked feature form
- * (fixed cost per token): the forward is recomputed, then one pass forward
- * over the sequence with S gives dq and one pass backward with
- * G = sum_t phi(q_t) [dy_t / den_t | -(dy_t . y_t) / den_t]^T gives dk and dv.
- * The recomputed forward takes the prefill's path (tensor cores where
- * sata_prefill_ex would use them, keeping den); the two gradient scans run for
- * every supported shape, their contractions on tensor cores with tf32 operands
- * split into high and low parts (fp32-level accuracy).
+ * (fixed cost per token).  With w_ts = T_P(q_t . k_s / c), T_P(x) = sum_{p<P}
+ * x^p / p!, and r_t = [dy_t / den_t | -(dy_t . y_t) / den_t]:
+ *   dq_t = 1/c sum_{s<=t} (r_t . [v_s|1]) T_{P-1}(x_ts) k_s,
+ *   dk_s = 1/c sum_{t>=s} (r_t . [v_s|1]) T_{P-1}(x_ts) q_t,
+ *   dv_s = sum_{t>=s} w_ts dy_t / den_t  (T_P' = T_{P-1}).
+ * The forward is recomputed on the prefill's path (keeping den).  Where that
+ * path is the tensor-core one and SATA_OPT_DETERMINISTIC is 0, the three sums
+ * are tensor-core scans: dq and dk over the features of T_{P-1} with d_K-wide
+ * values, dv the prefill's scan on the time-reversed sequence (fp16 operands
+ * after per-head power-of-two scales, fp32 accumulation, sums added with fp32
+ * atomics, so not bitwise repeatable).  Otherwise one CUDA-core pass forward
+ * with S gives dq and one backward with G = sum_t phi(q_t) r_t^T gives dk and
+ * dv, their contractions on tensor cores with tf32 operands split into high and
+ * low parts (fp32-level accuracy), partial sums added in a fixed order: bitwise
+ * reproducible when the forward is (SATA_OPT_DETERMINISTIC = 1, or the CUDA-core
+ * path).
  *   q, k: bf16 [B][H][N][d_K];  v: bf16 [B][H][N][d_V]  (the forward's inputs)
  *   dy:   fp32 [B][H][N][d_V]
  *   dq, dk: fp32 [B][H][N][d_K];  dv: fp32 [B][H][N][d_V]  (overwritten)
  *   workspace: NULL (library-owned) or a device buffer of ws_bytes >=
  *              sata_backward_workspace_bytes(...).
  *   stream: cudaStream_t (NULL: legacy stream).
- * The gradient scans add their partial sums in a fixed order; the result is
- * bitwise reproducible when the forward is (SATA_OPT_DETERMINISTIC = 1, or the
- * CUDA-core path).
  * N = 0 is a no-op.  Errors as sata_prefill_ex.
  */
 SATA_API int sata_backward_workspace_bytes(int B, int H, int64_t N, int d_K, int d_V, int P, size_t *bytes);
