@@ -758,9 +758,10 @@ __global__ void __launch_bounds__(kScanThreads, 1) tc_scan_kernel(const ScanPara
     int *sl = reinterpret_cast<int *>(smem + C::OFF_L);
 
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-    // unit-major order: every head's largest units are scheduled first
-    const int64_t bh = blockIdx.x % p.BH;
-    const int u = blockIdx.x / p.BH;
+    // head-major order (a head's units, largest first, then the next head's): the CTAs
+    // resident at a time share one or two heads' token rows and sums in L2
+    const int64_t bh = blockIdx.x / p.G;
+    const int u = blockIdx.x % p.G;
     const int ktile = p.unit_k[u];
     const int nl = p.unit_nl[u];
     const int NU = (nl * (DV + 1) + 15) / 16 * 16;   // MMA N of this unit
@@ -896,13 +897,13 @@ __global__ void __launch_bounds__(kScanThreads, 1) tc_scan_kernel(const ScanPara
                 }
                 *reinterpret_cast<uint4 *>(wrow + z8 * 128) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
             }
-            if (cl + 1 < p.nc) {
-                fetch_row<DK>(p.k16, p, bh, sl, cl + 1, t, x, kl);
-            }
             fence_proxy_async();
             __syncwarp();
             // test hook: one producer signal withheld, so the issuer's wait expires
             if (lane == 0 && !(warp == kWarpK0 && p.c0 + cl == p.stall_chunk)) mbar_arrive(BAR(C::B_AKF));
+            // the next chunk's k row, requested after the signal: its slot values are used as
+            // soon as they land, so the load latency would otherwise sit before the update
+            if (cl + 1 < p.nc) fetch_row<DK>(p.k16, p, bh, sl, cl + 1, t, x, kl);
         }
     } else if (warp < kWarpC0) {
         // ------------------------------------------------ q side: P2(q) operand, readout drain
