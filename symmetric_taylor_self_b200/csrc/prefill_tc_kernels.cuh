@@ -727,18 +727,6 @@ __device__ __forceinline__ void conv_z(const uint32_t (&rr)[16], int nl, const f
     }
 }
 
-// conversion: exponent taking a true-frame state value of column n to the prescaled TMEM
-// frame (S' = S 2^-(p e_k + e_v), Z' = Z 2^-(p e_k)), and the column's slot.
-template <int NL, int DV>
-__device__ __forceinline__ int frame_exp(int n, int nl, const int (&dg)[NL], int ek, int ev, int &s_out) {
-    if (n < nl * DV) {
-        s_out = n / DV;
-        return -(seli(dg, s_out) * ek + ev);
-    }
-    s_out = n - nl * DV;
-    return -(seli(dg, s_out) * ek);
-}
-
 // JAC = false: the prefill scan (features of degree < P, den from the Z columns).
 // JAC = true: a gradient scan of the backward pass: pair rows of degree <= P - 2 (the
 // derivative T_{P-1} of the Taylor weight), slots index the key-side vector as a value
@@ -978,22 +966,37 @@ __global__ void __launch_bounds__(kScanThreads, 1) tc_scan_kernel(const ScanPara
         const int ngv = nl * DV / 16;   // groups of V columns; group ngv holds the Z columns (and padding)
         bool ok = true;
         if (p.load_state) {   // incoming state -> TMEM (prescaled frame)
+            // a V group is 16 contiguous columns of one feature's S row (four 16-byte loads);
+            // the Z group gathers one Z value per slot
 #pragma unroll 1
             for (int g = 0; g < NG; ++g) {
                 if (g < ngu) {
                     uint32_t v16[16];
+                    if (16 * g < nl * DV) {
+                        const int sv = (16 * g) / DV;
+                        const int f = seli(fi, sv);
+                        const float sc = pow2f_sat(-(seli(dg, sv) * he.ek + he.ev));
+                        const float4 *src = reinterpret_cast<const float4 *>(p.S + (bh * p.F + (f >= 0 ? f : 0)) * DV +
+                                                                             (16 * g) % DV);
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        const int n = 16 * g + i;
-                        int s = 0;
-                        const int fe = frame_exp<NL, DV>(n, nl, dg, he.ek, he.ev, s);
-                        float x = 0.f;
-                        if (s < nl && n < nl * (DV + 1)) {
-                            const int f = seli(fi, s);
-                            if (f >= 0) x = (n < nl * DV ? p.S[(bh * p.F + f) * DV + (n % DV)] : p.Z[bh * p.F + f]) *
-                                            pow2f_sat(fe);
+                        for (int j = 0; j < 4; ++j) {
+                            const float4 x = f >= 0 ? src[j] : make_float4(0.f, 0.f, 0.f, 0.f);
+                            v16[4 * j] = __float_as_uint(x.x * sc);
+                            v16[4 * j + 1] = __float_as_uint(x.y * sc);
+                            v16[4 * j + 2] = __float_as_uint(x.z * sc);
+                            v16[4 * j + 3] = __float_as_uint(x.w * sc);
                         }
-                        v16[i] = __float_as_uint(x);
+                    } else {
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) {
+                            const int sz = 16 * g + i - nl * DV;
+                            float x = 0.f;
+                            if (sz < nl) {
+                                const int f = seli(fi, sz);
+                                if (f >= 0) x = p.Z[bh * p.F + f] * pow2f_sat(-(seli(dg, sz) * he.ek));
+                            }
+                            v16[i] = __float_as_uint(x);
+                        }
                     }
                     tc_st16(tmem + lane_off + C::COL_S + 16 * g, v16);
                 }
@@ -1063,17 +1066,26 @@ __global__ void __launch_bounds__(kScanThreads, 1) tc_scan_kernel(const ScanPara
                     uint32_t rr[16];
                     tc_ld16(tmem + lane_off + C::COL_S + 16 * g, rr);
                     tc_wait_ld();
+                    if (16 * g < nl * DV) {   // 16 contiguous columns of one S row
+                        const int sv = (16 * g) / DV;
+                        const int f = seli(fi, sv);
+                        const float sc = pow2f_sat(seli(dg, sv) * he.ek + he.ev);
+                        if (f >= 0) {
+                            float4 *dst = reinterpret_cast<float4 *>(p.S + (bh * p.F + f) * DV + (16 * g) % DV);
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        const int n = 16 * g + i;
-                        int s = 0;
-                        const int fe = frame_exp<NL, DV>(n, nl, dg, he.ek, he.ev, s);
-                        if (s < nl && n < nl * (DV + 1)) {
-                            const int f = seli(fi, s);
-                            if (f >= 0) {
-                                const float x = __uint_as_float(rr[i]) * pow2f_sat(-fe);
-                                if (n < nl * DV) p.S[(bh * p.F + f) * DV + (n % DV)] = x;
-                                else p.Z[bh * p.F + f] = x;
+                            for (int j = 0; j < 4; ++j)
+                                dst[j] = make_float4(__uint_as_float(rr[4 * j]) * sc, __uint_as_float(rr[4 * j + 1]) * sc,
+                                                     __uint_as_float(rr[4 * j + 2]) * sc,
+                                                     __uint_as_float(rr[4 * j + 3]) * sc);
+                        }
+                    } else {
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) {
+                            const int sz = 16 * g + i - nl * DV;
+                            if (sz < nl) {
+                                const int f = seli(fi, sz);
+                                if (f >= 0)
+                                    p.Z[bh * p.F + f] = __uint_as_float(rr[i]) * pow2f_sat(seli(dg, sz) * he.ek);
                             }
                         }
                     }
