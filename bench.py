@@ -142,16 +142,20 @@ def gpu_uuid(torch, dev):
         return str(dev)
 
 
-def kernel_source_hash(name):
-    p = os.path.join(ROOT, "symmetric_taylor_self_b200", "csrc", name)
-    if not os.path.exists(p):
-        return None
-    return hashlib.sha256(open(p, "rb").read()).hexdigest()[:16]
+def kernel_source_hash(names):
+    """sha256 (16 hex digits) of the kernel's source file(s) under csrc/, in order."""
+    h = hashlib.sha256()
+    for name in ([names] if isinstance(names, str) else names):
+        p = os.path.join(ROOT, "symmetric_taylor_self_b200", "csrc", name)
+        if not os.path.exists(p):
+            return None
+        h.update(open(p, "rb").read())
+    return h.hexdigest()[:16]
 
 
 def ncu_traffic(kernel):
-    """DRAM bytes per launch from the committed ncu summary, if the kernel source
-    is unchanged since the capture; else None."""
+    """DRAM bytes per launch from the committed ncu summary, if the kernel's sources
+    are unchanged since the capture; else None."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
         return None
