@@ -303,6 +303,42 @@ struct FinBwd {
     static_assert(SMEM <= 232448, "finish shared memory");
 };
 
+// Loads rows [0, n) of a frame chunk into shared memory as fp32, row stride `ld`:
+// bf16 rows of D values (16-byte loads) or fp32 rows of the r buffer (D + 1 values of
+// stride bwd_rs, 16-byte loads); u = [v | 1] rows are bf16 rows plus the constant.
+template <int D, bool REV>
+__device__ __forceinline__ void fin_rows_bf16(float *dst, int ld, const __nv_bfloat16 *src, int64_t bh, int64_t N,
+                                              int64_t f0, int n) {
+    for (int e = threadIdx.x; e < n * (D / 8); e += 256) {
+        const int i = e / (D / 8), j = e % (D / 8);
+        const int64_t f = f0 + i;
+        const int64_t o = REV ? N - 1 - f : f;
+        const uint4 w = __ldg(reinterpret_cast<const uint4 *>(src + (bh * N + o) * D) + j);
+        const uint32_t x[4] = {w.x, w.y, w.z, w.w};
+        float *d = dst + i * ld + 8 * j;
+#pragma unroll
+        for (int h = 0; h < 4; ++h) {
+            d[2 * h] = __uint_as_float(x[h] << 16);
+            d[2 * h + 1] = __uint_as_float(x[h] & 0xFFFF0000u);
+        }
+    }
+}
+template <int DV, bool REV>
+__device__ __forceinline__ void fin_rows_r(float *dst, int ld, int ncols, const float *r, int64_t bh, int64_t N,
+                                           int64_t f0, int n) {
+    constexpr int Q = bwd_rs(DV) / 4;
+    for (int e = threadIdx.x; e < n * Q; e += 256) {
+        const int i = e / Q, j = e % Q;
+        const int64_t f = f0 + i;
+        const int64_t o = REV ? N - 1 - f : f;
+        const float4 w = __ldg(reinterpret_cast<const float4 *>(r + (bh * N + o) * bwd_rs(DV)) + j);
+        const float x[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+        for (int h = 0; h < 4; ++h)
+            if (4 * j + h < ncols) dst[i * ld + 4 * j + h] = x[h];
+    }
+}
+
 template <int DK, int DV, int KIND>
 __global__ void __launch_bounds__(256)
 bwd_tc_finish_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k,
@@ -324,71 +360,128 @@ bwd_tc_finish_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *_
     const int nr = nt - r0 < FC::RQ ? nt - r0 : FC::RQ;
     const int ns = r0 + nr;                    // keys 0 .. ns-1 of the chunk
     constexpr bool REV = KIND != 0;
-    auto orig = [N](int64_t f) { return REV ? N - 1 - f : f; };
     const __nv_bfloat16 *qa = KIND == 0 ? q : k, *kb = KIND == 0 ? k : q;
     const int tid = threadIdx.x;
-    for (int e = tid; e < nr * DK; e += 256) {
-        const int i = e / DK, a = e % DK;
-        A[i * FC::AW + a] = __bfloat162float(qa[(bh * N + orig(f0 + r0 + i)) * DK + a]);
-    }
-    for (int e = tid; e < ns * DK; e += 256) {
-        const int i = e / DK, a = e % DK;
-        B[i * FC::AW + a] = __bfloat162float(kb[(bh * N + orig(f0 + i)) * DK + a]);
-    }
+    fin_rows_bf16<DK, REV>(A, FC::AW, qa, bh, N, f0 + r0, nr);
+    fin_rows_bf16<DK, REV>(B, FC::AW, kb, bh, N, f0, ns);
     if constexpr (KIND != 2) {
         // r rows on the query side for dq, on the key side for dk; u = [v | 1] on the other
-        for (int e = tid; e < nr * (DV + 1); e += 256) {
-            const int i = e / (DV + 1), j = e % (DV + 1);
-            const int64_t o = bh * N + orig(f0 + r0 + i);
-            M[i * FC::MW + j] = KIND == 0 ? r[o * bwd_rs(DV) + j] : (j < DV ? __bfloat162float(v[o * DV + j]) : 1.f);
-        }
-        for (int e = tid; e < ns * (DV + 1); e += 256) {
-            const int i = e / (DV + 1), j = e % (DV + 1);
-            const int64_t o = bh * N + orig(f0 + i);
-            S[i * FC::SW + j] = KIND == 0 ? (j < DV ? __bfloat162float(v[o * DV + j]) : 1.f) : r[o * bwd_rs(DV) + j];
-        }
+        float *mr = KIND == 0 ? M : S, *mu = KIND == 0 ? S : M;
+        const int ldr = KIND == 0 ? FC::MW : FC::SW, ldu = KIND == 0 ? FC::SW : FC::MW;
+        fin_rows_r<DV, REV>(mr, ldr, DV + 1, r, bh, N, KIND == 0 ? f0 + r0 : f0, KIND == 0 ? nr : ns);
+        const int nu = KIND == 0 ? ns : nr;
+        fin_rows_bf16<DV, REV>(mu, ldu, v, bh, N, KIND == 0 ? f0 : f0 + r0, nu);
+        for (int i = tid; i < nu; i += 256) mu[i * ldu + DV] = 1.f;
     } else {
-        for (int e = tid; e < ns * DV; e += 256) {
-            const int i = e / DV, j = e % DV;
-            S[i * FC::SW + j] = r[(bh * N + orig(f0 + i)) * bwd_rs(DV) + j];
+        fin_rows_r<DV, REV>(S, FC::SW, DV, r, bh, N, f0, ns);
+    }
+    // rows past the chunk's end: zero, so that whole tiles can be computed
+    for (int e = tid; e < (FC::RQ - nr) * FC::AW; e += 256) A[nr * FC::AW + e] = 0.f;
+    for (int e = tid; e < (kL - ns) * FC::AW; e += 256) B[ns * FC::AW + e] = 0.f;
+    if constexpr (KIND != 2)
+        for (int e = tid; e < (FC::RQ - nr) * FC::MW; e += 256) M[nr * FC::MW + e] = 0.f;
+    for (int e = tid; e < (kL - ns) * FC::SW; e += 256) S[ns * FC::SW + e] = 0.f;
+    __syncthreads();
+    // weights: each thread a 4 x 4 tile (query rows 4 wi .. 4 wi + 3, keys ks + 32 j); a
+    // warp shares its query rows (broadcast) and spans 32 consecutive keys (odd strides:
+    // no bank conflicts)
+    {
+        const int wi = tid / 32, ks = tid % 32;
+        const int i0 = 4 * wi;
+        if (i0 < nr) {
+            float x[4][4], d[4][4];
+#pragma unroll
+            for (int a = 0; a < 4; ++a)
+#pragma unroll
+                for (int b = 0; b < 4; ++b) x[a][b] = d[a][b] = 0.f;
+            const int smax = r0 + i0 + 3;   // the tile's last query row sees keys up to it
+#pragma unroll 4
+            for (int e = 0; e < DK; ++e) {
+                float av[4], bv[4];
+#pragma unroll
+                for (int a = 0; a < 4; ++a) av[a] = A[(i0 + a) * FC::AW + e];
+#pragma unroll
+                for (int b = 0; b < 4; ++b) bv[b] = B[(ks + 32 * b) * FC::AW + e];
+#pragma unroll
+                for (int a = 0; a < 4; ++a)
+#pragma unroll
+                    for (int b = 0; b < 4; ++b) x[a][b] = fmaf(av[a], bv[b], x[a][b]);
+            }
+            if constexpr (KIND != 2) {
+#pragma unroll 4
+                for (int e = 0; e <= DV; ++e) {
+                    float mv[4], sv[4];
+#pragma unroll
+                    for (int a = 0; a < 4; ++a) mv[a] = M[(i0 + a) * FC::MW + e];
+#pragma unroll
+                    for (int b = 0; b < 4; ++b) sv[b] = S[(ks + 32 * b) * FC::SW + e];
+#pragma unroll
+                    for (int a = 0; a < 4; ++a)
+#pragma unroll
+                        for (int b = 0; b < 4; ++b) d[a][b] = fmaf(mv[a], sv[b], d[a][b]);
+                }
+            }
+#pragma unroll
+            for (int a = 0; a < 4; ++a)
+#pragma unroll
+                for (int b = 0; b < 4; ++b) {
+                    const int s = ks + 32 * b, i = i0 + a;
+                    float w = 0.f;
+                    if (s <= r0 + i && s <= smax) {
+                        const float xx = x[a][b] * inv_c;
+                        w = KIND == 2 ? taylor_n(xx, P) : d[a][b] * taylor_n(xx, P - 1) * inv_c;
+                    }
+                    Wt[i * FC::WW + s] = w;
+                }
         }
     }
     __syncthreads();
-    for (int e = tid; e < nr * kL; e += 256) {
-        const int i = e / kL, s = e % kL;
-        float w = 0.f;
-        if (s <= r0 + i) {
-            float x = 0.f;
-#pragma unroll 8
-            for (int a = 0; a < DK; ++a) x = fmaf(A[i * FC::AW + a], B[s * FC::AW + a], x);
-            x *= inv_c;
-            if constexpr (KIND == 2) {
-                w = taylor_n(x, P);
-            } else {
-                float dw = 0.f;
-#pragma unroll 8
-                for (int j = 0; j <= DV; ++j) dw = fmaf(M[i * FC::MW + j], S[s * FC::SW + j], dw);
-                w = dw * taylor_n(x, P - 1) * inv_c;
+    // outputs: a warp takes 4 query rows (broadcast weights), a lane NCOL / 32 columns
+    constexpr int NCOL = KIND == 2 ? DV : DK;
+    constexpr int CPL = (NCOL + 31) / 32;
+    {
+        const int wi = tid / 32, lane = tid % 32;
+        const int i0 = 4 * wi;
+        if (i0 < nr) {
+            float acc[4][CPL];
+#pragma unroll
+            for (int a = 0; a < 4; ++a)
+#pragma unroll
+                for (int cc = 0; cc < CPL; ++cc) acc[a][cc] = 0.f;
+            const int smax = r0 + i0 + 3 < ns - 1 ? r0 + i0 + 3 : ns - 1;
+            for (int s = 0; s <= smax; ++s) {
+                float wv[4];
+#pragma unroll
+                for (int a = 0; a < 4; ++a) wv[a] = Wt[(i0 + a) * FC::WW + s];
+#pragma unroll
+                for (int cc = 0; cc < CPL; ++cc) {
+                    const int col = lane + 32 * cc;
+                    if (col < NCOL) {
+                        const float val = KIND == 2 ? S[s * FC::SW + col] : B[s * FC::AW + col];
+#pragma unroll
+                        for (int a = 0; a < 4; ++a) acc[a][cc] = fmaf(wv[a], val, acc[a][cc]);
+                    }
+                }
+            }
+#pragma unroll
+            for (int a = 0; a < 4; ++a) {
+                const int t = r0 + i0 + a;   // token of the chunk (frame)
+                if (i0 + a >= nr) break;
+                const int64_t f = f0 + t;
+                const int64_t o = REV ? N - 1 - f : f;
+#pragma unroll
+                for (int cc = 0; cc < CPL; ++cc) {
+                    const int col = lane + 32 * cc;
+                    if (col >= NCOL) continue;
+                    float inter;
+                    if constexpr (KIND == 2)   // the prefill scan's sums: quads [BH][nch][DQ][128]
+                        inter = sums[(((bh * nch + c) * sum_quads(DV) + col / 4) * kL + t) * 4 + col % 4];
+                    else                       // the gradient scan's sums [BH][d_K][N]
+                        inter = sums[(bh * DK + col) * N + f];
+                    out[(bh * N + o) * NCOL + col] = inter + acc[a][cc];
+                }
             }
         }
-        Wt[i * FC::WW + s] = w;
-    }
-    __syncthreads();
-    constexpr int NCOL = KIND == 2 ? DV : DK;
-    for (int e = tid; e < nr * NCOL; e += 256) {
-        const int i = e / NCOL, col = e % NCOL;
-        const int t = r0 + i;   // token of the chunk (frame)
-        float acc = 0.f;
-        for (int s = 0; s <= t; ++s)
-            acc = fmaf(Wt[i * FC::WW + s], KIND == 2 ? S[s * FC::SW + col] : B[s * FC::AW + col], acc);
-        const int64_t f = f0 + t;
-        float inter;
-        if constexpr (KIND == 2) {   // the prefill scan's sums: quads [BH][nch][DQ][128]
-            inter = sums[(((bh * nch + c) * sum_quads(DV) + col / 4) * kL + t) * 4 + col % 4];
-        } else {                     // the gradient scan's sums [BH][d_K][N]
-            inter = sums[(bh * DK + col) * N + f];
-        }
-        out[(bh * N + orig(f)) * NCOL + col] = inter + acc;
     }
 }
 

@@ -530,7 +530,8 @@ def _check_grads(sata, oracle_mod, B, H, N, d_K, d_V, P, seed, heads=None):
                                          (64, 64, 4, 130), (16, 32, 3, 65), (12, 8, 2, 50),
                                          (8, 8, 5, 40), (4, 4, 1, 33), (128, 128, 2, 37),
                                          (6, 8, 7, 29), (32, 4, 4, 140), (128, 128, 2, 100),
-                                         (64, 128, 2, 70)])
+                                         (64, 128, 2, 70), (64, 16, 4, 300), (128, 64, 3, 260),
+                                         (32, 64, 4, 290), (64, 32, 1, 200), (16, 16, 2, 400)])
 def test_backward_matches_oracle(sata, oracle_mod, path, d_K, d_V, P, N):
     """auto: the forward and the three gradient scans run on tensor cores for the
     tensor-core shapes with P <= 4; cuda_core: everything on CUDA cores."""
@@ -608,8 +609,11 @@ def test_backward_workload_full_size(sata, oracle_mod, name):
     w = wl.WORKLOADS[name]
     (q, k, v), _ = wl.make_inputs(w)
     dy = wl.cotangent(w)
+    sata.sata_reset_kernel_stats()
     dq, dk, dv = sata.prefill_backward(q.cuda(), k.cuda(), v.cuda(), dy.cuda(), w.P)
     torch.cuda.synchronize()
+    assert sata.sata_sync_status() == 0
+    assert "bwd_tc_scan" in sata.sata_kernel_stats()
     ref = oracle_mod.grad_heads(q, k, v, dy, w.P, heads=list(w.oracle_heads))
     for (b, h), (rq, rk, rv) in ref.items():
         for nm, g, r in (("dq", dq, rq), ("dk", dk, rk), ("dv", dv, rv)):
