@@ -1492,7 +1492,10 @@ const UnitPlan *unit_plan(int D, int P, int NL) {
 // to bound the partial buffer.
 struct Plan {
     const UnitPlan *up = nullptr;
-    int G = 1, nchunks = 0, nc_seg = 0, nseg = 0;
+    int G = 1, nchunks = 0, nc_seg = 0, nseg = 0;   // nc_seg: chunks of the longest segment
+    // host-buffer path: segment starts (chunks) of a non-uniform split, seg_c0[nseg] = nchunks
+    bool profiled = false;
+    int seg_c0[kHostSegments + 1] = {};
     size_t off_stats = 0, off_q16 = 0, off_k16 = 0, off_v16 = 0, off_red = 0, off_part = 0, off_state = 0,
            total = 0;
 };
@@ -1518,6 +1521,23 @@ bool make_plan(int BH, int64_t N, int64_t F, int P, bool need_state, int min_seg
     if (nseg < 1) nseg = 1;
     pl.nc_seg = (int)((pl.nchunks + nseg - 1) / nseg);
     pl.nseg = (pl.nchunks + pl.nc_seg - 1) / pl.nc_seg;
+    if (!deterministic && min_segments == kHostSegments && pl.nchunks >= 16 * kHostSegments) {
+        // Copies pipelined with the kernels: the first segment's inputs and the last one's
+        // output are exposed, so those segments are short.  A segment's inputs copy in about
+        // a third of its compute time and its output in about a quarter, so each segment can
+        // be a few times its predecessor while its inputs still land in time, and the last a
+        // fraction of the one before it.  10 %, 20 %, 55 %, 15 % of the chunks measured best
+        // of the splits tried (uniform quarters: 4 % slower end to end at 65536 tokens).
+        static_assert(kHostSegments == 4, "split profile");
+        const int cum[kHostSegments] = {0, 10, 30, 85};
+        for (int i = 0; i < kHostSegments; ++i) pl.seg_c0[i] = (int)((int64_t)pl.nchunks * cum[i] / 100);
+        pl.seg_c0[kHostSegments] = pl.nchunks;
+        pl.profiled = true;
+        pl.nseg = kHostSegments;
+        pl.nc_seg = 0;
+        for (int i = 0; i < kHostSegments; ++i)
+            if (pl.seg_c0[i + 1] - pl.seg_c0[i] > pl.nc_seg) pl.nc_seg = pl.seg_c0[i + 1] - pl.seg_c0[i];
+    }
     pl.off_stats = 0;
     pl.off_q16 = align256((size_t)BH * 4 * sizeof(float));
     const size_t rows = (size_t)BH * pl.nchunks * kL;   // whole chunks, chunk-interleaved
@@ -1601,8 +1621,9 @@ cudaError_t run(const DeviceBasis &basis, int BH, int64_t N, const void *q, cons
         ~Release() { for (cudaEvent_t x : ev) cudaEventDestroy(x); }
     } release{events};
     for (int s = 0; s < nseg; ++s) {
-        const int c0s = s * pl.nc_seg;
-        const int ncs = (pl.nchunks - c0s < pl.nc_seg) ? pl.nchunks - c0s : pl.nc_seg;
+        const int c0s = pl.profiled ? pl.seg_c0[s] : s * pl.nc_seg;
+        const int ncs = pl.profiled ? pl.seg_c0[s + 1] - c0s
+                                    : ((pl.nchunks - c0s < pl.nc_seg) ? pl.nchunks - c0s : pl.nc_seg);
         const int64_t tok0 = (int64_t)c0s * kL, tok1 = (int64_t)(c0s + ncs) * kL < N ? (int64_t)(c0s + ncs) * kL : N;
         if (io) {   // this segment's inputs: host -> device on the copy stream, compute waits for them
             cudaEvent_t ev;
