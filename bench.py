@@ -8,9 +8,10 @@ One "step" is one causal SATA prefill of the d_K = d_V = 64, P = 4 workload
 in HBM.  Decode is measured beside it on the decode workload (B=64, H=32,
 d_K = d_V = 32, a state built by an 8192-token prefill, then decode steps) and
 reported under "decode", and the backward pass of the prefill (gradients of q,
-k, v on the d = 64, P = 4 head shape over 4096 tokens) under "backward".  For N > 1 (torchrun) every rank runs its own copy of
-the workload on its own GPU (weak scaling, no collective on the data path);
-times are max over ranks.
+k, v on the d = 64, P = 4 head shape over 4096 tokens) under "backward".  For N > 1
+(torchrun) the job has 8N heads and rank r owns heads [8r, 8r + 8) of it, each
+head its own seeded draw (weak scaling: the work per GPU is fixed; no
+collective on the data path); times are max over ranks.
 
 --impl reference times the float64 CPU oracle on a bounded sample of the same
 workload (the only other code in this file that may run the oracle is the
@@ -332,7 +333,9 @@ def main():
     w = wl.WORKLOADS[args.workload]
 
     # ---------------- prefill (headline) ----------------
-    (q, k, v), _ = wl.make_inputs(w)
+    # N ranks: one job of B x (H N) heads, rank r owning heads [H r, H (r + 1)) of every
+    # batch row (each its own seeded draw); no collective on the data path
+    (q, k, v), _ = wl.make_inputs(w, h0=rank * w.H, H_total=w.H * world)
     qd, kd, vd = q.to(dev), k.to(dev), v.to(dev)
     out = torch.empty((w.B, w.H, w.N, w.d_V), dtype=torch.float32, device=dev)
     in_bytes = sum(t.numel() * t.element_size() for t in (q, k, v))
@@ -410,7 +413,8 @@ def main():
         "accumulate": "f32", "data": "synthetic (seeded N(0,1) bf16 inputs; no dataset involved)",
         "config": {"workload": f"{w.name}: B={w.B} H={w.H} N={w.N} d_K={w.d_K} d_V={w.d_V} P={w.P} "
                                f"F={w.F}", "per_rank_batch": w.B, "seq_len": w.N,
-                   "parallelism": f"{world} independent replicas (heads/batches sharded by rank)",
+                   "parallelism": (f"heads sharded: rank r owns heads [{w.H}r, {w.H}(r+1)) of a "
+                                   f"{w.H * world}-head job, no collective") if world > 1 else "one GPU",
                    "l2": f"inputs {in_bytes / 1e6:.0f} MB + output {out_bytes / 1e6:.0f} MB per step > 126 MB L2",
                    "path": args.path},
         "roofline": roof, "gpu_launches": launches, "clocks": clocks, "e2e": e2e, "decode": dec,

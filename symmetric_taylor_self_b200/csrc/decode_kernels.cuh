@@ -69,10 +69,13 @@ struct TableBasis {
 
 // Basis derived arithmetically (P <= 4): each thread unranks its first feature
 // and steps through kFG / kThreads consecutive ones.  Index d stands for the
-// constant 1 (the padding that makes every feature a triple).
+// constant 1 (the padding that makes every feature a triple).  ic[p] = c^-p,
+// each rounded once from double on the host; a coefficient is 1/prod(mult!) times
+// ic[p], so it can differ from the table path's (one rounding of the product) in
+// its last bit.
 struct DerivedBasis {
     int d;
-    float inv_c;
+    float ic[4];
 
     // Padded triple (a, b, l) of feature f in basis order, and its degree p.
     __device__ static void unrank(int64_t f, int d, int &a, int &b, int &l, int &p) {
@@ -120,12 +123,12 @@ struct DerivedBasis {
     }
 
     // alpha_p * C_p = C_p / (p! c^p) for the triple, C_p = p! / prod(mult!).
-    __device__ static float coef(int a, int b, int l, int p, float inv_c) {
+    __device__ static float coef(int a, int b, int l, int p, const float (&ic)[4]) {
         if (p == 0) return 1.f;
-        if (p == 1) return inv_c;
-        if (p == 2) return (b == l ? 0.5f : 1.f) * inv_c * inv_c;
+        if (p == 1) return ic[1];
+        if (p == 2) return (b == l ? 0.5f : 1.f) * ic[2];
         const float inv_mult = (a == b && b == l) ? (1.f / 6.f) : ((a == b || b == l) ? 0.5f : 1.f);
-        return inv_mult * inv_c * inv_c * inv_c;
+        return inv_mult * ic[3];
     }
 
     __device__ void fill(int64_t f0, int nf, const float *xq, const float *xk, float *phik,
@@ -138,7 +141,7 @@ struct DerivedBasis {
         for (int u = 0; u < kPerThread && fl + u < nf; ++u) {
             if (u > 0) next(d, a, b, l, p);
             phik[fl + u] = xk[a] * xk[b] * xk[l];
-            aq[fl + u] = coef(a, b, l, p, inv_c) * (xq[a] * xq[b] * xq[l]);
+            aq[fl + u] = coef(a, b, l, p, ic) * (xq[a] * xq[b] * xq[l]);
         }
     }
 };

@@ -27,6 +27,7 @@
 //     in a context before any stream capture.
 //   - The kernels are the ordinary decode step's (decode_kernels.cuh) with the
 //     basis derived in registers, so the two entry points compute alike.
+#include <cmath>
 #include <cstdint>
 #include <mutex>
 
@@ -111,7 +112,8 @@ extern "C" int sata_decode_step_static(sata_state *st, const void *q, const void
     float *scratch = nullptr;
     cudaError_t e = static_scratch(&scratch);
     if (e == cudaSuccess) {
-        const dec::DerivedBasis db{st->d_K, 1.0f / sqrtf((float)st->d_K)};
+        const double c = sqrt((double)st->d_K);
+        const dec::DerivedBasis db{st->d_K, {1.f, (float)(1.0 / c), (float)(1.0 / (c * c)), (float)(1.0 / (c * c * c))}};
         e = dec::launch_any(d_V, db, BH, st->d_K, F, st->S, st->Z, q, k, v, out, scratch,
                             (cudaStream_t)st->stream, false);
     }

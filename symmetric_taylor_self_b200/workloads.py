@@ -78,13 +78,15 @@ WORKLOADS = {
 }
 
 
-def head_seed(w: Workload, b: int, h: int) -> int:
-    return w.seed * 2 ** 20 + b * w.H + h
+def head_seed(w: Workload, b: int, h: int, H_total: int | None = None) -> int:
+    """Seed of head (b, h) of the workload, or of a job of H_total heads per batch
+    row made of several copies of its head shape (head h of H_total)."""
+    return w.seed * 2 ** 20 + b * (w.H if H_total is None else H_total) + h
 
 
-def head_inputs(w: Workload, b: int, h: int, dtype=torch.bfloat16):
+def head_inputs(w: Workload, b: int, h: int, dtype=torch.bfloat16, H_total: int | None = None):
     """q, k, v for one head over all N + steps tokens, as ``dtype`` CPU tensors."""
-    g = torch.Generator("cpu").manual_seed(head_seed(w, b, h))
+    g = torch.Generator("cpu").manual_seed(head_seed(w, b, h, H_total))
     T = w.N + w.steps
     q = torch.randn(T, w.d_K, generator=g)
     k = torch.randn(T, w.d_K, generator=g)
@@ -95,9 +97,11 @@ def head_inputs(w: Workload, b: int, h: int, dtype=torch.bfloat16):
     return q.to(dtype), k.to(dtype), v.to(dtype)
 
 
-def make_inputs(w: Workload, dtype=torch.bfloat16):
+def make_inputs(w: Workload, dtype=torch.bfloat16, h0: int = 0, H_total: int | None = None):
     """Prefill tensors [B, H, N, d] and, for decode workloads, per-step tensors
-    [steps, B, H, d] (empty when steps == 0).  CPU, ``dtype``."""
+    [steps, B, H, d] (empty when steps == 0).  CPU, ``dtype``.  With H_total, the
+    H heads are heads h0 .. h0 + H - 1 of a job of H_total heads per batch row (the
+    shard one rank of a head-sharded job owns); by default the workload itself."""
     T = w.N + w.steps
     q = torch.empty(w.B, w.H, T, w.d_K, dtype=dtype)
     k = torch.empty(w.B, w.H, T, w.d_K, dtype=dtype)
@@ -105,7 +109,7 @@ def make_inputs(w: Workload, dtype=torch.bfloat16):
 
     def fill(bh):
         b, h = divmod(bh, w.H)
-        q[b, h], k[b, h], v[b, h] = head_inputs(w, b, h, dtype)
+        q[b, h], k[b, h], v[b, h] = head_inputs(w, b, h0 + h, dtype, H_total)
 
     # heads are independent draws (one generator each): fill them on host threads
     with ThreadPoolExecutor(max_workers=min(16, len(os.sched_getaffinity(0)))) as ex:
