@@ -1,8 +1,8 @@
 """Multi-rank host logic on CPU: gloo ranks on 127.0.0.1.
 
-bench.py: on GPUs every rank runs its own copy of the workload (heads are
-independent, no collective on the data path); the only cross-rank steps are
-the barrier and the max-over-ranks time.  The sequence split (seqsplit.py)
+bench.py: on GPUs rank r owns heads [H r, H (r + 1)) of a job of H x world
+heads (heads are independent, no collective on the data path); the only
+cross-rank steps are the barrier and the max-over-ranks time.  The sequence split (seqsplit.py)
 has one real exchange, the all-gather of segment states and their prefix sum.
 """
 import os
@@ -224,3 +224,20 @@ def test_sequence_split_single_rank_without_process_group():
         yr, _, Sr, Zr = oracle.scan(q[0, h], k[0, h], v[0, h], 4)
         np.testing.assert_allclose(y[0, h].numpy(), yr, rtol=1e-12, atol=1e-12)
         np.testing.assert_allclose(st["S"][0, h].numpy(), Sr, rtol=1e-12, atol=1e-12)
+
+
+def test_rank_head_shards_partition_one_job():
+    """The shards the ranks draw (workloads.make_inputs with h0, H_total) are the
+    heads of one larger job: concatenated in rank order they equal the inputs of
+    the same workload with H x world heads."""
+    import dataclasses
+    sys.path.insert(0, ROOT)
+    from symmetric_taylor_self_b200 import workloads as wl
+    w = dataclasses.replace(wl.WORKLOADS["prefill_d16"], N=256)
+    world = 3
+    shards = [wl.make_inputs(w, h0=r * w.H, H_total=w.H * world)[0] for r in range(world)]
+    big = dataclasses.replace(w, H=w.H * world)
+    whole = wl.make_inputs(big)[0]
+    for i in range(3):
+        assert torch.equal(torch.cat([sh[i] for sh in shards], dim=1), whole[i])
+    assert not torch.equal(shards[0][0], shards[1][0])
