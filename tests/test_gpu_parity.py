@@ -228,6 +228,35 @@ def test_prefill_d64_internal_segments(sata, oracle_mod, mode):
         assert np.abs(Zg - Z).max() / np.abs(Z).max() <= TOL
 
 
+def test_prefill_host_profiled_segments(sata, oracle_mod):
+    """The host-buffer entry point over 65 chunks splits the sequence into four
+    unequal segments (10 %, 20 %, 55 %, 15 % of the chunks: 6, 13, 36 and 10
+    here), carrying the state between them: every token of two heads and their
+    final state against the oracle, and the output against the device-buffer
+    call within the tolerance (the segments prescale their rows separately)."""
+    _set_path(sata, "auto")
+    B, H, N, d = 1, 2, 8300, 32
+    q, k, v = wl.random_inputs(B, H, N, d, d, seed=6500)
+    st = sata.State(B, H, d, d, 4)
+    stream = torch.cuda.Stream()
+    st.set_stream(stream)
+    yh = torch.empty((B, H, N, d), dtype=torch.float32).pin_memory()
+    sata.sata_reset_kernel_stats()
+    sata.sata_prefill_host(q.pin_memory(), k.pin_memory(), v.pin_memory(), yh, B, H, N, d, d, 4, st.st, stream)
+    stream.synchronize()
+    assert sata.sata_sync_status(stream) == 0
+    assert sata.sata_kernel_stats()["tc_scan"][0] == 4
+    ref = _oracle_heads(oracle_mod, q, k, v, 4, [(0, 0), (0, 1)])
+    _check_heads(yh, ref, what=f"host segments d={d} N={N}")
+    for (b, h), (_, _, S, Z) in ref.items():
+        Sg, Zg = st.S[b, h].double().cpu().numpy(), st.Z[b, h].double().cpu().numpy()
+        assert np.abs(Sg - S).max() / np.abs(S).max() <= TOL
+        assert np.abs(Zg - Z).max() / np.abs(Z).max() <= TOL
+    yd = sata.prefill(q.cuda(), k.cuda(), v.cuda(), P=4).cpu()
+    err, _, _ = token_rel_err(yh.double().numpy().reshape(-1, d), yd.double().numpy().reshape(-1, d))
+    assert err <= TOL
+
+
 def test_prefill_d64_long_head(sata, oracle_mod):
     """One d = 64 head over 8192 tokens against the oracle's recurrence: every
     token and the final state."""
