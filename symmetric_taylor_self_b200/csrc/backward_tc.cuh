@@ -196,12 +196,18 @@ bwd_tc_r_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__rest
 
 // Buffers of the gradient scans' operands (prescaled fp16, chunk-interleaved as the
 // prefill's rows: chunk_rows).  Normal order: q, k, v.  Reversed order (frame token
-// t' = N - 1 - t): q, k, g = r[:d_V] and rho = r[d_V] ([BH][nch][128]); u = [v | 1]
-// reversed in fp32 [BH][N][bwd_rs] (the dk readout's multipliers).
+// t' = N - 1 - t): q, k, g = r[:d_V] and rho = r[d_V] ([BH][nch][128]).  The readouts'
+// multipliers in fp32, chunk-interleaved float4 quads (bwd_rs / 4 per token): r in time
+// order (dq) and u = [v | 1] reversed (dk).
 struct BwdImages {
     __half *q, *k, *v, *qr, *kr, *gr, *rho;
-    float *ur;
+    float *rq, *uq;
 };
+
+// Quad j of a multiplier row of frame token f into its chunk-interleaved place.
+__device__ __forceinline__ void put_quad(float *img, int64_t bh, int nch, int mq, int64_t f, int j, float4 x) {
+    reinterpret_cast<float4 *>(img)[((bh * nch + f / kL) * mq + j) * kL + f % kL] = x;
+}
 
 // Piece j (8 values) of a row into a chunk-interleaved image at frame token f.
 template <int D>
@@ -258,7 +264,7 @@ bwd_tc_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
         put_piece<DK>(im.kr, bh, nch, tr, j, b);
     }
     const float *rr = r + row * bwd_rs(DV);
-    float *ur = im.ur + (bh * N + tr) * bwd_rs(DV);
+    constexpr int MQ = bwd_rs(DV) / 4;
 #pragma unroll 2
     for (int j = 0; j < DV / 8; ++j) {
         const uint4 w = __ldg(reinterpret_cast<const uint4 *>(v + row * DV) + j);
@@ -266,15 +272,21 @@ bwd_tc_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
         const float4 g0 = __ldg(reinterpret_cast<const float4 *>(rr) + 2 * j);
         const float4 g1 = __ldg(reinterpret_cast<const float4 *>(rr) + 2 * j + 1);
         put_piece<DV>(im.gr, bh, nch, tr, j, f32x8_to_half_scaled(g0, g1, sr));
+        put_quad(im.rq, bh, nch, MQ, t, 2 * j, g0);
+        put_quad(im.rq, bh, nch, MQ, t, 2 * j + 1, g1);
         const uint32_t x[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-            reinterpret_cast<float2 *>(ur)[4 * j + i] =
-                make_float2(__uint_as_float(x[i] << 16), __uint_as_float(x[i] & 0xFFFF0000u));
+        put_quad(im.uq, bh, nch, MQ, tr, 2 * j,
+                 make_float4(__uint_as_float(x[0] << 16), __uint_as_float(x[0] & 0xFFFF0000u),
+                             __uint_as_float(x[1] << 16), __uint_as_float(x[1] & 0xFFFF0000u)));
+        put_quad(im.uq, bh, nch, MQ, tr, 2 * j + 1,
+                 make_float4(__uint_as_float(x[2] << 16), __uint_as_float(x[2] & 0xFFFF0000u),
+                             __uint_as_float(x[3] << 16), __uint_as_float(x[3] & 0xFFFF0000u)));
     }
-    ur[DV] = 1.f;
 #pragma unroll
-    for (int j = DV + 1; j < bwd_rs(DV); ++j) ur[j] = 0.f;
+    for (int j = DV / 4; j < MQ; ++j) {   // the last quads: r[d_V] (and zero padding); u's 1
+        put_quad(im.rq, bh, nch, MQ, t, j, __ldg(reinterpret_cast<const float4 *>(rr) + j));
+        put_quad(im.uq, bh, nch, MQ, tr, j, make_float4(j == DV / 4 ? 1.f : 0.f, 0.f, 0.f, 0.f));
+    }
     im.rho[(bh * nch + tr / kL) * kL + tr % kL] = __float2half_rn(__ldg(rr + DV) * sr);
 }
 
@@ -489,7 +501,7 @@ bwd_tc_finish_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *_
 // recomputed forward, then the operand images and sums; y, den and r follow it.
 struct BwdTcLayout {
     size_t fwd = 0, front = 0, off_mx = 0, off_stn = 0, off_str = 0, off_img = 0, off_sq = 0, off_sk = 0,
-           off_sv = 0, off_ur = 0, off_y = 0, off_den = 0, off_r = 0, total = 0;
+           off_sv = 0, off_ur = 0, off_rq = 0, off_y = 0, off_den = 0, off_r = 0, total = 0;
     size_t img_q = 0, img_v = 0, img_rho = 0;
 };
 
@@ -511,7 +523,8 @@ bool bwd_tc_layout(int BH, int64_t N, int64_t F, int P, BwdTcLayout &L) {
     L.off_sk = L.off_sq + align256((size_t)BH * DK * N * 4);
     L.off_sv = L.off_sk + align256((size_t)BH * DK * N * 4);
     L.off_ur = L.off_sv + align256((size_t)BH * nch * sum_quads(DV) * kL * 16);
-    const size_t mine = L.off_ur + align256((size_t)BH * N * bwd_rs(DV) * 4);
+    L.off_rq = L.off_ur + align256(rows * bwd_rs(DV) * 4);
+    const size_t mine = L.off_rq + align256(rows * bwd_rs(DV) * 4);
     L.front = L.fwd > mine ? L.fwd : mine;
     L.off_y = align256(L.front);
     L.off_den = L.off_y + align256((size_t)BH * N * DV * 4);
@@ -553,7 +566,8 @@ cudaError_t bwd_tc_run(const DeviceBasis &basis, int BH, int64_t N, const void *
     im.v = (__half *)(w + L.off_img + 4 * L.img_q);
     im.gr = (__half *)(w + L.off_img + 4 * L.img_q + L.img_v);
     im.rho = (__half *)(w + L.off_img + 4 * L.img_q + 2 * L.img_v);
-    im.ur = (float *)(w + L.off_ur);
+    im.uq = (float *)(w + L.off_ur);
+    im.rq = (float *)(w + L.off_rq);
     float *sq = (float *)(w + L.off_sq), *sk = (float *)(w + L.off_sk), *sv = (float *)(w + L.off_sv);
 
     const dim3 rgrid((unsigned)((N + 127) / 128), (unsigned)BH);
@@ -618,8 +632,8 @@ cudaError_t bwd_tc_run(const DeviceBasis &basis, int BH, int64_t N, const void *
         sp.stats = st_n;
         sp.zval16 = nullptr;
         sp.zscaled = 0;
-        sp.mult = r;
-        sp.mult_stride = bwd_rs(DV);
+        sp.mult = im.rq;
+        sp.mult_quads = bwd_rs(DV) / 4;
         sp.sums_jac = sq;
         launch_begin(kBwdTcScan, stream);
         tc_scan_kernel<DK, DV, true><<<BH * sp.G, kScanThreads, C::SMEM, stream>>>(sp);
@@ -632,7 +646,7 @@ cudaError_t bwd_tc_run(const DeviceBasis &basis, int BH, int64_t N, const void *
         sp.stats = st_r;
         sp.zval16 = im.rho;
         sp.zscaled = 1;
-        sp.mult = im.ur;
+        sp.mult = im.uq;
         sp.sums_jac = sk;
         launch_begin(kBwdTcScan, stream);
         tc_scan_kernel<DK, DV, true><<<BH * sp.G, kScanThreads, C::SMEM, stream>>>(sp);

@@ -141,12 +141,13 @@ struct ScanParams {
     int64_t wait_ns;
     // gradient scans (JAC kernels) only: Z-column values per token (prescaled fp16, chunk-
     // interleaved [BH][nch][128]; null: the constant 1), whether the Z columns carry the
-    // column prescale, the readout's per-token multipliers (fp32 [BH][N][mult_stride], true
-    // frame) and the sums [BH][d_K][N] the drain adds into
+    // column prescale, the readout's per-token multipliers (fp32, true frame, chunk-
+    // interleaved float4 quads: quad j of token t of chunk c of head bh at element
+    // ((bh nch + c) mult_quads + j) 128 + t) and the sums [BH][d_K][N] the drain adds into
     const __half *zval16 = nullptr;
     int zscaled = 0;
     const float *mult = nullptr;
-    int mult_stride = 0;
+    int mult_quads = 0;
     float *sums_jac = nullptr;
 };
 
@@ -654,13 +655,14 @@ __device__ __forceinline__ void q_drain_jac(const ScanParams &p, int64_t bh, int
     const float upv = pow2f_sat(sg + ev), upz = pow2f_sat(sg + (p.zscaled ? ev : 0));
     const int64_t tok = (int64_t)(p.c0 + cl) * kL + t;
     const bool valid = tok < p.N;
-    const float *m = p.mult + (bh * p.N + (valid ? tok : 0)) * p.mult_stride;
+    // 32 consecutive tokens read 512 contiguous bytes per quad
+    const float4 *m4 = reinterpret_cast<const float4 *>(p.mult) + ((int64_t)bh * p.nch + p.c0 + cl) * p.mult_quads * kL + t;
     float acc[NL], accz[NL];
     {
         uint32_t rz[16];
         tc_ld16(tm + C::COL_R + nl * DV, rz);
         tc_wait_ld();
-        const float mz = valid ? __ldg(m + DV) : 0.f;
+        const float mz = valid ? __ldg(m4 + (DV / 4) * kL).x : 0.f;
 #pragma unroll
         for (int s = 0; s < NL; ++s) {
             acc[s] = 0.f;
@@ -673,8 +675,7 @@ __device__ __forceinline__ void q_drain_jac(const ScanParams &p, int64_t bh, int
         float mv[GW];
 #pragma unroll
         for (int i4 = 0; i4 < GW / 4; ++i4) {
-            const float4 x = valid ? __ldg(reinterpret_cast<const float4 *>(m + GW * g) + i4)
-                                   : make_float4(0.f, 0.f, 0.f, 0.f);
+            const float4 x = valid ? __ldg(m4 + (GW / 4 * g + i4) * kL) : make_float4(0.f, 0.f, 0.f, 0.f);
             mv[4 * i4] = x.x;
             mv[4 * i4 + 1] = x.y;
             mv[4 * i4 + 2] = x.z;
