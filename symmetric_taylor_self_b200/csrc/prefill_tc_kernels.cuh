@@ -509,26 +509,33 @@ template <int D>
 __device__ __forceinline__ void prep_rows(const __nv_bfloat16 *__restrict__ x, __half *__restrict__ x16,
                                           const float *__restrict__ stats, int which, int BH, int64_t N,
                                           int64_t t0, int64_t t1, int nch) {
-    const int64_t per_head = (t1 - t0) * (D / 8);
-    const int64_t total = (int64_t)BH * per_head;
+    // one thread per token row: its D/8 pieces are one contiguous read, and for each piece
+    // consecutive tokens store consecutive 16-byte elements
+    const int64_t ntok = t1 - t0;
+    const int64_t total = (int64_t)BH * ntok;
     for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < total; e += (int64_t)gridDim.x * blockDim.x) {
-        const int64_t bh = e / per_head, rem = e % per_head;
-        const int64_t tok = t0 + rem % (t1 - t0);   // tokens fastest: coalesced stores
-        const int j = (int)(rem / (t1 - t0));
+        const int64_t bh = e / ntok;
+        const int64_t tok = t0 + (e - bh * ntok);
         const HeadExp he = head_exps(stats + bh * 4);
         const int ex = which == 0 ? he.eq : (which == 1 ? he.ek : he.ev);
         const float sc = pow2f(-ex);
-        const uint4 u = __ldg(reinterpret_cast<const uint4 *>(x + (bh * N + tok) * D) + j);
-        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-        uint32_t o[4];
+        const uint4 *src = reinterpret_cast<const uint4 *>(x + (bh * N + tok) * D);
+        uint4 *dst = reinterpret_cast<uint4 *>(x16) + (bh * nch + tok / kL) * (D / 8) * kL + tok % kL;
+        uint4 u[D / 8];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const float lo = __uint_as_float(w[i] << 16), hi = __uint_as_float(w[i] & 0xFFFF0000u);
-            const __half2 h = __floats2half2_rn(lo * sc, hi * sc);
-            o[i] = *reinterpret_cast<const uint32_t *>(&h);
+        for (int j = 0; j < D / 8; ++j) u[j] = __ldg(src + j);
+#pragma unroll
+        for (int j = 0; j < D / 8; ++j) {
+            const uint32_t w[4] = {u[j].x, u[j].y, u[j].z, u[j].w};
+            uint32_t o[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const float lo = __uint_as_float(w[i] << 16), hi = __uint_as_float(w[i] & 0xFFFF0000u);
+                const __half2 h = __floats2half2_rn(lo * sc, hi * sc);
+                o[i] = *reinterpret_cast<const uint32_t *>(&h);
+            }
+            dst[j * kL] = make_uint4(o[0], o[1], o[2], o[3]);
         }
-        uint4 *dst = reinterpret_cast<uint4 *>(x16) + ((bh * nch + tok / kL) * (D / 8) + j) * kL + tok % kL;
-        *dst = make_uint4(o[0], o[1], o[2], o[3]);
     }
 }
 template <int DK, int DV>
@@ -1646,7 +1653,7 @@ cudaError_t run(const DeviceBasis &basis, int BH, int64_t N, const void *q, cons
             tc_stats_kernel<DK, DV><<<(unsigned)((int64_t)bx * BH), 256, 0, stream>>>(qb, kb, vb, stats, N, tok0,
                                                                                     tok1, bx);
             if ((e = cudaGetLastError()) == cudaSuccess) {
-                const int64_t nwork = (int64_t)BH * ntok * (DK / 8);
+                const int64_t nwork = (int64_t)BH * ntok;   // one thread per token row
                 const int pgrid = (int)((nwork + 255) / 256 < 148 * 16 ? (nwork + 255) / 256 : 148 * 16);
                 tc_prep_kernel<DK, DV><<<pgrid, 256, 0, stream>>>(qb, kb, vb, stats, q16, k16, v16, BH, N, tok0, tok1,
                                                                    pl.nchunks, flags);
