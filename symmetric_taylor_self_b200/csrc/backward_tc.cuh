@@ -1,5 +1,5 @@
 // Backward pass of the prefill on tensor cores: the three gradient scans run as
-// tcgen05 scans of the prefill's kind (prefill_tc_kernels.cuh), the intra-chunk
+// tcgen05 scans of the prefill's kind (prefill_tc_scan.cuh), the intra-chunk
 // pairs in a CUDA-core finish kernel.
 //
 // The method's pages define no backward pass ([CC-TAYLOR] "Self-attention at

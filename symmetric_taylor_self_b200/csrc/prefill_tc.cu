@@ -1,4 +1,5 @@
-// Tensor-core prefill: shape dispatch to the instances of prefill_tc_kernels.cuh
+// Tensor-core prefill and backward: shape dispatch to the instances of the prefill_tc_*.cuh
+// and backward_tc.cuh templates
 // (one prefill_tc_*.cu file per group of shapes, compiled in parallel).
 #include "prefill_tc_shapes.h"
 #include "sata_internal.h"
