@@ -560,7 +560,8 @@ def _check_grads(sata, oracle_mod, B, H, N, d_K, d_V, P, seed, heads=None):
                                          (8, 8, 5, 40), (4, 4, 1, 33), (128, 128, 2, 37),
                                          (6, 8, 7, 29), (32, 4, 4, 140), (128, 128, 2, 100),
                                          (64, 128, 2, 70), (64, 16, 4, 300), (128, 64, 3, 260),
-                                         (32, 64, 4, 290), (64, 32, 1, 200), (16, 16, 2, 400)])
+                                         (32, 64, 4, 290), (64, 32, 1, 200), (16, 16, 2, 400),
+                                         (128, 128, 4, 160), (128, 64, 4, 140)])
 def test_backward_matches_oracle(sata, oracle_mod, path, d_K, d_V, P, N):
     """auto: the forward and the three gradient scans run on tensor cores for the
     tensor-core shapes with P <= 4; cuda_core: everything on CUDA cores."""
