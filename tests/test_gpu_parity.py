@@ -257,6 +257,25 @@ def test_prefill_host_profiled_segments(sata, oracle_mod):
     assert err <= TOL
 
 
+@pytest.mark.parametrize("d_K,d_V,N", [(64, 32, 700), (128, 128, 300), (32, 64, 520)])
+def test_prefill_host_other_shapes(sata, oracle_mod, d_K, d_V, N):
+    """The host-buffer entry point on the other tensor-core shapes (four token
+    segments with the state carried between them): every token of both heads
+    against the oracle."""
+    _set_path(sata, "auto")
+    B, H = 1, 2
+    q, k, v = wl.random_inputs(B, H, N, d_K, d_V, seed=6600 + d_K + d_V)
+    stream = torch.cuda.Stream()
+    yh = torch.empty((B, H, N, d_V), dtype=torch.float32).pin_memory()
+    sata.sata_reset_kernel_stats()
+    sata.sata_prefill_host(q.pin_memory(), k.pin_memory(), v.pin_memory(), yh, B, H, N, d_K, d_V, 4, None, stream)
+    stream.synchronize()
+    assert sata.sata_sync_status(stream) == 0
+    assert sata.sata_kernel_stats()["tc_scan"][0] == 4
+    ref = _oracle_heads(oracle_mod, q, k, v, 4, [(0, 0), (0, 1)])
+    _check_heads(yh, ref, what=f"host d_K={d_K} d_V={d_V} N={N}")
+
+
 def test_prefill_d64_long_head(sata, oracle_mod):
     """One d = 64 head over 8192 tokens against the oracle's recurrence: every
     token and the final state."""
