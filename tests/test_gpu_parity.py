@@ -259,9 +259,9 @@ def test_prefill_host_profiled_segments(sata, oracle_mod):
 
 @pytest.mark.parametrize("d_K,d_V,N", [(64, 32, 700), (128, 128, 300), (32, 64, 520)])
 def test_prefill_host_other_shapes(sata, oracle_mod, d_K, d_V, N):
-    """The host-buffer entry point on the other tensor-core shapes (four token
-    segments with the state carried between them): every token of both heads
-    against the oracle."""
+    """The host-buffer entry point on the other tensor-core shapes (three token
+    segments at these lengths, the state carried between them): every token of
+    both heads against the oracle."""
     _set_path(sata, "auto")
     B, H = 1, 2
     q, k, v = wl.random_inputs(B, H, N, d_K, d_V, seed=6600 + d_K + d_V)
@@ -271,7 +271,7 @@ def test_prefill_host_other_shapes(sata, oracle_mod, d_K, d_V, N):
     sata.sata_prefill_host(q.pin_memory(), k.pin_memory(), v.pin_memory(), yh, B, H, N, d_K, d_V, 4, None, stream)
     stream.synchronize()
     assert sata.sata_sync_status(stream) == 0
-    assert sata.sata_kernel_stats()["tc_scan"][0] == 4
+    assert sata.sata_kernel_stats()["tc_scan"][0] == 3
     ref = _oracle_heads(oracle_mod, q, k, v, 4, [(0, 0), (0, 1)])
     _check_heads(yh, ref, what=f"host d_K={d_K} d_V={d_V} N={N}")
 
