@@ -39,6 +39,7 @@ namespace sata {
 namespace {
 
 __host__ __device__ constexpr int bwd_rs(int DV) { return (DV + 1 + 3) / 4 * 4; }   // r, u row stride
+constexpr int kRHead = 14;   // r's prescaled maximum: below 2^14 (fp16 holds up to 65504)
 
 // Unit plan of a gradient scan: per pair tile holding a pair of degree <= P - 2,
 // the d_K slot indices i in groups of NL; coefficient C/p'! of the pair (0 on
@@ -244,16 +245,21 @@ bwd_tc_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
     const int64_t bh = blockIdx.y;
     const float fq = __uint_as_float(mx[bh * 4 + 0]), fk = __uint_as_float(mx[bh * 4 + 1]),
                 fv = __uint_as_float(mx[bh * 4 + 2]), fr = __uint_as_float(mx[bh * 4 + 3]);
+    // r is prescaled so that its largest value lies in [2^(kRHead-1), 2^kRHead) rather than
+    // below 1: one token with a tiny denominator can make |r| span many octaves, and below 1
+    // the rest would fall into fp16's subnormal range (the scans then widen their operand
+    // bound by kRHead octaves)
+    const float fr_s = fr * pow2f(-kRHead);
     if (blockIdx.x == 0 && threadIdx.x == 0) {
         st_n[bh * 4 + 0] = fq; st_n[bh * 4 + 1] = fk; st_n[bh * 4 + 2] = fv; st_n[bh * 4 + 3] = 0.f;
-        st_r[bh * 4 + 0] = fk; st_r[bh * 4 + 1] = fq; st_r[bh * 4 + 2] = fr; st_r[bh * 4 + 3] = 0.f;
+        st_r[bh * 4 + 0] = fk; st_r[bh * 4 + 1] = fq; st_r[bh * 4 + 2] = fr_s; st_r[bh * 4 + 3] = 0.f;
         if (!(fq <= FLT_MAX && fk <= FLT_MAX && fv <= FLT_MAX && fr <= FLT_MAX)) atomicExch(flags + kFlagRange, 1);
     }
     const int64_t t = (int64_t)blockIdx.x * 128 + threadIdx.x;
     if (t >= N) return;
     const int64_t row = bh * N + t, tr = N - 1 - t;
     const float sq = pow2f(-scale_exp(fq)), sk = pow2f(-scale_exp(fk)), sv = pow2f(-scale_exp(fv)),
-                sr = pow2f(-scale_exp(fr));
+                sr = pow2f(-scale_exp(fr_s));
 #pragma unroll 2
     for (int j = 0; j < DK / 8; ++j) {
         const uint4 a = bf16x8_to_half_scaled(__ldg(reinterpret_cast<const uint4 *>(q + row * DK) + j), sq);
@@ -647,6 +653,7 @@ cudaError_t bwd_tc_run(const DeviceBasis &basis, int BH, int64_t N, const void *
         sp.zval16 = im.rho;
         sp.zscaled = 1;
         sp.mult = im.uq;
+        sp.col_head = kRHead;
         sp.sums_jac = sk;
         launch_begin(kBwdTcScan, stream);
         tc_scan_kernel<DK, DV, true><<<BH * sp.G, kScanThreads, C::SMEM, stream>>>(sp);
@@ -667,6 +674,7 @@ cudaError_t bwd_tc_run(const DeviceBasis &basis, int BH, int64_t N, const void *
         sp.v16 = im.gr;
         sp.stats = st_r;
         sp.part = sv;
+        sp.col_head = kRHead;
         launch_begin(kBwdTcScan, stream);
         tc_scan_kernel<DK, DV><<<BH * sp.G, kScanThreads, C::SMEM, stream>>>(sp);
         launch_end(kBwdTcScan, stream);

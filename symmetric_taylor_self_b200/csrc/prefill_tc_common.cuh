@@ -153,6 +153,10 @@ struct ScanParams {
     int zscaled = 0;
     const float *mult = nullptr;
     int mult_quads = 0;
+    // exponent headroom of the column values (the values' rows are prescaled so that the
+    // largest is below 2^col_head rather than 1: the gradient scans' r, whose range can span
+    // more octaves than fp16 resolves below 1); widens the readout operand's bound
+    int col_head = 0;
     float *sums_jac = nullptr;
 };
 
@@ -296,16 +300,17 @@ __device__ __forceinline__ int state_sigma_rows(int cl, int e_ms, int e_row) {
     const int s = eb + e_row - 15;
     return s < -120 ? -120 : (s > 120 ? 120 : s);
 }
-__device__ __forceinline__ int state_sigma(int cl, int e_ms, int E, int P, int lc) {
+// col_head: exponent of the largest prescaled column value (0: every value below 1).
+__device__ __forceinline__ int state_sigma(int cl, int e_ms, int E, int P, int lc, int col_head = 0) {
     const int r = (P - 1) * (E - lc);
-    return state_sigma_rows(cl, e_ms, r > 0 ? r : 0);
+    return state_sigma_rows(cl, e_ms, (r > 0 ? r : 0) + col_head);
 }
 // The same for a gradient scan: a pair row of degree p' <= P - 2 carries
 // C/p'! c^-(p'+1) 2^(p' E + e_k) <= 2^(p' (E - lc) + e_k - lc) (the slot index is a
 // key-side factor only; the derivative's 1/c is in the row).
-__device__ __forceinline__ int jac_sigma(int cl, int E, int ek, int P, int lc) {
+__device__ __forceinline__ int jac_sigma(int cl, int E, int ek, int P, int lc, int col_head = 0) {
     const int r = (P - 2) * (E - lc);
-    return state_sigma_rows(cl, -1000, (r > 0 ? r : 0) + ek - lc);
+    return state_sigma_rows(cl, -1000, (r > 0 ? r : 0) + ek - lc + col_head);
 }
 
 struct Waiter {

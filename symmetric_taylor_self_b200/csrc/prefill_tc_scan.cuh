@@ -30,7 +30,7 @@ __device__ __forceinline__ void q_drain(const ScanParams &p, int64_t bh, int64_t
     using C = Cfg<DK, DV>;
     constexpr int NL = C::NL;
     tc_after();
-    const int sg = state_sigma(cl, e_ms, E, p.P, p.lc);
+    const int sg = state_sigma(cl, e_ms, E, p.P, p.lc, p.col_head);
     const float upv = pow2f_sat(sg + ev), upz = pow2f_sat(sg);
     const bool valid = (int64_t)(p.c0 + cl) * kL + t < p.N;
     constexpr int DQ = sum_quads(DV);
@@ -96,7 +96,7 @@ __device__ __forceinline__ void q_drain_jac(const ScanParams &p, int64_t bh, int
     using C = Cfg<DK, DV>;
     constexpr int NL = C::NL;
     tc_after();
-    const int sg = jac_sigma(cl, E, ek, p.P, p.lc);
+    const int sg = jac_sigma(cl, E, ek, p.P, p.lc, p.col_head);
     const float upv = pow2f_sat(sg + ev), upz = pow2f_sat(sg + (p.zscaled ? ev : 0));
     const int64_t tok = (int64_t)(p.c0 + cl) * kL + t;
     const bool valid = tok < p.N;
@@ -455,7 +455,7 @@ __global__ void __launch_bounds__(kScanThreads, 1) tc_scan_kernel(const ScanPara
             // B double buffer: the readout of chunk cl-2 has read it
             if (cl >= 2 && !(ok = W.wait(BAR(C::B_BSE + b), ((cl >> 1) - 1) & 1))) break;
             tc_after();
-            const int sg = JAC ? jac_sigma(cl, E, he.ek, p.P, p.lc) : state_sigma(cl, e_ms, E, p.P, p.lc);
+            const int sg = JAC ? jac_sigma(cl, E, he.ek, p.P, p.lc, p.col_head) : state_sigma(cl, e_ms, E, p.P, p.lc, p.col_head);
             float sc[NL];
 #pragma unroll
             for (int s = 0; s < NL; ++s) sc[s] = cf[s] * pow2f_sat(pe[s] - sg);
