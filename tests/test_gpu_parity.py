@@ -593,6 +593,37 @@ def test_backward_matches_oracle(sata, oracle_mod, path, d_K, d_V, P, N):
     _set_path(sata, "auto")
 
 
+_T4_ROOT = -1.5960716379833215   # the real root of 1 + x + x^2/2 + x^3/6
+
+
+@pytest.mark.parametrize("path", list(PATHS))
+@pytest.mark.parametrize("d_K,d_V", [(128, 64), (128, 128), (64, 64), (32, 32)])
+def test_backward_near_root_denominator(sata, oracle_mod, path, d_K, d_V):
+    """Head 1's first token has q_0 . k_0 / c just above the real root of the
+    P = 4 series, so its denominator T_4(x) is about 0.01 and its cotangent
+    dy / den is ~100x every other token's: the gradients of the other tokens
+    must keep their accuracy beside it."""
+    _set_path(sata, path)
+    N, P = 600, 4
+    q, k, v = wl.random_inputs(1, 2, N, d_K, d_V, seed=5400 + d_K + d_V)
+    dy = wl.random_cotangent(1, 2, N, d_V, seed=5401)
+    k0 = k[0, 1, 0].double()
+    alpha = (_T4_ROOT + 0.015) * math.sqrt(d_K) / float(k0 @ k0)
+    q[0, 1, 0] = (alpha * k0).to(q.dtype)
+    x = float(q[0, 1, 0].double() @ k0) / math.sqrt(d_K)
+    den0 = 1 + x + x * x / 2 + x ** 3 / 6
+    assert 2e-3 < den0 < 3e-2
+    dq, dk, dv = sata.prefill_backward(q.cuda(), k.cuda(), v.cuda(), dy.cuda(), P)
+    torch.cuda.synchronize()
+    assert sata.sata_sync_status() == 0
+    ref = oracle_mod.grad_heads(q, k, v, dy, P, heads=[(0, 0), (0, 1)])
+    for (b, h), (rq, rk, rv) in ref.items():
+        for name, g, r in (("dq", dq, rq), ("dk", dk, rk), ("dv", dv, rv)):
+            err = tensor_rel_err(g[b, h].double().cpu().numpy(), r)
+            assert err <= TOL, f"{name} head {(b, h)} d_K={d_K} d_V={d_V}: {err:.3e}"
+    _set_path(sata, "auto")
+
+
 def test_backward_single_token(sata):
     """N = 1: y_0 = v_0 whatever q and k are, so dv = dy and dq = dk = 0 (up to
     rounding: dw = g.v - g.y cancels)."""
