@@ -39,7 +39,7 @@ namespace sata {
 namespace {
 
 __host__ __device__ constexpr int bwd_rs(int DV) { return (DV + 1 + 3) / 4 * 4; }   // r, u row stride
-constexpr int kRHead = 14;   // r's prescaled maximum: below 2^14 (fp16 holds up to 65504)
+constexpr int kRHead = 14;   // r's prescaled maximum: below 2^14 (an fp16 operand holds up to 65504)
 
 // Unit plan of a gradient scan: per pair tile holding a pair of degree <= P - 2,
 // the d_K slot indices i in groups of NL; coefficient C/p'! of the pair (0 on
@@ -233,22 +233,23 @@ __device__ __forceinline__ uint4 f32x8_to_half_scaled(float4 a, float4 b, float 
                       *reinterpret_cast<const uint32_t *>(&h2), *reinterpret_cast<const uint32_t *>(&h3));
 }
 
-// One thread per token row: the operand images of the three scans, and (block 0 of
-// each head) their per-head maxima rows: st_n = (|q|, |k|, |v|, 0) for dq, st_r =
-// (|k|, |q|, |r|, 0) for dk and dv.
+// One thread per token row: the operand images of the three scans, (block 0 of each
+// head) their per-head maxima rows: st_n = (|q|, |k|, |v|, 0) for dq, st_r = (|k|, |q|,
+// |r|, 0) for dk and dv, and the per-chunk maxima of the prescaled r (g and -(g.y)) in
+// the reversed frame, cm[head][chunk] (zeroed before; fp32 bit patterns).
 template <int DK, int DV>
 __global__ void __launch_bounds__(128)
 bwd_tc_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k,
                    const __nv_bfloat16 *__restrict__ v, const float *__restrict__ r,
                    const unsigned int *__restrict__ mx, float *__restrict__ st_n, float *__restrict__ st_r,
-                   BwdImages im, int64_t N, int nch, int *flags) {
+                   unsigned int *__restrict__ cm, BwdImages im, int64_t N, int nch, int *flags) {
     const int64_t bh = blockIdx.y;
     const float fq = __uint_as_float(mx[bh * 4 + 0]), fk = __uint_as_float(mx[bh * 4 + 1]),
                 fv = __uint_as_float(mx[bh * 4 + 2]), fr = __uint_as_float(mx[bh * 4 + 3]);
     // r is prescaled so that its largest value lies in [2^(kRHead-1), 2^kRHead) rather than
     // below 1: one token with a tiny denominator can make |r| span many octaves, and below 1
-    // the rest would fall into fp16's subnormal range (the scans then widen their operand
-    // bound by kRHead octaves)
+    // the rest would fall into fp16's subnormal range.  The dk and dv scans bound their
+    // readout operand by the per-chunk maxima cm instead of by this largest value.
     const float fr_s = fr * pow2f(-kRHead);
     if (blockIdx.x == 0 && threadIdx.x == 0) {
         st_n[bh * 4 + 0] = fq; st_n[bh * 4 + 1] = fk; st_n[bh * 4 + 2] = fv; st_n[bh * 4 + 3] = 0.f;
@@ -271,6 +272,7 @@ bwd_tc_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
     }
     const float *rr = r + row * bwd_rs(DV);
     constexpr int MQ = bwd_rs(DV) / 4;
+    float rmax = 0.f;
 #pragma unroll 2
     for (int j = 0; j < DV / 8; ++j) {
         const uint4 w = __ldg(reinterpret_cast<const uint4 *>(v + row * DV) + j);
@@ -278,6 +280,8 @@ bwd_tc_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
         const float4 g0 = __ldg(reinterpret_cast<const float4 *>(rr) + 2 * j);
         const float4 g1 = __ldg(reinterpret_cast<const float4 *>(rr) + 2 * j + 1);
         put_piece<DV>(im.gr, bh, nch, tr, j, f32x8_to_half_scaled(g0, g1, sr));
+        rmax = fmaxf(rmax, fmaxf(fmaxf(fmaxf(fabsf(g0.x), fabsf(g0.y)), fmaxf(fabsf(g0.z), fabsf(g0.w))),
+                                 fmaxf(fmaxf(fabsf(g1.x), fabsf(g1.y)), fmaxf(fabsf(g1.z), fabsf(g1.w)))));
         put_quad(im.rq, bh, nch, MQ, t, 2 * j, g0);
         put_quad(im.rq, bh, nch, MQ, t, 2 * j + 1, g1);
         const uint32_t x[4] = {w.x, w.y, w.z, w.w};
@@ -293,7 +297,11 @@ bwd_tc_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
         put_quad(im.rq, bh, nch, MQ, t, j, __ldg(reinterpret_cast<const float4 *>(rr) + j));
         put_quad(im.uq, bh, nch, MQ, tr, j, make_float4(j == DV / 4 ? 1.f : 0.f, 0.f, 0.f, 0.f));
     }
-    im.rho[(bh * nch + tr / kL) * kL + tr % kL] = __float2half_rn(__ldg(rr + DV) * sr);
+    const float rho = __ldg(rr + DV);
+    im.rho[(bh * nch + tr / kL) * kL + tr % kL] = __float2half_rn(rho * sr);
+    rmax = fmaxf(rmax, fabsf(rho)) * sr;
+    if (!(rmax <= FLT_MAX)) rmax = FLT_MAX;   // a non-finite r has raised the range flag
+    atomicMax(cm + bh * nch + tr / kL, __float_as_uint(rmax));
 }
 
 // T_n(x) = sum_{p<n} x^p / p! (0 for n = 0), Horner from the top term.
@@ -506,7 +514,7 @@ bwd_tc_finish_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *_
 // Workspace of the tensor-core backward.  The front region first serves the
 // recomputed forward, then the operand images and sums; y, den and r follow it.
 struct BwdTcLayout {
-    size_t fwd = 0, front = 0, off_mx = 0, off_stn = 0, off_str = 0, off_img = 0, off_sq = 0, off_sk = 0,
+    size_t fwd = 0, front = 0, off_mx = 0, off_stn = 0, off_str = 0, off_cm = 0, off_img = 0, off_sq = 0, off_sk = 0,
            off_sv = 0, off_ur = 0, off_rq = 0, off_y = 0, off_den = 0, off_r = 0, total = 0;
     size_t img_q = 0, img_v = 0, img_rho = 0;
 };
@@ -524,7 +532,8 @@ bool bwd_tc_layout(int BH, int64_t N, int64_t F, int P, BwdTcLayout &L) {
     L.off_mx = 0;
     L.off_stn = align256((size_t)BH * 16);
     L.off_str = L.off_stn + align256((size_t)BH * 16);
-    L.off_img = L.off_str + align256((size_t)BH * 16);
+    L.off_cm = L.off_str + align256((size_t)BH * 16);
+    L.off_img = L.off_cm + align256((size_t)BH * nch * 4);
     L.off_sq = L.off_img + 4 * L.img_q + 2 * L.img_v + L.img_rho;
     L.off_sk = L.off_sq + align256((size_t)BH * DK * N * 4);
     L.off_sv = L.off_sk + align256((size_t)BH * DK * N * 4);
@@ -564,6 +573,7 @@ cudaError_t bwd_tc_run(const DeviceBasis &basis, int BH, int64_t N, const void *
 
     unsigned int *mx = (unsigned int *)(w + L.off_mx);
     float *st_n = (float *)(w + L.off_stn), *st_r = (float *)(w + L.off_str);
+    unsigned int *cm = (unsigned int *)(w + L.off_cm);
     BwdImages im;
     im.q = (__half *)(w + L.off_img);
     im.k = (__half *)(w + L.off_img + L.img_q);
@@ -579,12 +589,13 @@ cudaError_t bwd_tc_run(const DeviceBasis &basis, int BH, int64_t N, const void *
     const dim3 rgrid((unsigned)((N + 127) / 128), (unsigned)BH);
     launch_begin(kBwdTcPrep, stream);
     e = cudaMemsetAsync(mx, 0, (size_t)BH * 16, stream);
+    if (e == cudaSuccess) e = cudaMemsetAsync(cm, 0, (size_t)BH * nch * 4, stream);
     if (e == cudaSuccess) {
         bwd_tc_r_kernel<DK, DV><<<rgrid, 128, 0, stream>>>(qb, kb, vb, dy, y, den, r, mx, N);
         e = cudaGetLastError();
     }
     if (e == cudaSuccess) {
-        bwd_tc_prep_kernel<DK, DV><<<rgrid, 128, 0, stream>>>(qb, kb, vb, r, mx, st_n, st_r, im, N, nch, flags);
+        bwd_tc_prep_kernel<DK, DV><<<rgrid, 128, 0, stream>>>(qb, kb, vb, r, mx, st_n, st_r, cm, im, N, nch, flags);
         e = cudaGetLastError();
     }
     launch_end(kBwdTcPrep, stream);
@@ -653,7 +664,7 @@ cudaError_t bwd_tc_run(const DeviceBasis &basis, int BH, int64_t N, const void *
         sp.zval16 = im.rho;
         sp.zscaled = 1;
         sp.mult = im.uq;
-        sp.col_head = kRHead;
+        sp.colmax = (const float *)cm;   // columns g and -(g.y)
         sp.sums_jac = sk;
         launch_begin(kBwdTcScan, stream);
         tc_scan_kernel<DK, DV, true><<<BH * sp.G, kScanThreads, C::SMEM, stream>>>(sp);
@@ -674,7 +685,8 @@ cudaError_t bwd_tc_run(const DeviceBasis &basis, int BH, int64_t N, const void *
         sp.v16 = im.gr;
         sp.stats = st_r;
         sp.part = sv;
-        sp.col_head = kRHead;
+        sp.colmax = (const float *)cm;   // columns g, and the Z columns' 1
+        sp.colmax_floor = 1.f;
         launch_begin(kBwdTcScan, stream);
         tc_scan_kernel<DK, DV><<<BH * sp.G, kScanThreads, C::SMEM, stream>>>(sp);
         launch_end(kBwdTcScan, stream);

@@ -134,7 +134,8 @@ struct ScanParams {
     const int32_t *unit_l;           // [G][NL]
     const float *unit_coef;          // [G][NL][128] C/p! of feature (pair, l), 0 if none
     const int32_t *unit_fidx;        // [G][NL][128] basis index of feature (pair, l), -1 if none
-    float *S, *Z;                    // state in/out (true frame)
+    float *S, *Z;
+    int s_ld = 0, s_off = 0;         // S rows s_ld values apart (0: DV), this call's columns from s_off                    // state in/out (true frame)
     float *part;                     // sums [BH][nc][DV+1][128] (red_atomic) or [BH][G][nc][DV+1][128]
     int red_atomic;
     int *flags;
@@ -153,10 +154,12 @@ struct ScanParams {
     int zscaled = 0;
     const float *mult = nullptr;
     int mult_quads = 0;
-    // exponent headroom of the column values (the values' rows are prescaled so that the
-    // largest is below 2^col_head rather than 1: the gradient scans' r, whose range can span
-    // more octaves than fp16 resolves below 1); widens the readout operand's bound
-    int col_head = 0;
+    // per-chunk maxima of the prescaled column values ([BH][nch], this scan's frame), or null:
+    // every column value is at most 1.  With them the readout operand's bound sums the
+    // maxima of the chunks so far instead of counting their tokens at the largest value (a
+    // gradient scan's r can hold one token hundreds of times the others)
+    const float *colmax = nullptr;
+    float colmax_floor = 0.f;   // the least column maximum (1: Z columns that carry 1)
     float *sums_jac = nullptr;
 };
 
@@ -288,29 +291,39 @@ __device__ __forceinline__ HeadExp head_exps(const float *st) {
     return HeadExp{scale_exp(st[0]), scale_exp(st[1]), scale_exp(st[2])};
 }
 // Exponent sigma_c of the readout operand's scale before chunk cl of this call:
-// |S'| < 2^e_ms + 128 cl + 1 (every prescaled feature and value is at most 1 in
-// magnitude, e_ms bounds the prescaled incoming state), and a degree-p row carries
-// C/p! c^-p 2^(p E) <= 2^(p (E - lc)) <= 2^max(0, (P-1)(E - lc)) (C/p! <= 1, lc =
+// |S'| < 2^e_ms + 2^e_tok with 2^e_tok > 128 cl + 1 (every prescaled feature and value is
+// at most 1 in magnitude; e_ms bounds the prescaled incoming state), or, with per-chunk
+// maxima m_c of the column values, 2^e_tok > 128 sum_{c < cl} m_c + 1; and a degree-p row
+// carries C/p! c^-p 2^(p E) <= 2^(p (E - lc)) <= 2^max(0, (P-1)(E - lc)) (C/p! <= 1, lc =
 // floor(log2 c)), so |B| < 2^15 for every row.  The bound is tight for the rows that
 // reach it; a looser one would push the small rows of B into fp16's subnormal range.
-__device__ __forceinline__ int state_sigma_rows(int cl, int e_ms, int e_row) {
-    const uint32_t tok = (uint32_t)cl * kL + 1u;
-    const int e_tok = 32 - __clz(tok);
+__device__ __forceinline__ int tok_exp(int cl) { return 32 - __clz((uint32_t)cl * kL + 1u); }
+__device__ __forceinline__ int tok_exp_sum(float cum) {   // 128 cum + 1 < 2^e (a normal float >= 1)
+    return (int)((__float_as_uint(fmaf(128.f, cum, 1.f)) >> 23) & 0xFFu) - 126;
+}
+__device__ __forceinline__ int state_sigma_rows(int e_tok, int e_ms, int e_row) {
     const int eb = (e_ms > e_tok ? e_ms : e_tok) + 1;
     const int s = eb + e_row - 15;
     return s < -120 ? -120 : (s > 120 ? 120 : s);
 }
-// col_head: exponent of the largest prescaled column value (0: every value below 1).
-__device__ __forceinline__ int state_sigma(int cl, int e_ms, int E, int P, int lc, int col_head = 0) {
+__device__ __forceinline__ int state_sigma(int e_tok, int e_ms, int E, int P, int lc) {
     const int r = (P - 1) * (E - lc);
-    return state_sigma_rows(cl, e_ms, (r > 0 ? r : 0) + col_head);
+    return state_sigma_rows(e_tok, e_ms, r > 0 ? r : 0);
 }
 // The same for a gradient scan: a pair row of degree p' <= P - 2 carries
 // C/p'! c^-(p'+1) 2^(p' E + e_k) <= 2^(p' (E - lc) + e_k - lc) (the slot index is a
 // key-side factor only; the derivative's 1/c is in the row).
-__device__ __forceinline__ int jac_sigma(int cl, int E, int ek, int P, int lc, int col_head = 0) {
+__device__ __forceinline__ int jac_sigma(int e_tok, int E, int ek, int P, int lc) {
     const int r = (P - 2) * (E - lc);
-    return state_sigma_rows(cl, -1000, (r > 0 ? r : 0) + ek - lc + col_head);
+    return state_sigma_rows(e_tok, -1000, (r > 0 ? r : 0) + ek - lc);
+}
+// The column bound's exponent before chunk cl (cum: the maxima of chunks < cl summed in
+// chunk order; every role sums them the same way, so all agree on sigma).
+__device__ __forceinline__ int col_exp(const ScanParams &p, int cl, float cum) {
+    return p.colmax ? tok_exp_sum(cum) : tok_exp(cl);
+}
+__device__ __forceinline__ float col_max(const ScanParams &p, int64_t bh, int cl) {
+    return fmaxf(p.colmax[bh * p.nch + p.c0 + cl], p.colmax_floor);
 }
 
 struct Waiter {

@@ -73,7 +73,7 @@ __global__ void __launch_bounds__(128)
 tc_finish_kernel(const __half *__restrict__ q16, const __half *__restrict__ k16, const __half *__restrict__ v16,
                  const float *__restrict__ stats, const float *__restrict__ red, float *__restrict__ out,
                  float *__restrict__ den_out, int c0, int nc, int nch, int64_t N, int P, float inv_c, int *flags,
-                 int64_t wait_ns) {
+                 int64_t wait_ns, int dvs, int voff) {
     using F = FinCfg<DK, DV>;
     constexpr int NV = F::NV;
     extern __shared__ uint8_t fraw[];
@@ -252,10 +252,10 @@ tc_finish_kernel(const __half *__restrict__ q16, const __half *__restrict__ k16,
     tc_before();
     __syncthreads();
     if (ok) {
-        float4 *o4 = reinterpret_cast<float4 *>(out + (bh * N + t0) * DV);
         for (int e = tid; e < nt * (DV / 4); e += 128) {
             const int r = e / (DV / 4), c4 = e % (DV / 4);
-            o4[e] = *reinterpret_cast<const float4 *>(stg + r * F::STG + 4 * c4);
+            reinterpret_cast<float4 *>(out + (bh * N + t0 + r) * dvs + voff)[c4] =
+                *reinterpret_cast<const float4 *>(stg + r * F::STG + 4 * c4);
         }
     }
     if (warp == 0) {

@@ -211,13 +211,19 @@ cudaError_t copy_rows(void *dst, const void *src, int BH, int64_t N, int64_t t0,
                              (size_t)(t1 - t0) * width * elem, BH, kind, s);
 }
 
+// dvs, voff: v, out and a caller's S have rows of dvs values, of which this call covers
+// the DV columns from voff on (dvs = DV, voff = 0: whole rows).  The caller's Z is
+// written whole by every such call.  Not with host buffers.
 template <int DK, int DV>
 cudaError_t run(const DeviceBasis &basis, int BH, int64_t N, const void *q, const void *k, const void *v,
                 float *out, float *S, float *Z, bool state_in, void *ws, size_t ws_bytes, int *flags,
-                cudaStream_t stream, const HostIO *io, float *den_out) {
+                cudaStream_t stream, const HostIO *io, float *den_out, int dvs = DV, int voff = 0) {
     using C = Cfg<DK, DV>;
     const int64_t F = basis.F;
     const bool own_state = (S == nullptr);
+    if (dvs < DV || voff < 0 || voff + DV > dvs || dvs % 8 != 0 || voff % 8 != 0 || (io && dvs != DV))
+        return cudaErrorInvalidValue;
+    const int s_ld = own_state ? DV : dvs, s_off = own_state ? 0 : voff;   // the state's rows
     const int min_seg = io ? kHostSegments : 1;
     const bool det = g_opt_deterministic != 0;
     Plan pl;
@@ -295,17 +301,17 @@ cudaError_t run(const DeviceBasis &basis, int BH, int64_t N, const void *q, cons
             if (bx < 1) bx = 1;
             launch_begin(kTcPrep, stream);
             tc_stats_kernel<DK, DV><<<(unsigned)((int64_t)bx * BH), 256, 0, stream>>>(qb, kb, vb, stats, N, tok0,
-                                                                                    tok1, bx);
+                                                                                    tok1, bx, dvs);
             if ((e = cudaGetLastError()) == cudaSuccess) {
                 const int64_t nwork = (int64_t)BH * ntok;   // one thread per token row
                 const int pgrid = (int)((nwork + 255) / 256 < 148 * 16 ? (nwork + 255) / 256 : 148 * 16);
                 tc_prep_kernel<DK, DV><<<pgrid, 256, 0, stream>>>(qb, kb, vb, stats, q16, k16, v16, BH, N, tok0, tok1,
-                                                                   pl.nchunks, flags);
+                                                                   pl.nchunks, flags, dvs, voff);
             }
             launch_end(kTcPrep, stream);
             if (e != cudaSuccess || (e = cudaGetLastError()) != cudaSuccess) return e;
             if (load_state) {
-                tc_state_stats_kernel<<<dim3(BH, 8), 256, 0, stream>>>(S, Z, stats, F, DV);
+                tc_state_stats_kernel<<<dim3(BH, 8), 256, 0, stream>>>(S, Z, stats, F, s_ld);
                 if ((e = cudaGetLastError()) != cudaSuccess) return e;
             }
         }
@@ -322,6 +328,8 @@ cudaError_t run(const DeviceBasis &basis, int BH, int64_t N, const void *q, cons
         sp.unit_fidx = (const int32_t *)(tab + up.off_fidx);
         sp.S = S;
         sp.Z = Z;
+        sp.s_ld = s_ld;
+        sp.s_off = s_off;
         if (!det && (e = cudaMemsetAsync(red, 0, (size_t)BH * ncs * sum_quads(DV) * kL * 16, stream)) !=
                         cudaSuccess)
             return e;
@@ -356,7 +364,8 @@ cudaError_t run(const DeviceBasis &basis, int BH, int64_t N, const void *q, cons
         }
         launch_begin(kTcFinish, stream);
         tc_finish_kernel<DK, DV><<<(int)((int64_t)BH * ncs), 128, FinCfg<DK, DV>::SMEM, stream>>>(
-            q16, k16, v16, stats, red, out, den_out, c0s, ncs, pl.nchunks, N, basis.P, inv_c, flags, wait_ns);
+            q16, k16, v16, stats, red, out, den_out, c0s, ncs, pl.nchunks, N, basis.P, inv_c, flags, wait_ns, dvs,
+            voff);
         launch_end(kTcFinish, stream);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
         if (io) {   // this segment's output: device -> host on the second copy stream
@@ -385,8 +394,9 @@ cudaError_t run(const DeviceBasis &basis, int BH, int64_t N, const void *q, cons
     cudaError_t tc_run_##a##_##b(const DeviceBasis &basis, int BH, int64_t N, const void *q, const void *k,   \
                                  const void *v, float *out, float *S, float *Z, bool state_in, void *ws,       \
                                  size_t ws_bytes, int *flags, cudaStream_t stream, const HostIO *io,          \
-                                 float *den_out) {                                                            \
-        return run<a, b>(basis, BH, N, q, k, v, out, S, Z, state_in, ws, ws_bytes, flags, stream, io, den_out);  \
+                                 float *den_out, int dvs, int voff) {                                         \
+        return run<a, b>(basis, BH, N, q, k, v, out, S, Z, state_in, ws, ws_bytes, flags, stream, io, den_out,   \
+                         dvs, voff);                                                                          \
     }
 
 }  // namespace sata

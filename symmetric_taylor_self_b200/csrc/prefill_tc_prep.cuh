@@ -11,7 +11,9 @@ namespace {
 
 // Per-head maxima of |q|, |k|, |v| over tokens [t0, t1): max of the bf16 bit
 // patterns without sign (a NaN input orders above +inf), then one atomic max per
-// block on the fp32 bit pattern (non-negative floats order like their bits).
+// block on the fp32 bit pattern (non-negative floats order like their bits).  v's
+// rows are dvs values apart (dvs >= DV when a call covers a column range of wider
+// rows); the maximum is taken over the whole rows, a valid bound for every range.
 __device__ __forceinline__ uint32_t absmax_bits(uint4 u, uint32_t m) {
     m = __vmaxu2(m, u.x & 0x7FFF7FFFu);
     m = __vmaxu2(m, u.y & 0x7FFF7FFFu);
@@ -26,14 +28,14 @@ template <int DK, int DV>
 __global__ void __launch_bounds__(256)
 tc_stats_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k,
                 const __nv_bfloat16 *__restrict__ v, float *__restrict__ stats, int64_t N, int64_t t0, int64_t t1,
-                int bpb) {
+                int bpb, int dvs) {
     const int64_t bh = blockIdx.x / bpb;   // bpb blocks per head
     const int bx = blockIdx.x % bpb;
     uint32_t mq = 0, mk = 0, mv = 0;
-    const int64_t nqk = (t1 - t0) * (DK / 8), nv = (t1 - t0) * (DV / 8);
+    const int64_t nqk = (t1 - t0) * (DK / 8), nv = (t1 - t0) * (dvs / 8);
     const uint4 *q4 = reinterpret_cast<const uint4 *>(q + (bh * N + t0) * DK);
     const uint4 *k4 = reinterpret_cast<const uint4 *>(k + (bh * N + t0) * DK);
-    const uint4 *v4 = reinterpret_cast<const uint4 *>(v + (bh * N + t0) * DV);
+    const uint4 *v4 = reinterpret_cast<const uint4 *>(v + (bh * N + t0) * dvs);
     for (int64_t e = (int64_t)bx * 256 + threadIdx.x; e < nqk; e += (int64_t)bpb * 256) {
         mq = absmax_bits(__ldg(q4 + e), mq);
         mk = absmax_bits(__ldg(k4 + e), mk);
@@ -55,11 +57,12 @@ tc_stats_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__rest
 
 // Prescaled fp16 token rows of tokens [t0, t1): q16 = q 2^-e_q, k16 = k 2^-e_k,
 // v16 = v 2^-e_v (exact scalings by powers of two; every value below 1).  A head
-// whose inputs are not finite raises the range flag (its outputs are NaN).
+// whose inputs are not finite raises the range flag (its outputs are NaN).  Source
+// rows are ld values apart, the D values taken from column off on.
 template <int D>
 __device__ __forceinline__ void prep_rows(const __nv_bfloat16 *__restrict__ x, __half *__restrict__ x16,
                                           const float *__restrict__ stats, int which, int BH, int64_t N,
-                                          int64_t t0, int64_t t1, int nch) {
+                                          int64_t t0, int64_t t1, int nch, int ld, int off) {
     // one thread per token row: its D/8 pieces are one contiguous read, and for each piece
     // consecutive tokens store consecutive 16-byte elements
     const int64_t ntok = t1 - t0;
@@ -70,7 +73,7 @@ __device__ __forceinline__ void prep_rows(const __nv_bfloat16 *__restrict__ x, _
         const HeadExp he = head_exps(stats + bh * 4);
         const int ex = which == 0 ? he.eq : (which == 1 ? he.ek : he.ev);
         const float sc = pow2f(-ex);
-        const uint4 *src = reinterpret_cast<const uint4 *>(x + (bh * N + tok) * D);
+        const uint4 *src = reinterpret_cast<const uint4 *>(x + (bh * N + tok) * ld + off);
         uint4 *dst = reinterpret_cast<uint4 *>(x16) + (bh * nch + tok / kL) * (D / 8) * kL + tok % kL;
         uint4 u[D / 8];
 #pragma unroll
@@ -94,17 +97,18 @@ __global__ void __launch_bounds__(256)
 tc_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k,
                const __nv_bfloat16 *__restrict__ v, const float *__restrict__ stats, __half *__restrict__ q16,
                __half *__restrict__ k16, __half *__restrict__ v16, int BH, int64_t N, int64_t t0, int64_t t1,
-               int nch, int *flags) {
+               int nch, int *flags, int dvs, int voff) {
     if (blockIdx.x == 0)
         for (int bh = threadIdx.x; bh < BH; bh += blockDim.x)
             if (!(stats[bh * 4] <= FLT_MAX && stats[bh * 4 + 1] <= FLT_MAX && stats[bh * 4 + 2] <= FLT_MAX))
                 atomicExch(flags + kFlagRange, 1);
-    prep_rows<DK>(q, q16, stats, 0, BH, N, t0, t1, nch);
-    prep_rows<DK>(k, k16, stats, 1, BH, N, t0, t1, nch);
-    prep_rows<DV>(v, v16, stats, 2, BH, N, t0, t1, nch);
+    prep_rows<DK>(q, q16, stats, 0, BH, N, t0, t1, nch, DK, 0);
+    prep_rows<DK>(k, k16, stats, 1, BH, N, t0, t1, nch, DK, 0);
+    prep_rows<DV>(v, v16, stats, 2, BH, N, t0, t1, nch, dvs, voff);
 }
 
-// max |S|, |Z| of each head of an incoming state -> stats[bh][3]
+// max |S|, |Z| of each head of an incoming state -> stats[bh][3] (S rows of DV values: the
+// whole rows when a call covers a column range of them)
 __global__ void tc_state_stats_kernel(const float *__restrict__ S, const float *__restrict__ Z,
                                       float *__restrict__ stats, int64_t F, int DV) {
     const int64_t bh = blockIdx.x;

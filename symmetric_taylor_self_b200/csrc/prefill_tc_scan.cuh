@@ -25,12 +25,12 @@ __device__ __forceinline__ void fetch_row(const __half *x16, const ScanParams &p
 // unit's partial).  Arrives on rf_bar once every column is read.
 template <int DK, int DV>
 __device__ __forceinline__ void q_drain(const ScanParams &p, int64_t bh, int64_t part_base, int nl, int e_ms, int E,
-                                        int ev, int cl, int t, int lane, uint32_t tm, uint32_t rf_bar,
+                                        int ev, int cl, int e_tok, int t, int lane, uint32_t tm, uint32_t rf_bar,
                                         const float (&qv)[Cfg<DK, DV>::NL]) {
     using C = Cfg<DK, DV>;
     constexpr int NL = C::NL;
     tc_after();
-    const int sg = state_sigma(cl, e_ms, E, p.P, p.lc, p.col_head);
+    const int sg = state_sigma(e_tok, e_ms, E, p.P, p.lc);
     const float upv = pow2f_sat(sg + ev), upz = pow2f_sat(sg);
     const bool valid = (int64_t)(p.c0 + cl) * kL + t < p.N;
     constexpr int DQ = sum_quads(DV);
@@ -92,11 +92,11 @@ __device__ __forceinline__ void q_drain(const ScanParams &p, int64_t bh, int64_t
 // is read.
 template <int DK, int DV>
 __device__ __forceinline__ void q_drain_jac(const ScanParams &p, int64_t bh, int nl, int E, int ek, int ev, int cl,
-                                            int t, int lane, uint32_t tm, uint32_t rf_bar, const int *sl) {
+                                            int e_tok, int t, int lane, uint32_t tm, uint32_t rf_bar, const int *sl) {
     using C = Cfg<DK, DV>;
     constexpr int NL = C::NL;
     tc_after();
-    const int sg = jac_sigma(cl, E, ek, p.P, p.lc, p.col_head);
+    const int sg = jac_sigma(e_tok, E, ek, p.P, p.lc);
     const float upv = pow2f_sat(sg + ev), upz = pow2f_sat(sg + (p.zscaled ? ev : 0));
     const int64_t tok = (int64_t)(p.c0 + cl) * kL + t;
     const bool valid = tok < p.N;
@@ -347,6 +347,7 @@ __global__ void __launch_bounds__(kScanThreads, 1) tc_scan_kernel(const ScanPara
         const int64_t part_base = p.red_atomic ? (int64_t)bh * p.nc : ((int64_t)bh * p.G + u) * p.nc;
         uint32_t pq[64], xl[NL];
         float qlp[NL];
+        float cum = 0.f;   // column maxima of the chunks before the one drained next
         bool ok = true;
         if (p.nc > 0) {
             uint32_t x[C::XW];
@@ -363,11 +364,14 @@ __global__ void __launch_bounds__(kScanThreads, 1) tc_scan_kernel(const ScanPara
             __syncwarp();
             if (lane == 0) mbar_arrive(BAR(C::B_AQF));
             if (cl > 0) {
+                const int et = col_exp(p, cl - 1, cum);
                 if constexpr (JAC)
-                    q_drain_jac<DK, DV>(p, bh, nl, E, he.ek, he.ev, cl - 1, t, lane, tmem + lane_off, BAR(C::B_RF), sl);
+                    q_drain_jac<DK, DV>(p, bh, nl, E, he.ek, he.ev, cl - 1, et, t, lane, tmem + lane_off, BAR(C::B_RF),
+                                        sl);
                 else
-                    q_drain<DK, DV>(p, bh, part_base, nl, e_ms, E, he.ev, cl - 1, t, lane, tmem + lane_off,
+                    q_drain<DK, DV>(p, bh, part_base, nl, e_ms, E, he.ev, cl - 1, et, t, lane, tmem + lane_off,
                                     BAR(C::B_RF), qlp);
+                if (p.colmax) cum += col_max(p, bh, cl - 1);
             }
 #pragma unroll
             for (int s = 0; s < NL; ++s) qlp[s] = h_lo(xl[s]);
@@ -380,11 +384,13 @@ __global__ void __launch_bounds__(kScanThreads, 1) tc_scan_kernel(const ScanPara
             }
         }
         if (ok && p.nc > 0 && W.wait(BAR(C::B_RD), (p.nc - 1) & 1)) {
+            const int et = col_exp(p, p.nc - 1, cum);
             if constexpr (JAC)
-                q_drain_jac<DK, DV>(p, bh, nl, E, he.ek, he.ev, p.nc - 1, t, lane, tmem + lane_off, BAR(C::B_RF), sl);
+                q_drain_jac<DK, DV>(p, bh, nl, E, he.ek, he.ev, p.nc - 1, et, t, lane, tmem + lane_off, BAR(C::B_RF),
+                                    sl);
             else
-                q_drain<DK, DV>(p, bh, part_base, nl, e_ms, E, he.ev, p.nc - 1, t, lane, tmem + lane_off, BAR(C::B_RF),
-                                qlp);
+                q_drain<DK, DV>(p, bh, part_base, nl, e_ms, E, he.ev, p.nc - 1, et, t, lane, tmem + lane_off,
+                                BAR(C::B_RF), qlp);
         }
         tc_before();
     } else {
@@ -410,6 +416,7 @@ __global__ void __launch_bounds__(kScanThreads, 1) tc_scan_kernel(const ScanPara
         constexpr int NG = C::NG;
         const int ngu = NU / 16;
         const int ngv = nl * DV / 16;   // groups of V columns; group ngv holds the Z columns (and padding)
+        float cum = 0.f;                // column maxima of the chunks before cl
         bool ok = true;
         if (p.load_state) {   // incoming state -> TMEM (prescaled frame)
             // a V group is 16 contiguous columns of one feature's S row (four 16-byte loads);
@@ -422,8 +429,8 @@ __global__ void __launch_bounds__(kScanThreads, 1) tc_scan_kernel(const ScanPara
                         const int sv = (16 * g) / DV;
                         const int f = seli(fi, sv);
                         const float sc = pow2f_sat(-(seli(dg, sv) * he.ek + he.ev));
-                        const float4 *src = reinterpret_cast<const float4 *>(p.S + (bh * p.F + (f >= 0 ? f : 0)) * DV +
-                                                                             (16 * g) % DV);
+                        const float4 *src = reinterpret_cast<const float4 *>(
+                            p.S + (bh * p.F + (f >= 0 ? f : 0)) * (p.s_ld > 0 ? p.s_ld : DV) + p.s_off + (16 * g) % DV);
 #pragma unroll
                         for (int j = 0; j < 4; ++j) {
                             const float4 x = f >= 0 ? src[j] : make_float4(0.f, 0.f, 0.f, 0.f);
@@ -455,7 +462,9 @@ __global__ void __launch_bounds__(kScanThreads, 1) tc_scan_kernel(const ScanPara
             // B double buffer: the readout of chunk cl-2 has read it
             if (cl >= 2 && !(ok = W.wait(BAR(C::B_BSE + b), ((cl >> 1) - 1) & 1))) break;
             tc_after();
-            const int sg = JAC ? jac_sigma(cl, E, he.ek, p.P, p.lc, p.col_head) : state_sigma(cl, e_ms, E, p.P, p.lc, p.col_head);
+            if (p.colmax && cl > 0) cum += col_max(p, bh, cl - 1);
+            const int et = col_exp(p, cl, cum);
+            const int sg = JAC ? jac_sigma(et, E, he.ek, p.P, p.lc) : state_sigma(et, e_ms, E, p.P, p.lc);
             float sc[NL];
 #pragma unroll
             for (int s = 0; s < NL; ++s) sc[s] = cf[s] * pow2f_sat(pe[s] - sg);
@@ -517,7 +526,8 @@ __global__ void __launch_bounds__(kScanThreads, 1) tc_scan_kernel(const ScanPara
                         const int f = seli(fi, sv);
                         const float sc = pow2f_sat(seli(dg, sv) * he.ek + he.ev);
                         if (f >= 0) {
-                            float4 *dst = reinterpret_cast<float4 *>(p.S + (bh * p.F + f) * DV + (16 * g) % DV);
+                            float4 *dst = reinterpret_cast<float4 *>(p.S + (bh * p.F + f) * (p.s_ld > 0 ? p.s_ld : DV) +
+                                                                     p.s_off + (16 * g) % DV);
 #pragma unroll
                             for (int j = 0; j < 4; ++j)
                                 dst[j] = make_float4(__uint_as_float(rr[4 * j]) * sc, __uint_as_float(rr[4 * j + 1]) * sc,

@@ -19,7 +19,7 @@ namespace sata {
     cudaError_t tc_run_##a##_##b(const DeviceBasis &basis, int BH, int64_t N, const void *q, const void *k,    \
                                  const void *v, float *out, float *S, float *Z, bool state_in, void *ws,        \
                                  size_t ws_bytes, int *flags, cudaStream_t stream, const HostIO *io,           \
-                                 float *den_out);
+                                 float *den_out, int dvs, int voff);
 SATA_TC_SHAPES(SATA_TC_DECLARE)
 #undef SATA_TC_DECLARE
 #define SATA_TC_BWD_DECLARE(a, b)                                                                               \

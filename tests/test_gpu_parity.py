@@ -356,6 +356,50 @@ def test_state_output_and_continuation(sata, oracle_mod, path):
     assert st.tokens == N and st2.tokens == N
 
 
+@pytest.mark.parametrize("d_K", [64, 128])
+def test_value_halves_state_continuation(sata, oracle_mod, d_K):
+    """d_V = 128 on device buffers runs as two d_V = 64 prefills over the column
+    halves of v, out and S, both producing Z. Two calls carrying the state (the
+    second half must find the incoming Z, not the first half's result): outputs
+    of both calls and the final S and Z against the oracle; the fixed-order mode
+    repeats bit for bit; the host-buffer path (whole rows) agrees."""
+    _set_path(sata, "auto")
+    B, H, N, m, d_V = 1, 2, 260, 110, 128
+    q, k, v = wl.random_inputs(B, H, N, d_K, d_V, seed=5500 + d_K)
+    qc, kc, vc = q.cuda(), k.cuda(), v.cuda()
+    st = sata.State(B, H, d_K, d_V, 4)
+    sata.sata_reset_kernel_stats()
+    y_a = sata.prefill(qc[:, :, : N - m].contiguous(), kc[:, :, : N - m].contiguous(),
+                       vc[:, :, : N - m].contiguous(), P=4, state=st)
+    y_b = sata.prefill(qc[:, :, N - m:].contiguous(), kc[:, :, N - m:].contiguous(),
+                       vc[:, :, N - m:].contiguous(), P=4, state=st)
+    torch.cuda.synchronize()
+    assert sata.sata_sync_status() == 0
+    assert sata.sata_kernel_stats()["tc_scan"][0] == 4   # two calls x two halves
+    y = torch.cat([y_a, y_b], dim=2)
+    ref = oracle_mod.prefill(q, k, v, 4, heads=[(0, 1)])
+    yr, _, S, Z = ref[(0, 1)]
+    err, _, _ = token_rel_err(y[0, 1].cpu().numpy(), yr)
+    assert err <= TOL, f"two calls: {err:.3e}"
+    Sg, Zg = st.S[0, 1].double().cpu().numpy(), st.Z[0, 1].double().cpu().numpy()
+    assert np.abs(Sg - S).max() / np.abs(S).max() <= TOL
+    assert np.abs(Zg - Z).max() / np.abs(Z).max() <= TOL
+    sata.sata_set_option(sata.SATA_OPT_DETERMINISTIC, 1)
+    try:
+        y1 = sata.prefill(qc, kc, vc, P=4)
+        y2 = sata.prefill(qc, kc, vc, P=4)
+    finally:
+        sata.sata_set_option(sata.SATA_OPT_DETERMINISTIC, 0)
+    assert torch.equal(y1, y2)
+    stream = torch.cuda.Stream()
+    yh = torch.empty((B, H, N, d_V), dtype=torch.float32).pin_memory()
+    sata.sata_prefill_host(q.pin_memory(), k.pin_memory(), v.pin_memory(), yh, B, H, N, d_K, d_V, 4, None, stream)
+    stream.synchronize()
+    assert sata.sata_sync_status(stream) == 0
+    assert tensor_rel_err(yh[0, 1].double().numpy(), yr) <= TOL
+    assert tensor_rel_err(y1[0, 1].double().cpu().numpy(), yr) <= TOL
+
+
 @pytest.mark.parametrize("path", list(PATHS))
 def test_deterministic(sata, path):
     """With SATA_OPT_DETERMINISTIC = 1 every path is bitwise reproducible."""
