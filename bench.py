@@ -181,6 +181,7 @@ def flops_per_token(d_K, d_V, P):
 
 # prefill workloads measured beside the headline one (lines under "extra")
 EXTRA_WORKLOADS = ("tiny_d8", "prefill_d16", "prefill_d32", "prefill_d128", "prefill_d64_dv32", "prefill_d16_p6")
+F32_INPUT_WORKLOADS = ("tiny_d8",)   # specified with fp32 q, k, v
 
 
 # ---------------------------------------------------------- distributed ----
@@ -464,15 +465,21 @@ def prefill_roofline(stats, w, steps, peaks, peaks_src, clocks):
 
 def bench_extra(torch, sata, wl, name, args, world, dev, stream, peaks, peaks_src):
     """One more prefill workload, each timed step preceded (outside its events)
-    by a 256 MB write that flushes L2, since some of these inputs fit in L2."""
+    by a 256 MB write that flushes L2, since some of these inputs fit in L2.  The
+    workloads specified with fp32 inputs (tiny_d8) run on them as drawn
+    (sata_prefill_f32); the others take the bf16 inputs."""
     w = wl.WORKLOADS[name]
-    (q, k, v), _ = wl.make_inputs(w)
+    f32_in = name in F32_INPUT_WORKLOADS
+    (q, k, v), _ = wl.make_inputs(w, dtype=torch.float32 if f32_in else torch.bfloat16)
     qd, kd, vd = q.to(dev), k.to(dev), v.to(dev)
     out = torch.empty((w.B, w.H, w.N, w.d_V), dtype=torch.float32, device=dev)
     flush = torch.empty(64 << 20, dtype=torch.float32, device=dev)
 
     def step():
-        sata.sata_prefill_ex(qd, kd, vd, out, w.B, w.H, w.N, w.d_K, w.d_V, w.P, None, None, stream)
+        if f32_in:
+            sata.sata_prefill_f32(qd, kd, vd, out, w.B, w.H, w.N, w.d_K, w.d_V, w.P, None, stream)
+        else:
+            sata.sata_prefill_ex(qd, kd, vd, out, w.B, w.H, w.N, w.d_K, w.d_V, w.P, None, None, stream)
 
     for _ in range(max(3, args.warmup)):
         step()
@@ -492,6 +499,7 @@ def bench_extra(torch, sata, wl, name, args, world, dev, stream, peaks, peaks_sr
     line = {"metric": "SATA prefill tokens/s", "workload": f"{w.name}: B={w.B} H={w.H} N={w.N} d_K={w.d_K} "
             f"d_V={w.d_V} P={w.P} F={w.F}", "value": job_throughput(w.B * w.N, args.steps, world, total),
             "unit": "tokens/s", "steps": args.steps, "ms_per_step": total / args.steps,
+            "inputs": "fp32 q, k, v as drawn" if f32_in else "bf16 q, k, v",
             "dtype": "f16" if roof and roof["kernel"].startswith("tc") else "f32",
             "l2": "L2 flushed (256 MB write) before each timed step", "roofline": roof,
             "gpu_launches": sum(n for n, _ in stats.values()),

@@ -184,6 +184,21 @@ SATA_API int sata_prefill_ex(const void *q, const void *k, const void *v, float 
                     sata_state *st, void *workspace, size_t ws_bytes, void *stream);
 
 /*
+ * As sata_prefill_ex with fp32 q, k, v (same layouts) and a library-owned
+ * workspace: the inputs are used as given, with no rounding to bf16.  Runs on
+ * the CUDA-core prefill (fp32 arithmetic throughout) for every supported shape,
+ * the same chunked form of the recurrence ([CC-TAYLOR] "Feature maps and linear
+ * attention").  For inputs that are specified in fp32 (the tiny d = 8 case);
+ * bf16 inputs should use sata_prefill_ex, whose tensor-core path is much faster.
+ *   q, k, v, out: device pointers, 16-byte aligned, owned by the caller.
+ *   st, stream:   as in sata_prefill_ex.
+ * Errors as sata_prefill_ex.
+ */
+SATA_API int sata_prefill_f32(const float *q, const float *k, const float *v, float *out,
+                    int B, int H, int64_t N, int d_K, int d_V, int P,
+                    sata_state *st, void *stream);
+
+/*
  * As sata_prefill_ex, with q, k, v and out in HOST memory (same layouts and
  * dtypes) and a library-owned workspace.  The same computation as
  * sata_prefill_ex, so the output is the same; the difference is the transfers:

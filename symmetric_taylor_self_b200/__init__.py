@@ -13,5 +13,5 @@ from .binding import (  # noqa: F401
     SATA_ERANGE, SATA_EALIGN, SATA_OPT_PREFILL_PATH, SATA_OPT_WAIT_LIMIT, SATA_OPT_TEST_STALL,
     SATA_OPT_TIME_KERNELS, SATA_OPT_DETERMINISTIC, sata_kernel_stats, sata_reset_kernel_stats, sata_decode_step_static,
     sata_prefill_host, sata_backward_workspace_bytes, sata_prefill_backward, prefill_backward,
-    attention, sata_state_accumulate,
+    attention, sata_state_accumulate, sata_prefill_f32, prefill_f32,
 )

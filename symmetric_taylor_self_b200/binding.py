@@ -37,7 +37,7 @@ EXPORTED = (
     "sata_state_bytes", "sata_state_init", "sata_workspace_bytes", "sata_prefill",
     "sata_prefill_ex", "sata_decode_step", "sata_set_option", "sata_get_option",
     "sata_kernel_stats", "sata_reset_kernel_stats", "sata_decode_step_static", "sata_prefill_host",
-    "sata_backward_workspace_bytes", "sata_prefill_backward", "sata_state_accumulate",
+    "sata_backward_workspace_bytes", "sata_prefill_backward", "sata_state_accumulate", "sata_prefill_f32",
 )
 
 
@@ -98,6 +98,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "sata_reset_kernel_stats": (i32, []),
         "sata_decode_step_static": (i32, [st_p, vp, vp, vp, vp]),
         "sata_prefill_host": (i32, [vp, vp, vp, vp, i32, i32, i64, i32, i32, i32, st_p, vp]),
+        "sata_prefill_f32": (i32, [vp, vp, vp, vp, i32, i32, i64, i32, i32, i32, st_p, vp]),
         "sata_backward_workspace_bytes": (i32, [i32, i32, i64, i32, i32, i32, P_sz]),
         "sata_state_accumulate": (i32, [st_p, vp, vp, i64]),
         "sata_prefill_backward": (i32, [vp, vp, vp, vp, vp, vp, vp, i32, i32, i64, i32, i32, i32,
@@ -232,6 +233,12 @@ def sata_prefill_ex(q, k, v, out, B, H, N, d_K, d_V, P, st=None, workspace=None,
                                   ws_bytes, _stream(stream)), "sata_prefill_ex")
 
 
+def sata_prefill_f32(q, k, v, out, B, H, N, d_K, d_V, P, st=None, stream=None):
+    _check(load().sata_prefill_f32(_ptr(q), _ptr(k), _ptr(v), _ptr(out), B, H, N, d_K, d_V, P,
+                                   None if st is None else ctypes.byref(st), _stream(stream)),
+           "sata_prefill_f32")
+
+
 def sata_prefill_host(q, k, v, out, B, H, N, d_K, d_V, P, st=None, stream=None):
     """q, k, v, out: CPU tensors (pinned for overlap); the library copies them in
     and out segment by segment around the kernels (see include/sata.h)."""
@@ -303,6 +310,20 @@ def prefill(q, k, v, P: int = 4, state: State | None = None, out=None, workspace
     _need(out, torch.float32, (B, H, N, d_V), "out")
     sata_prefill_ex(q, k, v, out, B, H, N, d_K, d_V, P, None if state is None else state.st,
                     workspace, stream)
+    return out
+
+
+def prefill_f32(q, k, v, P: int = 4, state: State | None = None, out=None, stream=None):
+    """As prefill, with fp32 [B, H, N, d] inputs used as given (CUDA-core path)."""
+    B, H, N, d_K = q.shape
+    d_V = v.shape[-1]
+    _need(q, torch.float32, (B, H, N, d_K), "q")
+    _need(k, torch.float32, (B, H, N, d_K), "k")
+    _need(v, torch.float32, (B, H, N, d_V), "v")
+    if out is None:
+        out = torch.empty((B, H, N, d_V), dtype=torch.float32, device=q.device)
+    _need(out, torch.float32, (B, H, N, d_V), "out")
+    sata_prefill_f32(q, k, v, out, B, H, N, d_K, d_V, P, None if state is None else state.st, stream)
     return out
 
 

@@ -18,7 +18,8 @@
 // state carries across segments in global memory.
 //
 // This path is general (any supported d_K, d_V, P) and exact to fp32; the
-// tensor-core path (prefill_tc.cu) is the fast one.
+// tensor-core path (prefill_tc.cu) is the fast one.  The token rows are bf16, or
+// fp32 (sata_prefill_f32: no input rounding at all).
 #include <cuda_bf16.h>
 
 #include "sata_internal.h"
@@ -41,11 +42,10 @@ struct SimtSmem {
 
 // Kernel A: inter-chunk readout partials and state update for one feature tile
 // of one head over the tokens [t0, t0 + T) of a segment (compiled per d_V: the
-// two contractions are register-tiled, simt_tiles.cuh).
-template <int DV>
+// two contractions are register-tiled, simt_tiles.cuh; TI: the rows' type).
+template <int DV, typename TI>
 __global__ void __launch_bounds__(kThreads)
-simt_scan_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k,
-                 const __nv_bfloat16 *__restrict__ v, float *__restrict__ S,
+simt_scan_kernel(const TI *__restrict__ q, const TI *__restrict__ k, const TI *__restrict__ v, float *__restrict__ S,
                  float *__restrict__ Z, const uint32_t *__restrict__ packed,
                  const uint32_t *__restrict__ packed_hi, const float *__restrict__ coef, int d_K,
                  int64_t F, int64_t N,
@@ -133,9 +133,10 @@ simt_scan_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__res
 
 // Kernel B: per chunk, sum the tiles' inter-chunk partials, add the intra-chunk
 // block and divide.
+template <typename TI>
 __global__ void __launch_bounds__(kThreads)
-simt_finish_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k,
-                   const __nv_bfloat16 *__restrict__ v, const float *__restrict__ partials,
+simt_finish_kernel(const TI *__restrict__ q, const TI *__restrict__ k, const TI *__restrict__ v,
+                   const float *__restrict__ partials,
                    int ntiles, int d_K, int d_V, int P, float inv_c, int64_t N, int64_t t0,
                    int T, int Tseg, float *__restrict__ out, float *__restrict__ den_out) {
     extern __shared__ float smem[];
@@ -156,8 +157,8 @@ simt_finish_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
         float a = 0.f, b = 0.f;
         if (t < nt) {
             const int64_t row = (bh * N + t0 + c0 + t) * d_K;
-            a = __bfloat162float(q[row + i]);
-            b = __bfloat162float(k[row + i]);
+            a = simt::in_f(q[row + i]);
+            b = simt::in_f(k[row + i]);
         }
         xq[e] = a;
         xk[e] = b;
@@ -165,7 +166,7 @@ simt_finish_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
     for (int e = tid; e < kL * DV1; e += kThreads) {
         const int t = e / DV1, j = e % DV1;
         float a = 0.f;
-        if (t < nt) a = j < d_V ? __bfloat162float(v[(bh * N + t0 + c0 + t) * d_V + j]) : 1.f;
+        if (t < nt) a = j < d_V ? simt::in_f(v[(bh * N + t0 + c0 + t) * d_V + j]) : 1.f;
         xv[e] = a;
     }
     __syncthreads();
@@ -219,10 +220,11 @@ size_t prefill_simt_workspace_bytes(int BH, int64_t N, int64_t F, int d_V, bool 
     return b;
 }
 
-cudaError_t launch_prefill_simt(const DeviceBasis &basis, int BH, int64_t N, int d_V,
-                                const void *q, const void *k, const void *v, float *out,
-                                float *S, float *Z, bool state_in, void *ws, size_t ws_bytes,
-                                cudaStream_t stream, float *den_out) {
+namespace {
+template <typename TI>
+cudaError_t run_simt(const DeviceBasis &basis, int BH, int64_t N, int d_V, const TI *q, const TI *k, const TI *v,
+                     float *out, float *S, float *Z, bool state_in, void *ws, size_t ws_bytes, cudaStream_t stream,
+                     float *den_out) {
     const int d_K = basis.d_K;
     const int64_t F = basis.F;
     const int ntiles = (int)((F + kTF - 1) / kTF);
@@ -237,17 +239,16 @@ cudaError_t launch_prefill_simt(const DeviceBasis &basis, int BH, int64_t N, int
         Z = S + (size_t)BH * F * d_V;
         state_in = false;
     }
-    using ScanFn = void (*)(const __nv_bfloat16 *, const __nv_bfloat16 *, const __nv_bfloat16 *, float *,
-                            float *, const uint32_t *, const uint32_t *, const float *, int, int64_t,
-                            int64_t, int64_t, int, int, int, float *);
+    using ScanFn = void (*)(const TI *, const TI *, const TI *, float *, float *, const uint32_t *,
+                            const uint32_t *, const float *, int, int64_t, int64_t, int64_t, int, int, int, float *);
     ScanFn scan = nullptr;
     switch (d_V) {
-        case 4: scan = simt_scan_kernel<4>; break;
-        case 8: scan = simt_scan_kernel<8>; break;
-        case 16: scan = simt_scan_kernel<16>; break;
-        case 32: scan = simt_scan_kernel<32>; break;
-        case 64: scan = simt_scan_kernel<64>; break;
-        case 128: scan = simt_scan_kernel<128>; break;
+        case 4: scan = simt_scan_kernel<4, TI>; break;
+        case 8: scan = simt_scan_kernel<8, TI>; break;
+        case 16: scan = simt_scan_kernel<16, TI>; break;
+        case 32: scan = simt_scan_kernel<32, TI>; break;
+        case 64: scan = simt_scan_kernel<64, TI>; break;
+        case 128: scan = simt_scan_kernel<128, TI>; break;
         default: return cudaErrorInvalidValue;
     }
     const size_t smemA = SimtSmem::bytes(d_K, d_V);
@@ -256,30 +257,38 @@ cudaError_t launch_prefill_simt(const DeviceBasis &basis, int BH, int64_t N, int
     cudaError_t e = cudaFuncSetAttribute(scan, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smemA);
     if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(simt_finish_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)smemB);
+    e = cudaFuncSetAttribute(simt_finish_kernel<TI>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smemB);
     if (e != cudaSuccess) return e;
     const float inv_c = 1.0f / sqrtf((float)d_K);
     for (int64_t t0 = 0; t0 < N; t0 += Tseg) {
         const int T = (int)(N - t0 < Tseg ? N - t0 : Tseg);
         const int load = (t0 > 0 || state_in) ? 1 : 0;
         launch_begin(kSimtScan, stream);
-        scan<<<dim3(BH, ntiles), kThreads, smemA, stream>>>(
-            (const __nv_bfloat16 *)q, (const __nv_bfloat16 *)k, (const __nv_bfloat16 *)v, S, Z,
-            basis.packed, basis.packed_hi, basis.coef, d_K, F, N, t0, T, (int)Tseg, load, partials);
+        scan<<<dim3(BH, ntiles), kThreads, smemA, stream>>>(q, k, v, S, Z, basis.packed, basis.packed_hi, basis.coef,
+                                                            d_K, F, N, t0, T, (int)Tseg, load, partials);
         launch_end(kSimtScan, stream);
         e = cudaGetLastError();
         if (e != cudaSuccess) return e;
         const int nchunks = (T + kL - 1) / kL;
         launch_begin(kSimtFinish, stream);
-        simt_finish_kernel<<<dim3(BH, nchunks), kThreads, smemB, stream>>>(
-            (const __nv_bfloat16 *)q, (const __nv_bfloat16 *)k, (const __nv_bfloat16 *)v,
-            partials, ntiles, d_K, d_V, basis.P, inv_c, N, t0, T, (int)Tseg, out, den_out);
+        simt_finish_kernel<TI><<<dim3(BH, nchunks), kThreads, smemB, stream>>>(
+            q, k, v, partials, ntiles, d_K, d_V, basis.P, inv_c, N, t0, T, (int)Tseg, out, den_out);
         launch_end(kSimtFinish, stream);
         e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }
     return cudaSuccess;
+}
+}  // namespace
+
+cudaError_t launch_prefill_simt(const DeviceBasis &basis, int BH, int64_t N, int d_V, const void *q, const void *k,
+                                const void *v, float *out, float *S, float *Z, bool state_in, void *ws,
+                                size_t ws_bytes, cudaStream_t stream, float *den_out, bool f32_in) {
+    if (f32_in)
+        return run_simt(basis, BH, N, d_V, (const float *)q, (const float *)k, (const float *)v, out, S, Z, state_in,
+                        ws, ws_bytes, stream, den_out);
+    return run_simt(basis, BH, N, d_V, (const __nv_bfloat16 *)q, (const __nv_bfloat16 *)k, (const __nv_bfloat16 *)v,
+                    out, S, Z, state_in, ws, ws_bytes, stream, den_out);
 }
 
 }  // namespace sata

@@ -510,6 +510,31 @@ int sata_prefill_ex(const void *q, const void *k, const void *v, float *out, int
     return SATA_OK;
 }
 
+int sata_prefill_f32(const float *q, const float *k, const float *v, float *out, int B, int H, int64_t N, int d_K,
+                     int d_V, int P, sata_state *st, void *stream) {
+    int BH = 0;
+    int rc = check_prefill_args(B, H, N, d_K, d_V, P, st, &BH);
+    if (rc) return rc;
+    if (N == 0 || BH == 0) return SATA_OK;
+    if (!q || !k || !v || !out) return SATA_EINVAL;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return SATA_EALIGN;
+    const int64_t F = num_features(d_K, P);
+    const size_t need = prefill_simt_workspace_bytes(BH, N, F, d_V, st == nullptr);
+    cudaError_t e = cudaSuccess;
+    const DeviceBasis *basis = device_basis(d_K, P, &e);
+    if (!basis) return cuda_fail(e);
+    void *workspace = device_workspace(0, need, &e);
+    if (!workspace) {
+        g_last_cuda = (int)e;
+        return SATA_ENOMEM;
+    }
+    e = launch_prefill_simt(*basis, BH, N, d_V, q, k, v, out, st ? st->S : nullptr, st ? st->Z : nullptr,
+                            st != nullptr, workspace, need, (cudaStream_t)stream, nullptr, true);
+    if (e != cudaSuccess) return cuda_fail(e);
+    if (st) st->tokens += N;
+    return SATA_OK;
+}
+
 int sata_prefill_host(const void *q, const void *k, const void *v, float *out, int B, int H, int64_t N,
                       int d_K, int d_V, int P, sata_state *st, void *stream) {
     int BH = 0;

@@ -93,7 +93,7 @@ size_t prefill_simt_workspace_bytes(int BH, int64_t N, int64_t F, int d_V, bool 
 cudaError_t launch_prefill_simt(const DeviceBasis &basis, int BH, int64_t N, int d_V,
                                 const void *q, const void *k, const void *v, float *out,
                                 float *S, float *Z, bool state_in, void *ws, size_t ws_bytes,
-                                cudaStream_t stream, float *den_out = nullptr);
+                                cudaStream_t stream, float *den_out = nullptr, bool f32_in = false);
 
 // ---- state operations (state_ops.cu) ----
 // S += dS (nS floats), Z += dZ (nZ floats), on `stream`.

@@ -32,14 +32,17 @@ __device__ __forceinline__ float taylor_exp(float x, int n) {
 
 // Loads one chunk of kL token rows starting at row0 into shared memory:
 // x~q, x~k [kL][d_K + 1] (last column 1) and [v | 1] [kL][d_V + 1]; rows past nt
-// are zero.  16-byte loads (8 bf16) when d_K and d_V are multiples of 8, else
-// element loads; either way all of a thread's loads are issued before its
-// stores, so they are in flight together.
-__device__ __forceinline__ void load_qkv_chunk(const __nv_bfloat16 *q, const __nv_bfloat16 *k,
-                                               const __nv_bfloat16 *v, int64_t row0, int nt, int d_K, int d_V,
-                                               float *xq, float *xk, float *xv) {
+// are zero.  16-byte loads (8 bf16) when the rows are bf16 and d_K and d_V are
+// multiples of 8, else element loads; either way all of a thread's loads are
+// issued before its stores, so they are in flight together.
+__device__ __forceinline__ float in_f(__nv_bfloat16 x) { return __bfloat162float(x); }
+__device__ __forceinline__ float in_f(float x) { return x; }
+
+template <typename TI>   // bf16 or fp32 token rows
+__device__ __forceinline__ void load_qkv_chunk(const TI *q, const TI *k, const TI *v, int64_t row0, int nt, int d_K,
+                                               int d_V, float *xq, float *xk, float *xv) {
     const int DK1 = d_K + 1, DV1 = d_V + 1;
-    if ((d_K & 7) == 0 && (d_V & 7) == 0) {
+    if (sizeof(TI) == 2 && (d_K & 7) == 0 && (d_V & 7) == 0) {
         constexpr int U = (kL * (kMaxDK / 8) + kThreads - 1) / kThreads;
         const int nq = kL * (d_K / 8), nv = kL * (d_V / 8);
         uint4 bq[U], bk[U], bv[U];
@@ -94,8 +97,8 @@ __device__ __forceinline__ void load_qkv_chunk(const __nv_bfloat16 *q, const __n
         if (e < kL * DK1) {
             const int t = e / DK1, i = e % DK1;
             if (t < nt) {
-                a[u] = i < d_K ? __bfloat162float(q[(row0 + t) * d_K + i]) : 1.f;
-                b[u] = i < d_K ? __bfloat162float(k[(row0 + t) * d_K + i]) : 1.f;
+                a[u] = i < d_K ? in_f(q[(row0 + t) * d_K + i]) : 1.f;
+                b[u] = i < d_K ? in_f(k[(row0 + t) * d_K + i]) : 1.f;
             }
         }
     }
@@ -113,7 +116,7 @@ __device__ __forceinline__ void load_qkv_chunk(const __nv_bfloat16 *q, const __n
         a[u] = 0.f;
         if (e < kL * DV1) {
             const int t = e / DV1, j = e % DV1;
-            if (t < nt) a[u] = j < d_V ? __bfloat162float(v[(row0 + t) * d_V + j]) : 1.f;
+            if (t < nt) a[u] = j < d_V ? in_f(v[(row0 + t) * d_V + j]) : 1.f;
         }
     }
 #pragma unroll

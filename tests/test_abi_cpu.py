@@ -135,6 +135,16 @@ def test_argument_validation_needs_no_gpu(lib):
     assert lib.sata_prefill_host(fake, fake, fake, fake, 1, 1, 8, 8, 12, 4, None, None) == bd.SATA_EUNSUPPORTED
     assert lib.sata_prefill_host(None, fake, fake, fake, 1, 1, 8, 8, 8, 4, None, None) == bd.SATA_EINVAL
     assert lib.sata_prefill_host(None, None, None, None, 1, 1, 0, 8, 8, 4, None, None) == bd.SATA_OK
+    # fp32-input prefill: the same checks
+    f32 = lib.sata_prefill_f32
+    assert f32(fake, fake, fake, fake, 1, 1, 8, 8, 12, 4, None, None) == bd.SATA_EUNSUPPORTED
+    assert f32(fake, fake, fake, fake, 1, 1, 8, 8, 8, 9, None, None) == bd.SATA_EUNSUPPORTED
+    assert f32(fake, fake, fake, fake, 1, 1, -3, 8, 8, 4, None, None) == bd.SATA_EINVAL
+    assert f32(fake, None, fake, fake, 1, 1, 8, 8, 8, 4, None, None) == bd.SATA_EINVAL
+    assert f32(fake, fake, vp(0x10004), fake, 1, 1, 8, 8, 8, 4, None, None) == bd.SATA_EALIGN
+    assert f32(None, None, None, None, 1, 1, 0, 8, 8, 4, None, None) == bd.SATA_OK
+    st = bd.sata_state(B=1, H=1, d_K=8, d_V=8, P=3, F=120, S=0x10000, Z=0x10000, stream=None, tokens=0)
+    assert f32(fake, fake, fake, fake, 1, 1, 8, 8, 8, 4, ctypes.byref(st), None) == bd.SATA_EINVAL
     # backward
     bw = lambda *a: lib.sata_prefill_backward(*a, None, 0, None)
     assert bw(fake, fake, fake, fake, fake, fake, fake, 1, 1, 8, 8, 12, 4) == bd.SATA_EUNSUPPORTED

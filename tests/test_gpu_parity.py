@@ -116,6 +116,47 @@ def test_prefill_and_decode_other_head_sizes(sata, oracle_mod, d_K, d_V, N, tc):
     _check_heads(yall, _oracle_heads(oracle_mod, q, k, v, 4, [(0, 0)]), what=f"d_K={d_K} d_V={d_V}")
 
 
+def test_prefill_f32_tiny_workload(sata, oracle_mod):
+    """The tiny configuration as specified: fp32 q, k, v ~ N(0, 1), used as drawn
+    (sata_prefill_f32, CUDA-core path), every token against the oracle on the same
+    fp32 values; the bf16 entry point on the rounded draws differs from it by the
+    input rounding alone."""
+    w = wl.WORKLOADS["tiny_d8"]
+    (q, k, v), _ = wl.make_inputs(w, dtype=torch.float32)
+    sata.sata_reset_kernel_stats()
+    y = sata.prefill_f32(q.cuda(), k.cuda(), v.cuda(), P=w.P)
+    torch.cuda.synchronize()
+    assert sata.sata_sync_status() == 0
+    assert "simt_scan" in sata.sata_kernel_stats() and "tc_scan" not in sata.sata_kernel_stats()
+    ref = _oracle_heads(oracle_mod, q, k, v, w.P, [(0, 0)])
+    _check_heads(y, ref, what="tiny_d8, fp32 inputs")
+    # the rounded draws change the result by more than the float32 path's own error
+    yb = sata.prefill(q.to(torch.bfloat16).cuda(), k.to(torch.bfloat16).cuda(), v.to(torch.bfloat16).cuda(), P=w.P)
+    d = (yb - y).abs().max().item() / y.abs().max().item()
+    e = (y[0, 0].double().cpu() - torch.from_numpy(ref[(0, 0)][0])).abs().max().item() / y.abs().max().item()
+    assert d > 10 * e
+
+
+@pytest.mark.parametrize("d_K,d_V,N", [(64, 64, 300), (16, 32, 150), (5, 4, 70)])
+def test_prefill_f32_other_shapes(sata, oracle_mod, d_K, d_V, N):
+    """fp32 inputs on shapes the bf16 entry point serves on tensor cores, and an
+    odd d_K, in two calls through a state: every token of both heads, and the
+    final state, against the oracle."""
+    B, H, m = 1, 2, N // 3
+    q, k, v = wl.random_inputs(B, H, N, d_K, d_V, seed=5600 + d_K + d_V, dtype=torch.float32)
+    qc, kc, vc = q.cuda(), k.cuda(), v.cuda()
+    st = sata.State(B, H, d_K, d_V, 4)
+    ya = sata.prefill_f32(qc[:, :, :m].contiguous(), kc[:, :, :m].contiguous(), vc[:, :, :m].contiguous(), 4, st)
+    yb = sata.prefill_f32(qc[:, :, m:].contiguous(), kc[:, :, m:].contiguous(), vc[:, :, m:].contiguous(), 4, st)
+    torch.cuda.synchronize()
+    assert sata.sata_sync_status() == 0 and st.tokens == N
+    ref = _oracle_heads(oracle_mod, q, k, v, 4, [(0, 0), (0, 1)])
+    _check_heads(torch.cat([ya, yb], dim=2), ref, what=f"fp32 d_K={d_K} d_V={d_V}")
+    for (b, h), (_, _, S, Z) in ref.items():
+        assert np.abs(st.S[b, h].double().cpu().numpy() - S).max() / np.abs(S).max() <= TOL
+        assert np.abs(st.Z[b, h].double().cpu().numpy() - Z).max() / np.abs(Z).max() <= TOL
+
+
 @pytest.mark.parametrize("name", ["tiny_d8", "prefill_d16"])
 def test_prefill_workload_all_heads(sata, oracle_mod, name):
     _set_path(sata, "auto")
