@@ -411,8 +411,11 @@ int sata_workspace_bytes(int B, int H, int64_t N, int d_K, int d_V, int P, size_
     rc = check_shape(d_K, d_V, P);
     if (rc) return rc;
     if (g_opt_prefill_path == 2 && !prefill_tc_supported(d_K, d_V, P)) return SATA_EUNSUPPORTED;
-    // sized for the larger of the fresh-state and carried-state cases
-    *bytes = prefill_ws_bytes(BH, N, d_K, d_V, P, true, nullptr);
+    // sized for the larger of the fresh-state and carried-state cases (a fresh state may be
+    // carried in the workspace; a carried one may need a copy of its Z)
+    const size_t fresh = prefill_ws_bytes(BH, N, d_K, d_V, P, true, nullptr);
+    const size_t carried = prefill_ws_bytes(BH, N, d_K, d_V, P, false, nullptr);
+    *bytes = fresh > carried ? fresh : carried;
     return SATA_OK;
 }
 

@@ -412,8 +412,11 @@ def test_value_halves_state_continuation(sata, oracle_mod, d_K):
     sata.sata_reset_kernel_stats()
     y_a = sata.prefill(qc[:, :, : N - m].contiguous(), kc[:, :, : N - m].contiguous(),
                        vc[:, :, : N - m].contiguous(), P=4, state=st)
+    # the second call in a caller workspace of exactly the queried size (which covers a
+    # carried state's copy of Z)
+    ws = torch.empty(sata.sata_workspace_bytes(B, H, m, d_K, d_V, 4), dtype=torch.uint8, device="cuda")
     y_b = sata.prefill(qc[:, :, N - m:].contiguous(), kc[:, :, N - m:].contiguous(),
-                       vc[:, :, N - m:].contiguous(), P=4, state=st)
+                       vc[:, :, N - m:].contiguous(), P=4, state=st, workspace=ws)
     torch.cuda.synchronize()
     assert sata.sata_sync_status() == 0
     assert sata.sata_kernel_stats()["tc_scan"][0] == 4   # two calls x two halves
