@@ -712,6 +712,29 @@ def test_backward_near_root_denominator(sata, oracle_mod, path, d_K, d_V):
     _set_path(sata, "auto")
 
 
+@pytest.mark.parametrize("path", list(PATHS))
+@pytest.mark.parametrize("d_K,d_V,t0", [(64, 64, 317), (128, 64, 128), (32, 32, 599)])
+def test_backward_cotangent_outlier(sata, oracle_mod, path, d_K, d_V, t0):
+    """One token's dy is 10^4 times the others' (t0 mid-sequence, on a chunk
+    boundary, or last): in the reversed gradient scans the outlier's chunk comes
+    in the middle, at the start or at the end, and the chunks on either side of
+    it must keep their accuracy."""
+    _set_path(sata, path)
+    N, P = 600, 4
+    q, k, v = wl.random_inputs(1, 2, N, d_K, d_V, seed=5700 + d_K + t0)
+    dy = wl.random_cotangent(1, 2, N, d_V, seed=5701)
+    dy[0, 1, t0] *= 1e4
+    dq, dk, dv = sata.prefill_backward(q.cuda(), k.cuda(), v.cuda(), dy.cuda(), P)
+    torch.cuda.synchronize()
+    assert sata.sata_sync_status() == 0
+    ref = oracle_mod.grad_heads(q, k, v, dy, P, heads=[(0, 0), (0, 1)])
+    for (b, h), (rq, rk, rv) in ref.items():
+        for name, g, r in (("dq", dq, rq), ("dk", dk, rk), ("dv", dv, rv)):
+            err = tensor_rel_err(g[b, h].double().cpu().numpy(), r)
+            assert err <= TOL, f"{name} head {(b, h)} d_K={d_K} t0={t0}: {err:.3e}"
+    _set_path(sata, "auto")
+
+
 def test_backward_single_token(sata):
     """N = 1: y_0 = v_0 whatever q and k are, so dv = dy and dq = dk = 0 (up to
     rounding: dw = g.v - g.y cancels)."""
