@@ -311,7 +311,9 @@ cudaError_t run(const DeviceBasis &basis, int BH, int64_t N, const void *q, cons
             launch_end(kTcPrep, stream);
             if (e != cudaSuccess || (e = cudaGetLastError()) != cudaSuccess) return e;
             if (load_state) {
-                tc_state_stats_kernel<<<dim3(BH, 8), 256, 0, stream>>>(S, Z, stats, F, s_ld);
+                int ny = (148 * 8 + BH - 1) / BH;   // about eight blocks per SM over all heads
+                ny = ny < 8 ? 8 : (ny > 1024 ? 1024 : ny);
+                tc_state_stats_kernel<<<dim3(BH, ny), 256, 0, stream>>>(S, Z, stats, F, s_ld);
                 if ((e = cudaGetLastError()) != cudaSuccess) return e;
             }
         }

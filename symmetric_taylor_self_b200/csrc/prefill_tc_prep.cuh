@@ -108,17 +108,24 @@ tc_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restr
 }
 
 // max |S|, |Z| of each head of an incoming state -> stats[bh][3] (S rows of DV values: the
-// whole rows when a call covers a column range of them)
-__global__ void tc_state_stats_kernel(const float *__restrict__ S, const float *__restrict__ Z,
-                                      float *__restrict__ stats, int64_t F, int DV) {
+// whole rows when a call covers a column range of them).  The state is read once per
+// segment before the scan can start, so it is read as 16-byte elements (S is 16-byte
+// aligned, DV a multiple of 4) by a grid that spans the SMs, several loads in flight per
+// thread.
+__global__ void __launch_bounds__(256)
+tc_state_stats_kernel(const float *__restrict__ S, const float *__restrict__ Z, float *__restrict__ stats, int64_t F,
+                      int DV) {
     const int64_t bh = blockIdx.x;
+    const int64_t i0 = blockIdx.y * (int64_t)blockDim.x + threadIdx.x, stride = (int64_t)gridDim.y * blockDim.x;
+    const int64_t n4 = F * DV / 4;
+    const float4 *S4 = reinterpret_cast<const float4 *>(S + bh * F * DV);
     float m = 0.f;
-    const int64_t nS = F * DV;
-    for (int64_t i = blockIdx.y * (int64_t)blockDim.x + threadIdx.x; i < nS + F;
-         i += (int64_t)gridDim.y * blockDim.x) {
-        const float x = i < nS ? S[bh * nS + i] : Z[bh * F + (i - nS)];
-        m = fmaxf(m, fabsf(x));
+#pragma unroll 4
+    for (int64_t i = i0; i < n4; i += stride) {
+        const float4 x = __ldg(S4 + i);
+        m = fmaxf(m, fmaxf(fmaxf(fabsf(x.x), fabsf(x.y)), fmaxf(fabsf(x.z), fabsf(x.w))));
     }
+    for (int64_t i = i0; i < F; i += stride) m = fmaxf(m, fabsf(__ldg(Z + bh * F + i)));
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
     if ((threadIdx.x & 31) == 0) atomicMax(reinterpret_cast<int *>(stats + bh * 4 + 3), __float_as_int(m));

@@ -419,40 +419,54 @@ __global__ void __launch_bounds__(kScanThreads, 1) tc_scan_kernel(const ScanPara
         float cum = 0.f;                // column maxima of the chunks before cl
         bool ok = true;
         if (p.load_state) {   // incoming state -> TMEM (prescaled frame)
-            // a V group is 16 contiguous columns of one feature's S row (four 16-byte loads);
-            // the Z group gathers one Z value per slot
-#pragma unroll 1
-            for (int g = 0; g < NG; ++g) {
-                if (g < ngu) {
-                    uint32_t v16[16];
-                    if (16 * g < nl * DV) {
-                        const int sv = (16 * g) / DV;
-                        const int f = seli(fi, sv);
-                        const float sc = pow2f_sat(-(seli(dg, sv) * he.ek + he.ev));
-                        const float4 *src = reinterpret_cast<const float4 *>(
-                            p.S + (bh * p.F + (f >= 0 ? f : 0)) * (p.s_ld > 0 ? p.s_ld : DV) + p.s_off + (16 * g) % DV);
+            // a V group is 16 contiguous columns of one feature's S row (four 16-byte loads,
+            // scaled by one factor); the Z group gathers one Z value per slot (each scaled
+            // as it lands).  Two groups' loads are in flight before either is stored: each
+            // group is a round trip to HBM, paid once per unit and segment.
+            auto fetch = [&](int g, float4 (&x)[4], float &sc) {
+                if (16 * g < nl * DV) {
+                    const int sv = (16 * g) / DV;
+                    const int f = seli(fi, sv);
+                    sc = pow2f_sat(-(seli(dg, sv) * he.ek + he.ev));
+                    const float4 *src = reinterpret_cast<const float4 *>(
+                        p.S + (bh * p.F + (f >= 0 ? f : 0)) * (p.s_ld > 0 ? p.s_ld : DV) + p.s_off + (16 * g) % DV);
 #pragma unroll
-                        for (int j = 0; j < 4; ++j) {
-                            const float4 x = f >= 0 ? src[j] : make_float4(0.f, 0.f, 0.f, 0.f);
-                            v16[4 * j] = __float_as_uint(x.x * sc);
-                            v16[4 * j + 1] = __float_as_uint(x.y * sc);
-                            v16[4 * j + 2] = __float_as_uint(x.z * sc);
-                            v16[4 * j + 3] = __float_as_uint(x.w * sc);
-                        }
-                    } else {
+                    for (int j = 0; j < 4; ++j) x[j] = f >= 0 ? src[j] : make_float4(0.f, 0.f, 0.f, 0.f);
+                } else {
+                    sc = 1.f;
+                    float z[16];
 #pragma unroll
-                        for (int i = 0; i < 16; ++i) {
-                            const int sz = 16 * g + i - nl * DV;
-                            float x = 0.f;
-                            if (sz < nl) {
-                                const int f = seli(fi, sz);
-                                if (f >= 0) x = p.Z[bh * p.F + f] * pow2f_sat(-(seli(dg, sz) * he.ek));
-                            }
-                            v16[i] = __float_as_uint(x);
+                    for (int i = 0; i < 16; ++i) {
+                        const int sz = 16 * g + i - nl * DV;
+                        z[i] = 0.f;
+                        if (sz < nl) {
+                            const int f = seli(fi, sz);
+                            if (f >= 0) z[i] = p.Z[bh * p.F + f] * pow2f_sat(-(seli(dg, sz) * he.ek));
                         }
                     }
-                    tc_st16(tmem + lane_off + C::COL_S + 16 * g, v16);
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) x[j] = make_float4(z[4 * j], z[4 * j + 1], z[4 * j + 2], z[4 * j + 3]);
                 }
+            };
+            auto put = [&](int g, const float4 (&x)[4], float sc) {
+                uint32_t v16[16];
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    v16[4 * j] = __float_as_uint(x[j].x * sc);
+                    v16[4 * j + 1] = __float_as_uint(x[j].y * sc);
+                    v16[4 * j + 2] = __float_as_uint(x[j].z * sc);
+                    v16[4 * j + 3] = __float_as_uint(x[j].w * sc);
+                }
+                tc_st16(tmem + lane_off + C::COL_S + 16 * g, v16);
+            };
+#pragma unroll 1
+            for (int g = 0; g < ngu; g += 2) {
+                float4 xa[4], xb[4];
+                float sa = 1.f, sb = 1.f;
+                fetch(g, xa, sa);
+                if (g + 1 < ngu) fetch(g + 1, xb, sb);
+                put(g, xa, sa);
+                if (g + 1 < ngu) put(g + 1, xb, sb);
             }
             tc_wait_st();
         }
