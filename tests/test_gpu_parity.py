@@ -444,6 +444,20 @@ def test_value_halves_state_continuation(sata, oracle_mod, d_K):
     assert tensor_rel_err(y1[0, 1].double().cpu().numpy(), yr) <= TOL
 
 
+@pytest.mark.parametrize("d_K,P", [(64, 1), (64, 3), (128, 2), (128, 3)])
+def test_value_halves_lower_P(sata, oracle_mod, d_K, P):
+    """The d_V = 128 halves at P < 4 (other unit plans for the (d_K, 64) instance):
+    every token of both heads against the oracle."""
+    _set_path(sata, "auto")
+    sata.sata_reset_kernel_stats()
+    q, k, v = wl.random_inputs(1, 2, 170, d_K, 128, seed=5800 + d_K + P)
+    y = sata.prefill(q.cuda(), k.cuda(), v.cuda(), P=P)
+    torch.cuda.synchronize()
+    assert sata.sata_sync_status() == 0
+    assert sata.sata_kernel_stats()["tc_scan"][0] == 2
+    _check_heads(y, _oracle_heads(oracle_mod, q, k, v, P, [(0, 0), (0, 1)]), what=f"halves d_K={d_K} P={P}")
+
+
 @pytest.mark.parametrize("path", list(PATHS))
 def test_deterministic(sata, path):
     """With SATA_OPT_DETERMINISTIC = 1 every path is bitwise reproducible."""
