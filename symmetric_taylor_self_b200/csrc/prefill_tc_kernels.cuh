@@ -278,6 +278,12 @@ cudaError_t run(const DeviceBasis &basis, int BH, int64_t N, const void *q, cons
         std::vector<cudaEvent_t> &ev;
         ~Release() { for (cudaEvent_t x : ev) cudaEventDestroy(x); }
     } release{events};
+    if (io) {   // the copies follow the work already on `stream` (an earlier call may still read these buffers)
+        cudaEvent_t ev;
+        if ((e = new_event(&ev)) || (e = cudaEventRecord(ev, stream)) || (e = cudaStreamWaitEvent(io->h2d, ev, 0)) ||
+            (e = cudaStreamWaitEvent(io->d2h, ev, 0)))
+            return e;
+    }
     for (int s = 0; s < nseg; ++s) {
         const int c0s = pl.profiled ? pl.seg_c0[s] : s * pl.nc_seg;
         const int ncs = pl.profiled ? pl.seg_c0[s + 1] - c0s

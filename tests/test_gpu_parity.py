@@ -317,6 +317,27 @@ def test_prefill_host_other_shapes(sata, oracle_mod, d_K, d_V, N):
     _check_heads(yh, ref, what=f"host d_K={d_K} d_V={d_V} N={N}")
 
 
+def test_prefill_host_back_to_back_calls(sata):
+    """Two host-buffer calls on one stream with different inputs and no sync
+    between them (four segments each): each output equals the device-buffer
+    prefill of its own inputs. The second call's input copies may not start
+    before the first call's kernels have read the shared device copies."""
+    _set_path(sata, "auto")
+    B, H, N, d = 1, 8, 16384, 64
+    x1 = wl.random_inputs(B, H, N, d, d, seed=5900)
+    x2 = wl.random_inputs(B, H, N, d, d, seed=5901)
+    stream = torch.cuda.Stream()
+    ys = [torch.empty((B, H, N, d), dtype=torch.float32).pin_memory() for _ in range(2)]
+    pinned = [[t.pin_memory() for t in x] for x in (x1, x2)]
+    for (q, k, v), y in zip(pinned, ys):
+        sata.sata_prefill_host(q, k, v, y, B, H, N, d, d, 4, None, stream)
+    stream.synchronize()
+    assert sata.sata_sync_status(stream) == 0
+    for (q, k, v), y in zip((x1, x2), ys):
+        ref = sata.prefill(q.cuda(), k.cuda(), v.cuda(), P=4).cpu()
+        assert ((y - ref).abs().max() / ref.abs().max()).item() <= 1e-5
+
+
 def test_prefill_d64_long_head(sata, oracle_mod):
     """One d = 64 head over 8192 tokens against the oracle's recurrence: every
     token and the final state."""
