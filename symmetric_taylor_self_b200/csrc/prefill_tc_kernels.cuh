@@ -148,6 +148,10 @@ struct Plan {
     // host-buffer path: segment starts (chunks) of a non-uniform split, seg_c0[nseg] = nchunks
     bool profiled = false;
     int seg_c0[kHostSegments + 1] = {};
+    // host-buffer path: each segment's prep runs on a side stream ahead of the scans, so
+    // the per-head maxima have one buffer per segment
+    int nstats = 1;
+    size_t stats_bytes = 0;
     size_t off_stats = 0, off_q16 = 0, off_k16 = 0, off_v16 = 0, off_red = 0, off_part = 0, off_state = 0,
            total = 0;
 };
@@ -190,8 +194,11 @@ bool make_plan(int BH, int64_t N, int64_t F, int P, bool need_state, int min_seg
         for (int i = 0; i < kHostSegments; ++i)
             if (pl.seg_c0[i + 1] - pl.seg_c0[i] > pl.nc_seg) pl.nc_seg = pl.seg_c0[i + 1] - pl.seg_c0[i];
     }
+    const bool piped = !deterministic && min_segments == kHostSegments;
+    pl.nstats = piped ? pl.nseg : 1;
+    pl.stats_bytes = align256((size_t)BH * 4 * sizeof(float));
     pl.off_stats = 0;
-    pl.off_q16 = align256((size_t)BH * 4 * sizeof(float));
+    pl.off_q16 = pl.nstats * pl.stats_bytes;
     const size_t rows = (size_t)BH * pl.nchunks * kL;   // whole chunks, chunk-interleaved
     pl.off_k16 = pl.off_q16 + align256(rows * DK * 2);
     pl.off_v16 = pl.off_k16 + align256(rows * DK * 2);
@@ -244,9 +251,7 @@ cudaError_t run(const DeviceBasis &basis, int BH, int64_t N, const void *q, cons
         &e);
     if (!tab) return e != cudaSuccess ? e : cudaErrorMemoryAllocation;
     uint8_t *w = (uint8_t *)ws;
-    float *stats = (float *)(w + pl.off_stats);
     __half *q16 = (__half *)(w + pl.off_q16), *k16 = (__half *)(w + pl.off_k16), *v16 = (__half *)(w + pl.off_v16);
-    float *red = (float *)(w + pl.off_red);
     float *part = (float *)(w + pl.off_part);
     const int nseg = pl.nseg;
     if (own_state && nseg > 1) {
@@ -278,44 +283,59 @@ cudaError_t run(const DeviceBasis &basis, int BH, int64_t N, const void *q, cons
         std::vector<cudaEvent_t> &ev;
         ~Release() { for (cudaEvent_t x : ev) cudaEventDestroy(x); }
     } release{events};
+    // Host buffers (not in the fixed-order mode): each segment's maxima and prescaled rows are
+    // built on the side stream `ps` as soon as its rows have landed, so they run beside the
+    // previous segment's scan (in its last wave, where SMs fall idle) instead of between
+    // the scans; a segment's maxima have their own buffer.  The incoming-state bound, the
+    // scans and the finishes stay on `stream`, in order.  (A finish on the side stream
+    // competed with the next scan's first wave for SMs and gained little.)
+    const bool piped = io && !det;
+    cudaStream_t ps = piped ? io->aux : stream;
     if (io) {   // the copies follow the work already on `stream` (an earlier call may still read these buffers)
         cudaEvent_t ev;
         if ((e = new_event(&ev)) || (e = cudaEventRecord(ev, stream)) || (e = cudaStreamWaitEvent(io->h2d, ev, 0)) ||
-            (e = cudaStreamWaitEvent(io->d2h, ev, 0)))
+            (e = cudaStreamWaitEvent(io->d2h, ev, 0)) || (piped && (e = cudaStreamWaitEvent(ps, ev, 0))))
             return e;
     }
+    float *red = (float *)(w + pl.off_red);
     for (int s = 0; s < nseg; ++s) {
         const int c0s = pl.profiled ? pl.seg_c0[s] : s * pl.nc_seg;
         const int ncs = pl.profiled ? pl.seg_c0[s + 1] - c0s
                                     : ((pl.nchunks - c0s < pl.nc_seg) ? pl.nchunks - c0s : pl.nc_seg);
         const int64_t tok0 = (int64_t)c0s * kL, tok1 = (int64_t)(c0s + ncs) * kL < N ? (int64_t)(c0s + ncs) * kL : N;
-        if (io) {   // this segment's inputs: host -> device on the copy stream, compute waits for them
+        float *stats = (float *)(w + pl.off_stats + (size_t)(piped ? s : 0) * pl.stats_bytes);
+        if (io) {   // this segment's inputs: host -> device on the copy stream; its prep waits for them
             cudaEvent_t ev;
             if ((e = copy_rows((void *)q, io->q, BH, N, tok0, tok1, DK, 2, cudaMemcpyHostToDevice, io->h2d)) ||
                 (e = copy_rows((void *)k, io->k, BH, N, tok0, tok1, DK, 2, cudaMemcpyHostToDevice, io->h2d)) ||
                 (e = copy_rows((void *)v, io->v, BH, N, tok0, tok1, DV, 2, cudaMemcpyHostToDevice, io->h2d)) ||
-                (e = new_event(&ev)) || (e = cudaEventRecord(ev, io->h2d)) || (e = cudaStreamWaitEvent(stream, ev, 0)))
+                (e = new_event(&ev)) || (e = cudaEventRecord(ev, io->h2d)) || (e = cudaStreamWaitEvent(ps, ev, 0)))
                 return e;
         }
         const bool load_state = (s > 0 || state_in);
-        {   // this segment's maxima, prescaled rows and incoming-state bound
-            if ((e = cudaMemsetAsync(stats, 0, (size_t)BH * 4 * sizeof(float), stream)) != cudaSuccess) return e;
+        {   // this segment's maxima and prescaled rows (on ps), then the incoming-state bound
+            if ((e = cudaMemsetAsync(stats, 0, (size_t)BH * 4 * sizeof(float), ps)) != cudaSuccess) return e;
             const int64_t ntok = tok1 - tok0;
             int bx = (int)((ntok * (DK / 8) + 255) / 256);
             const int bmax = (148 * 8 + BH - 1) / BH;
             if (bx > bmax) bx = bmax;
             if (bx < 1) bx = 1;
-            launch_begin(kTcPrep, stream);
-            tc_stats_kernel<DK, DV><<<(unsigned)((int64_t)bx * BH), 256, 0, stream>>>(qb, kb, vb, stats, N, tok0,
-                                                                                    tok1, bx, dvs);
+            launch_begin(kTcPrep, ps);
+            tc_stats_kernel<DK, DV><<<(unsigned)((int64_t)bx * BH), 256, 0, ps>>>(qb, kb, vb, stats, N, tok0, tok1, bx,
+                                                                                dvs);
             if ((e = cudaGetLastError()) == cudaSuccess) {
                 const int64_t nwork = (int64_t)BH * ntok;   // one thread per token row
                 const int pgrid = (int)((nwork + 255) / 256 < 148 * 16 ? (nwork + 255) / 256 : 148 * 16);
-                tc_prep_kernel<DK, DV><<<pgrid, 256, 0, stream>>>(qb, kb, vb, stats, q16, k16, v16, BH, N, tok0, tok1,
-                                                                   pl.nchunks, flags, dvs, voff);
+                tc_prep_kernel<DK, DV><<<pgrid, 256, 0, ps>>>(qb, kb, vb, stats, q16, k16, v16, BH, N, tok0, tok1,
+                                                               pl.nchunks, flags, dvs, voff);
             }
-            launch_end(kTcPrep, stream);
+            launch_end(kTcPrep, ps);
             if (e != cudaSuccess || (e = cudaGetLastError()) != cudaSuccess) return e;
+            if (piped) {
+                cudaEvent_t ev;
+                if ((e = new_event(&ev)) || (e = cudaEventRecord(ev, ps)) || (e = cudaStreamWaitEvent(stream, ev, 0)))
+                    return e;
+            }
             if (load_state) {
                 int ny = (148 * 8 + BH - 1) / BH;   // about eight blocks per SM over all heads
                 ny = ny < 8 ? 8 : (ny > 1024 ? 1024 : ny);

@@ -32,7 +32,7 @@ struct DeviceRes {
     void *ws[4] = {nullptr, nullptr, nullptr, nullptr};
     size_t ws_bytes[4] = {0, 0, 0, 0};
     std::map<uint64_t, void *> tables;
-    cudaStream_t h2d = nullptr, d2h = nullptr;
+    cudaStream_t h2d = nullptr, d2h = nullptr, aux = nullptr;
 };
 std::map<int, DeviceRes> g_dev;
 std::map<std::pair<int, int>, HostBasis> g_host_bases;
@@ -183,7 +183,7 @@ void *device_workspace(int slot, size_t bytes, cudaError_t *err) {
     return r.ws[slot];
 }
 
-cudaError_t device_copy_streams(cudaStream_t *h2d, cudaStream_t *d2h) {
+cudaError_t device_copy_streams(cudaStream_t *h2d, cudaStream_t *d2h, cudaStream_t *aux) {
     std::lock_guard<std::mutex> lk(g_mu);
     cudaError_t err = cudaSuccess;
     const int dev = current_device(&err);
@@ -191,8 +191,10 @@ cudaError_t device_copy_streams(cudaStream_t *h2d, cudaStream_t *d2h) {
     DeviceRes &r = g_dev[dev];
     if (!r.h2d && (err = cudaStreamCreateWithFlags(&r.h2d, cudaStreamNonBlocking)) != cudaSuccess) return err;
     if (!r.d2h && (err = cudaStreamCreateWithFlags(&r.d2h, cudaStreamNonBlocking)) != cudaSuccess) return err;
+    if (!r.aux && (err = cudaStreamCreateWithFlags(&r.aux, cudaStreamNonBlocking)) != cudaSuccess) return err;
     *h2d = r.h2d;
     *d2h = r.d2h;
+    *aux = r.aux;
     return cudaSuccess;
 }
 
@@ -343,6 +345,7 @@ void sata_shutdown(void) {
         for (auto &t : kv.second.tables) cudaFree(t.second);
         if (kv.second.h2d) cudaStreamDestroy(kv.second.h2d);
         if (kv.second.d2h) cudaStreamDestroy(kv.second.d2h);
+        if (kv.second.aux) cudaStreamDestroy(kv.second.aux);
     }
     g_dev.clear();
     cudaSetDevice(cur);
@@ -574,8 +577,8 @@ int sata_prefill_host(const void *q, const void *k, const void *v, float *out, i
     void *dq = io_buf + oq, *dk = io_buf + ok_, *dv = io_buf + ov;
     float *dout = (float *)(io_buf + oo);
     if (use_tc) {
-        HostIO io{q, k, v, out, nullptr, nullptr};
-        if ((e = device_copy_streams(&io.h2d, &io.d2h)) != cudaSuccess) return cuda_fail(e);
+        HostIO io{q, k, v, out, nullptr, nullptr, nullptr};
+        if ((e = device_copy_streams(&io.h2d, &io.d2h, &io.aux)) != cudaSuccess) return cuda_fail(e);
         e = launch_prefill_tc(*basis, BH, N, d_V, dq, dk, dv, dout, S, Z, state_in, workspace, need, flags, s, &io);
     } else {   // CUDA-core path: whole copies around the call
         if ((e = cudaMemcpyAsync(dq, q, nq, cudaMemcpyHostToDevice, s)) == cudaSuccess &&

@@ -123,7 +123,8 @@ cudaError_t launch_prefill_backward(const DeviceBasis &basis, int BH, int64_t N,
 struct HostIO {
     const void *q, *k, *v;   // host [BH][N][d] bf16
     float *out;              // host [BH][N][d_V] fp32
-    cudaStream_t h2d, d2h;
+    cudaStream_t h2d, d2h;   // copy streams
+    cudaStream_t aux;        // a segment's prep and finish, beside the scans
 };
 constexpr int kHostSegments = 4;   // at least this many segments when copies are pipelined
 bool prefill_tc_supported(int d_K, int d_V, int P);
@@ -134,6 +135,6 @@ cudaError_t launch_prefill_tc(const DeviceBasis &basis, int BH, int64_t N, int d
                               float *S, float *Z, bool state_in, void *ws, size_t ws_bytes,
                               int *flags, cudaStream_t stream, const HostIO *io, float *den_out = nullptr);
 // Library-owned copy streams of the current device (non-blocking), created once.
-cudaError_t device_copy_streams(cudaStream_t *h2d, cudaStream_t *d2h);
+cudaError_t device_copy_streams(cudaStream_t *h2d, cudaStream_t *d2h, cudaStream_t *aux);
 
 }  // namespace sata
