@@ -46,7 +46,8 @@ tc_reduce_kernel(const float4 *__restrict__ part, float4 *__restrict__ red, int 
 //   O = W_hi [V'|1] + W_lo [V'|1]   TMEM,  V' = v 2^-e_v
 //   out[t] = (2^(e_t+e_v) O_num + num_t) / (2^e_t O_den + den_t), num/den the summed inter-chunk
 //            readouts (true frame)
-// One CTA (4 warps, thread = token row) per (head, chunk).
+// One CTA per (head, chunk): 8 warps, two per TMEM lane quarter (thread = token row), the
+// two halves of a row's weight columns and output columns split between them.
 template <int DK, int DV>
 struct FinCfg {
     static constexpr int KB = (DK + 63) / 64;          // 64-wide K atoms of Q and K
@@ -60,16 +61,17 @@ struct FinCfg {
     static constexpr int OFF_V = (V0 + 1023) / 1024 * 1024;   // [128 s][NV n] MN-major, no swizzle
     static constexpr int LBO_V = (NV / 8) * 128;
     static constexpr int OFF_BAR = OFF_V + 128 * NV * 2;
+    static constexpr int OFF_WM = OFF_BAR + 64;        // [2][128] row maxima of the two column halves
     static constexpr int TCOLS = 128 + NV <= 256 ? 256 : 512;
     // with all 512 TMEM columns, one CTA per SM (a shared-memory request above half the SM)
-    static constexpr int SMEM0 = OFF_BAR + 64 + 1024;
+    static constexpr int SMEM0 = OFF_WM + 1024 + 1024;
     static constexpr int SMEM = TCOLS == 512 && SMEM0 < 120 * 1024 ? 120 * 1024 : SMEM0;
     static_assert(2 * KB * 16384 >= 32768, "W_lo");
     static_assert(SMEM <= 232448, "shared memory");
 };
 
 template <int DK, int DV>
-__global__ void __launch_bounds__(128)
+__global__ void __launch_bounds__(256)
 tc_finish_kernel(const __half *__restrict__ q16, const __half *__restrict__ k16, const __half *__restrict__ v16,
                  const float *__restrict__ stats, const float *__restrict__ red, float *__restrict__ out,
                  float *__restrict__ den_out, int c0, int nc, int nch, int64_t N, int P, float inv_c, int *flags,
@@ -83,6 +85,7 @@ tc_finish_kernel(const __half *__restrict__ q16, const __half *__restrict__ k16,
     volatile uint32_t *tmem_slot = reinterpret_cast<volatile uint32_t *>(sm + F::OFF_BAR + 16);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + F::OFF_BAR + 20);
     const int tid = threadIdx.x, warp = tid / 32;
+    const int quarter = warp & 3, half = warp >> 2;   // TMEM lane quarter, column half
     const int64_t bh = blockIdx.x / nc;
     const int cl = blockIdx.x % nc;
     const int64_t t0 = (int64_t)(c0 + cl) * kL;
@@ -103,7 +106,7 @@ tc_finish_kernel(const __half *__restrict__ q16, const __half *__restrict__ k16,
     // ---- operands: prescaled fp16 rows (chunk-interleaved, token fastest), swizzled
     const uint4 *qcr = chunk_rows<DK>(q16, bh, nch, c0 + cl), *kcr = chunk_rows<DK>(k16, bh, nch, c0 + cl);
     const uint4 *vcr = chunk_rows<DV>(v16, bh, nch, c0 + cl);
-    for (int e = tid; e < kL * (DK / 8); e += 128) {   // Q and K: DK/8 pieces of 8 d per row
+    for (int e = tid; e < kL * (DK / 8); e += 256) {   // Q and K: DK/8 pieces of 8 d per row
         const int r = e % kL, c = e / kL;
         uint4 hq = make_uint4(0, 0, 0, 0), hk = make_uint4(0, 0, 0, 0);
         if (r < nt) {
@@ -114,7 +117,7 @@ tc_finish_kernel(const __half *__restrict__ q16, const __half *__restrict__ k16,
         *reinterpret_cast<uint4 *>(sm + F::OFF_Q + off) = hq;
         *reinterpret_cast<uint4 *>(sm + F::OFF_K + off) = hk;
     }
-    for (int e = tid; e < kL * (NV / 8); e += 128) {   // [V'|1]: row s, 8 n per 16-byte core row
+    for (int e = tid; e < kL * (NV / 8); e += 256) {   // [V'|1]: row s, 8 n per 16-byte core row
         const int r = e % kL, c = e / kL;
         uint4 hv = make_uint4(0, 0, 0, 0);
         if (r < nt) {
@@ -141,8 +144,8 @@ tc_finish_kernel(const __half *__restrict__ q16, const __half *__restrict__ k16,
     __syncwarp();
     bool ok = W.wait(bar, 0);
     tc_after();
-    const int t = tid;                               // token row = TMEM lane
-    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+    const int t = quarter * 32 + (tid & 31);         // token row = TMEM lane
+    const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
     // ---- W row t: polynomial, causal mask, power-of-two scale into the fp16 range
     // Horner form of sum_{p<P} x^p / p!, x = S' 2^E / c: h <- 1 + h * S' * (2^E / (c p)), P <= 4
     const float xs = pow2f_sat(he.eq + he.ek) * inv_c;
@@ -157,7 +160,7 @@ tc_finish_kernel(const __half *__restrict__ q16, const __half *__restrict__ k16,
     float wmax = 0.f;
     if (ok) {
 #pragma unroll 1
-        for (int c16 = 0; c16 < 8; ++c16) {
+        for (int c16 = 4 * half; c16 < 4 * half + 4; ++c16) {
             uint32_t rr[16];
             tc_ld16(tmem + lane_off + c16 * 16, rr);
             tc_wait_ld();
@@ -165,13 +168,19 @@ tc_finish_kernel(const __half *__restrict__ q16, const __half *__restrict__ k16,
             for (int i = 0; i < 16; ++i) wmax = fmaxf(wmax, fabsf(wval(__uint_as_float(rr[i]), c16 * 16 + i)));
         }
     }
+    {   // the row's maximum over both column halves
+        float *wm = reinterpret_cast<float *>(sm + F::OFF_WM);
+        wm[half * 128 + t] = wmax;
+        __syncthreads();
+        wmax = fmaxf(wm[t], wm[128 + t]);
+    }
     // e_t: 2^-e_t wmax < 2^15
     const int ebits = (int)((__float_as_uint(wmax) >> 23) & 255) - 127;
     const int e_t = ebits > 14 ? ebits - 14 : 0;
     const float down = pow2f_sat(-e_t);
     if (ok) {
 #pragma unroll 1
-        for (int c16 = 0; c16 < 8; ++c16) {
+        for (int c16 = 4 * half; c16 < 4 * half + 4; ++c16) {
             uint32_t rr[16];
             tc_ld16(tmem + lane_off + c16 * 16, rr);
             tc_wait_ld();
@@ -226,10 +235,11 @@ tc_finish_kernel(const __half *__restrict__ q16, const __half *__restrict__ k16,
             const float den = fmaf(__uint_as_float(rr[0]), upz, rp[(DV / 4) * kL].x);
             inv = 1.f / den;
             finite = fabsf(inv) <= FLT_MAX;
-            if (den_out && t < nt) den_out[bh * N + t0 + t] = den;   // kept for the backward pass
+            if (den_out && half == 0 && t < nt) den_out[bh * N + t0 + t] = den;   // kept for the backward pass
         }
+        constexpr int NG = DV / 16, NG0 = (NG + 1) / 2;   // output column groups: [0, NG0) and [NG0, NG)
 #pragma unroll
-        for (int c16 = 0; c16 < DV / 16; ++c16) {
+        for (int c16 = half ? NG0 : 0; c16 < (half ? NG : NG0); ++c16) {
             uint32_t rr[16];
             tc_ld16(tmem + 128 + lane_off + c16 * 16, rr);
             tc_wait_ld();
@@ -252,7 +262,7 @@ tc_finish_kernel(const __half *__restrict__ q16, const __half *__restrict__ k16,
     tc_before();
     __syncthreads();
     if (ok) {
-        for (int e = tid; e < nt * (DV / 4); e += 128) {
+        for (int e = tid; e < nt * (DV / 4); e += 256) {
             const int r = e / (DV / 4), c4 = e % (DV / 4);
             reinterpret_cast<float4 *>(out + (bh * N + t0 + r) * dvs + voff)[c4] =
                 *reinterpret_cast<const float4 *>(stg + r * F::STG + 4 * c4);

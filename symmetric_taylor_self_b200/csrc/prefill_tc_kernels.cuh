@@ -391,7 +391,7 @@ cudaError_t run(const DeviceBasis &basis, int BH, int64_t N, const void *q, cons
             if ((e = cudaGetLastError()) != cudaSuccess) return e;
         }
         launch_begin(kTcFinish, stream);
-        tc_finish_kernel<DK, DV><<<(int)((int64_t)BH * ncs), 128, FinCfg<DK, DV>::SMEM, stream>>>(
+        tc_finish_kernel<DK, DV><<<(int)((int64_t)BH * ncs), 256, FinCfg<DK, DV>::SMEM, stream>>>(
             q16, k16, v16, stats, red, out, den_out, c0s, ncs, pl.nchunks, N, basis.P, inv_c, flags, wait_ns, dvs,
             voff);
         launch_end(kTcFinish, stream);
