@@ -156,7 +156,9 @@ SATA_API int sata_state_init(sata_state *st, int B, int H, int d_K, int d_V, int
  */
 SATA_API int sata_state_accumulate(sata_state *st, const float *S, const float *Z, int64_t tokens);
 
-/* Workspace bytes sata_prefill_ex needs for this shape. */
+/* Workspace bytes sata_prefill_ex needs for this shape: the larger of the
+ * fresh-state and carried-state needs, so one size serves calls with or
+ * without a sata_state (under the options in force at the query). */
 SATA_API int sata_workspace_bytes(int B, int H, int64_t N, int d_K, int d_V, int P, size_t *bytes);
 
 /*
