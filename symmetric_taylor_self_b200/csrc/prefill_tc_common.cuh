@@ -326,6 +326,18 @@ __device__ __forceinline__ float col_max(const ScanParams &p, int64_t bh, int cl
     return fmaxf(p.colmax[bh * p.nch + p.c0 + cl], p.colmax_floor);
 }
 
+// Non-blocking test of an mbarrier phase (the issuer polls two chains).
+__device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tmbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}\n"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
 struct Waiter {
     volatile int *abort_flag;
     int *gflag;

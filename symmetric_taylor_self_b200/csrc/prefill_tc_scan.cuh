@@ -233,8 +233,17 @@ __global__ void __launch_bounds__(kScanThreads, 1) tc_scan_kernel(const ScanPara
     const Waiter W{abort_flag, p.flags + kFlagTimeout, p.wait_ns};
 
     if (warp == kWarpI) {
-        // ------------------------------------------------ MMA issue (one thread, both streams in chunk order)
-        if (lane == 0) {
+        // ------------------------------------------------ MMA issue (one thread, two chains)
+        // The update of chunk cu and the readout of chunk cr (cr < cu: a readout follows its
+        // chunk's update) are issued as soon as their operands are ready, whichever is ready
+        // first, so the update of chunk c + 1 need not wait behind the readout of chunk c (the
+        // drain of chunk c - 1 gates that readout).  No tested barrier can be a phase ahead of
+        // its test: each one's next phase needs an MMA this thread has not issued yet.  With
+        // nothing ready the thread sleeps briefly; no progress for the wait limit aborts as a
+        // blocking wait would.  (1.7 % faster than issuing both chains in chunk order for the
+        // prefill; the gradient scans, whose drain contracts every slot separately, ran 2.5 %
+        // slower with it and issue in chunk order.)
+        if (lane == 0 && JAC) {
             const uint32_t id_u = idesc_f16(128, NU, 1, 1);   // A, B MN-major in shared memory
             const uint32_t id_r = idesc_f16(128, NU, 0, 1);   // A in TMEM, B MN-major
             const uint32_t wb = sb + C::OFF_W;
@@ -244,7 +253,6 @@ __global__ void __launch_bounds__(kScanThreads, 1) tc_scan_kernel(const ScanPara
                 ok = W.wait(BAR(C::B_AKF), cl & 1) && W.wait(BAR(C::B_SR), cl & 1);
                 if (!ok) break;
                 tc_after();
-                // update: [S|Z] (+)= P2(K)^T [128 pairs x 128 t] . W [128 t x NU]
                 const uint32_t ak = sb + C::OFF_AK + b * C::AK_BYTES;
 #pragma unroll
                 for (int ks = 0; ks < 8; ++ks)
@@ -257,14 +265,64 @@ __global__ void __launch_bounds__(kScanThreads, 1) tc_scan_kernel(const ScanPara
                      (cl == 0 || W.wait(BAR(C::B_RF), (cl - 1) & 1));
                 if (!ok) break;
                 tc_after();
-                // readout: R = P2(Q) [128 t x 128 pairs] . B [128 pairs x NU]
                 const uint32_t bs = sb + C::OFF_BS + b * C::W_BYTES;
 #pragma unroll
                 for (int ks = 0; ks < 8; ++ks)
-                    tc_mma_ta(tmem + C::COL_R, tmem + C::COL_AQ + ks * 8, sdesc(bs + ks * 2 * C::LBO, C::LBO, 128, 0),
-                              id_r, ks > 0 ? 1u : 0u);
+                    tc_mma_ta(tmem + C::COL_R, tmem + C::COL_AQ + ks * 8,
+                              sdesc(bs + ks * 2 * C::LBO, C::LBO, 128, 0), id_r, ks > 0 ? 1u : 0u);
                 tc_commit(BAR(C::B_BSE + b));
                 tc_commit(BAR(C::B_RD));
+            }
+            // every issued MMA completes before TMEM is released
+            tc_commit(BAR(C::B_FIN));
+            W.drain(BAR(C::B_FIN), 0);
+        } else if (lane == 0) {
+            const uint32_t id_u = idesc_f16(128, NU, 1, 1);   // A, B MN-major in shared memory
+            const uint32_t id_r = idesc_f16(128, NU, 0, 1);   // A in TMEM, B MN-major
+            const uint32_t wb = sb + C::OFF_W;
+            int cu = 0, cr = 0;
+            int64_t t_last = gtimer();
+            while (cr < p.nc) {
+                bool prog = false;
+                if (cu < p.nc && mbar_test(BAR(C::B_AKF), cu & 1) && mbar_test(BAR(C::B_SR), cu & 1)) {
+                    const int cl = cu++, b = cl & 1;
+                    tc_after();
+                    // update: [S|Z] (+)= P2(K)^T [128 pairs x 128 t] . W [128 t x NU]
+                    const uint32_t ak = sb + C::OFF_AK + b * C::AK_BYTES;
+#pragma unroll
+                    for (int ks = 0; ks < 8; ++ks)
+                        tc_mma(tmem + C::COL_S, sdesc(ak + ks * 2048, 16384, 1024, 2),
+                               sdesc(wb + ks * 2 * C::LBO, C::LBO, 128, 0), id_u,
+                               (p.load_state || cl > 0 || ks > 0) ? 1u : 0u);
+                    tc_commit(BAR(C::B_AKE + b));
+                    tc_commit(BAR(C::B_UD));
+                    prog = true;
+                }
+                if (cr < cu && mbar_test(BAR(C::B_AQF), cr & 1) && mbar_test(BAR(C::B_BSF + (cr & 1)), (cr >> 1) & 1) &&
+                    (cr == 0 || mbar_test(BAR(C::B_RF), (cr - 1) & 1))) {
+                    const int cl = cr++, b = cl & 1;
+                    tc_after();
+                    // readout: R = P2(Q) [128 t x 128 pairs] . B [128 pairs x NU]
+                    const uint32_t bs = sb + C::OFF_BS + b * C::W_BYTES;
+#pragma unroll
+                    for (int ks = 0; ks < 8; ++ks)
+                        tc_mma_ta(tmem + C::COL_R, tmem + C::COL_AQ + ks * 8,
+                                  sdesc(bs + ks * 2 * C::LBO, C::LBO, 128, 0), id_r, ks > 0 ? 1u : 0u);
+                    tc_commit(BAR(C::B_BSE + b));
+                    tc_commit(BAR(C::B_RD));
+                    prog = true;
+                }
+                if (prog) {
+                    t_last = gtimer();
+                } else {
+                    if (*abort_flag) break;
+                    if (gtimer() - t_last > W.limit) {
+                        *abort_flag = 1;
+                        atomicExch(W.gflag, 1);
+                        break;
+                    }
+                    __nanosleep(40);
+                }
             }
             // every issued MMA completes before TMEM is released
             tc_commit(BAR(C::B_FIN));
