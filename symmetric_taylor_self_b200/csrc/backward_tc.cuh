@@ -587,18 +587,20 @@ cudaError_t bwd_tc_run(const DeviceBasis &basis, int BH, int64_t N, const void *
     float *sq = (float *)(w + L.off_sq), *sk = (float *)(w + L.off_sk), *sv = (float *)(w + L.off_sv);
 
     const dim3 rgrid((unsigned)((N + 127) / 128), (unsigned)BH);
-    launch_begin(kBwdTcPrep, stream);
     e = cudaMemsetAsync(mx, 0, (size_t)BH * 16, stream);
     if (e == cudaSuccess) e = cudaMemsetAsync(cm, 0, (size_t)BH * nch * 4, stream);
     if (e == cudaSuccess) {
+        launch_begin(kBwdTcR, stream);
         bwd_tc_r_kernel<DK, DV><<<rgrid, 128, 0, stream>>>(qb, kb, vb, dy, y, den, r, mx, N);
+        launch_end(kBwdTcR, stream);
         e = cudaGetLastError();
     }
     if (e == cudaSuccess) {
+        launch_begin(kBwdTcPrep, stream);
         bwd_tc_prep_kernel<DK, DV><<<rgrid, 128, 0, stream>>>(qb, kb, vb, r, mx, st_n, st_r, cm, im, N, nch, flags);
+        launch_end(kBwdTcPrep, stream);
         e = cudaGetLastError();
     }
-    launch_end(kBwdTcPrep, stream);
     if (e != cudaSuccess) return e;
     if ((e = cudaMemsetAsync(sq, 0, L.off_ur - L.off_sq, stream)) != cudaSuccess) return e;   // the three sums
 

@@ -28,7 +28,7 @@ const char *const kNames[kNumKernels] = {
     "decode_stream", "decode_finish", "simt_scan", "simt_finish",
     "tc_prep", "tc_scan", "tc_finish", "tc_reduce",
     "bwd_r", "bwd_q_scan", "bwd_kv_scan", "bwd_finish", "state_add", "bwd_tc_prep", "bwd_tc_scan",
-    "bwd_tc_finish",
+    "bwd_tc_finish", "tc_stats", "tc_state_stats", "bwd_tc_r",
 };
 
 void drain_locked() {

@@ -320,17 +320,20 @@ cudaError_t run(const DeviceBasis &basis, int BH, int64_t N, const void *q, cons
             const int bmax = (148 * 8 + BH - 1) / BH;
             if (bx > bmax) bx = bmax;
             if (bx < 1) bx = 1;
-            launch_begin(kTcPrep, ps);
+            launch_begin(kTcStats, ps);
             tc_stats_kernel<DK, DV><<<(unsigned)((int64_t)bx * BH), 256, 0, ps>>>(qb, kb, vb, stats, N, tok0, tok1, bx,
                                                                                 dvs);
-            if ((e = cudaGetLastError()) == cudaSuccess) {
+            launch_end(kTcStats, ps);
+            if ((e = cudaGetLastError()) != cudaSuccess) return e;
+            {
                 const int64_t nwork = (int64_t)BH * ntok;   // one thread per token row
                 const int pgrid = (int)((nwork + 255) / 256 < 148 * 16 ? (nwork + 255) / 256 : 148 * 16);
+                launch_begin(kTcPrep, ps);
                 tc_prep_kernel<DK, DV><<<pgrid, 256, 0, ps>>>(qb, kb, vb, stats, q16, k16, v16, BH, N, tok0, tok1,
                                                                pl.nchunks, flags, dvs, voff);
+                launch_end(kTcPrep, ps);
             }
-            launch_end(kTcPrep, ps);
-            if (e != cudaSuccess || (e = cudaGetLastError()) != cudaSuccess) return e;
+            if ((e = cudaGetLastError()) != cudaSuccess) return e;
             if (piped) {
                 cudaEvent_t ev;
                 if ((e = new_event(&ev)) || (e = cudaEventRecord(ev, ps)) || (e = cudaStreamWaitEvent(stream, ev, 0)))
@@ -339,7 +342,9 @@ cudaError_t run(const DeviceBasis &basis, int BH, int64_t N, const void *q, cons
             if (load_state) {
                 int ny = (148 * 8 + BH - 1) / BH;   // about eight blocks per SM over all heads
                 ny = ny < 8 ? 8 : (ny > 1024 ? 1024 : ny);
+                launch_begin(kTcStateStats, stream);
                 tc_state_stats_kernel<<<dim3(BH, ny), 256, 0, stream>>>(S, Z, stats, F, s_ld);
+                launch_end(kTcStateStats, stream);
                 if ((e = cudaGetLastError()) != cudaSuccess) return e;
             }
         }

@@ -67,7 +67,8 @@ const void *device_table(uint64_t key, size_t bytes, const std::function<void(ui
 // Kernel identities for launch statistics.
 enum KernelId {
     kDecodeStream = 0, kDecodeFinish, kSimtScan, kSimtFinish, kTcPrep, kTcScan, kTcFinish, kTcReduce,
-    kBwdR, kBwdQScan, kBwdKVScan, kBwdFinish, kStateAdd, kBwdTcPrep, kBwdTcScan, kBwdTcFinish, kNumKernels
+    kBwdR, kBwdQScan, kBwdKVScan, kBwdFinish, kStateAdd, kBwdTcPrep, kBwdTcScan, kBwdTcFinish, kTcStats,
+    kTcStateStats, kBwdTcR, kNumKernels
 };
 const char *kernel_name(int id);
 // Call around every kernel launch: begin() records a start event when timing is
