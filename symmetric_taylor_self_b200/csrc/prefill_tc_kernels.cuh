@@ -182,10 +182,12 @@ bool make_plan(int BH, int64_t N, int64_t F, int P, bool need_state, int min_seg
         // output are exposed, so those segments are short.  A segment's inputs copy in about
         // a third of its compute time and its output in about a quarter, so each segment can
         // be a few times its predecessor while its inputs still land in time, and the last a
-        // fraction of the one before it.  10 %, 20 %, 55 %, 15 % of the chunks measured best
-        // of the splits tried (uniform quarters: 4 % slower end to end at 65536 tokens).
+        // fraction of the one before it.  8 %, 18 %, 62 %, 12 % of the chunks measured best of
+        // the splits tried once the segments' own costs had come down (2.6 % faster end to end
+        // at 65536 tokens than 10/20/55/15, which had been best before; uniform quarters were
+        // 4 % slower than that).
         static_assert(kHostSegments == 4, "split profile");
-        const int cum[kHostSegments] = {0, 10, 30, 85};
+        const int cum[kHostSegments] = {0, 8, 26, 88};
         for (int i = 0; i < kHostSegments; ++i) pl.seg_c0[i] = (int)((int64_t)pl.nchunks * cum[i] / 100);
         pl.seg_c0[kHostSegments] = pl.nchunks;
         pl.profiled = true;
